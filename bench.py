@@ -1,0 +1,542 @@
+#!/usr/bin/env python3
+"""Benchmark of the FP32 NCHW conv2d forward library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload depthwise|tiny_grouped|fused_chain|dense_5x9]
+                    [--shapes] [--sweep]
+
+One step = one call of the library's entry point on one batch of the
+workload (default: the depthwise conv of a MobileNetV2 inverted-residual
+block, x[4,144,56,56], 3x3, s1, p1, groups=144).  Metric: algorithmic GB/s
+(x read once + w read once + y written once, per second), with GFLOP/s
+(2 x multiply-accumulates) and the roofline fraction alongside.
+
+Timing boundaries (the "GroupConv Atlas" distinguishes both):
+  value      device events around a CUDA graph holding exactly K captured
+             calls; inputs stay resident in HBM; consecutive calls rotate
+             through a pool of input/output buffers larger than 4 x L2, so no
+             call finds its data in L2.
+  e2e        per step: pinned-host -> device copy of the inputs, the call,
+             device -> pinned-host copy of the output, timed with events on
+             the same stream.
+  sync_api   host clock around one eager call + stream synchronize
+             (median over K calls).
+The oracle (FP64 CPU loop nest) is timed on the host cores as a reported
+baseline (`cpu_baseline`), and is what `--impl reference` times.
+
+Multi-GPU: every rank runs its own batch (the work shards along N with no
+exchange), time = max over ranks, value = all ranks' bytes / that time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from depthwise_convolution_fp32_b200 import inputs  # noqa: E402
+from depthwise_convolution_fp32_b200 import workloads as wl  # noqa: E402
+
+METRIC = "conv2d FP32 GB/s + GFLOP/s per shape, fraction of roofline (graph & sync timing)"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+PROFILES = os.path.join(ROOT, "profiles")
+
+
+# ------------------------------------------------------------------ helpers
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured", d
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback", {}
+
+
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources; a stored ncu traffic figure is only valid for
+    the sources it was captured from."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "depthwise_convolution_fp32_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".h", ".cuh")):
+            h.update(f.encode())
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(workload: str):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu
+    summary, or None when absent or captured from different sources."""
+    path = os.path.join(PROFILES, "traffic.json")
+    try:
+        d = json.load(open(path))
+        e = d[workload]
+        if e.get("source_hash") != kernel_source_hash():
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML on a background thread."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.samples = []
+        self.period = period_s
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self, t0=None, t1=None):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        win = [s for s in self.samples if (t0 is None or s[0] >= t0) and (t1 is None or s[0] <= t1)]
+        where = "timed"
+        if len(win) < 3:
+            win, where = self.samples, "warmup+timed"
+        reasons = set()
+        for _, _, rs in win:
+            for bit, name in self.REASONS.items():
+                if rs & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(m for _, m, _ in win), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(win), "window": where}
+
+
+# ------------------------------------------------------------------ workloads
+
+class Workload:
+    """A workload: seeded host inputs and a function that runs one step."""
+
+    def __init__(self, name: str):
+        self.name = name
+        if name == "depthwise":
+            s = wl.DEPTHWISE
+            self.shape = s
+            self.host = inputs.conv_inputs(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.groups,
+                                           wl.SEEDS["depthwise"], x_dist="normal", w_bound=1 / 3)
+        elif name == "tiny_grouped":
+            s = wl.TINY_GROUPED
+            self.shape = s
+            self.host = inputs.conv_inputs(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.groups,
+                                           wl.SEEDS["tiny_grouped"], x_dist="uniform11",
+                                           w_bound=1 / math.sqrt(18))
+        elif name == "dense_5x9":
+            s = wl.DENSE_5X9
+            self.shape = s
+            self.host = inputs.conv_inputs(s.N, s.C, s.H, s.W, s.K, s.R, s.S, 1,
+                                           wl.SEEDS["dense_5x9"], x_dist="uniform01",
+                                           w_bound=1 / math.sqrt(1440))
+        elif name == "fused_chain":
+            s = wl.FUSED_CHAIN.conv
+            self.shape = s
+            d = inputs.chain_inputs(s.N, s.C, s.H, s.W, s.K, s.R, s.S, 1, wl.FUSED_CHAIN.gn_groups,
+                                    seed=wl.SEEDS["fused_chain"])
+            self.host = d
+        elif name.startswith("sweep"):
+            i = int(name[5:])
+            s = wl.sweep80()[i]
+            self.shape = s
+            self.host = inputs.conv_inputs(s.N, s.C, s.H, s.W, s.K, 3, 3, s.groups, wl.sweep_seed(i),
+                                           x_dist="normal", w_bound=1 / math.sqrt(9 * s.cpg))
+        else:
+            raise ValueError(name)
+        self.chain = name == "fused_chain"
+
+    @property
+    def bytes(self) -> int:
+        return wl.FUSED_CHAIN.bytes if self.chain else self.shape.bytes
+
+    @property
+    def flops(self) -> int:
+        return self.shape.flops
+
+    @property
+    def kernels_per_step(self) -> int:
+        return 3 if self.chain else 1
+
+    def config(self):
+        s = self.shape
+        c = {"workload": self.name, "x": [s.N, s.C, s.H, s.W], "w": [s.K, s.cpg, s.R, s.S],
+             "y": [s.N, s.K, s.P, s.Q], "groups": s.groups, "stride": s.stride, "pad": s.pad,
+             "dilation": s.dil}
+        if self.chain:
+            c["gn_groups"] = wl.FUSED_CHAIN.gn_groups
+        return c
+
+
+class DeviceRunner:
+    """Device buffers (a rotating pool larger than L2) and the step call."""
+
+    def __init__(self, wk: Workload, device, l2_bytes: int):
+        import torch
+        import depthwise_convolution_fp32_b200 as gc
+        self.gc = gc
+        self.wk = wk
+        self.torch = torch
+        s = wk.shape
+        h = wk.host
+        self.w = h["w"].to(device)
+        self.K, self.P, self.Q = s.K, s.P, s.Q
+        per_set = (h["x"].numel() + s.n_out) * 4
+        # one set already larger than L2, or enough sets to cover 4 x L2
+        self.n_sets = 1 if per_set >= l2_bytes else math.ceil(4 * l2_bytes / per_set)
+        self.xs = []
+        self.ys = []
+        x0 = h["x"].to(device)
+        for i in range(self.n_sets):
+            self.xs.append(x0 if i == 0 else x0.clone())
+            self.ys.append(torch.empty((s.N, s.K, s.P, s.Q), device=device))
+        self.pool_bytes = self.n_sets * per_set
+        if wk.chain:
+            self.bias = (h["b_conv"] + h["b_extra"]).to(device)
+            self.scale = h["scale"].to(device)
+            self.gamma = h["gamma"].to(device)
+            self.beta = h["beta"].to(device)
+        else:
+            self.bias = h["bias"].to(device) if "bias" in h else None
+
+    def step(self, i: int, x=None, y=None):
+        s = self.wk.shape
+        x = self.xs[i % self.n_sets] if x is None else x
+        y = self.ys[i % self.n_sets] if y is None else y
+        if self.wk.chain:
+            self.gc.conv2d_bias_scale_sigmoid_groupnorm(
+                x, self.w, self.bias, self.scale, wl.FUSED_CHAIN.gn_groups, self.gamma, self.beta,
+                1e-5, s.stride, s.pad, s.dil, s.groups, out=y)
+        else:
+            self.gc.conv2d(x, self.w, self.bias, s.stride, s.pad, s.dil, s.groups, out=y)
+        return y
+
+
+def time_graph(runner: DeviceRunner, steps: int, warmup: int, dist_barrier):
+    """Capture exactly `steps` calls in one CUDA graph; time one replay."""
+    torch = runner.torch
+    for i in range(warmup):
+        runner.step(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(steps):
+                runner.step(i)
+    torch.cuda.synchronize()
+    g.replay()                      # untimed replay: graph upload
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    dist_barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        g.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    dist_barrier()
+    ms = ev0.elapsed_time(ev1)
+    del g
+    return ms, t0, t1
+
+
+def time_e2e(runner: DeviceRunner, steps: int, warmup: int, dist_barrier):
+    """Per step: pinned H2D copy of the inputs, the call, D2H of the output."""
+    torch = runner.torch
+    h = runner.wk.host
+    x_host = h["x"].pin_memory()
+    w_host = h["w"].pin_memory()
+    y_host = torch.empty(runner.ys[0].shape, dtype=torch.float32).pin_memory()
+    x_dev = runner.xs[0]
+    y_dev = runner.ys[0]
+    stream = torch.cuda.current_stream()
+
+    def one(i):
+        x_dev.copy_(x_host, non_blocking=True)
+        runner.w.copy_(w_host, non_blocking=True)
+        runner.step(i, x=x_dev, y=y_dev)
+        y_host.copy_(y_dev, non_blocking=True)
+
+    for i in range(warmup):
+        one(i)
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    dist_barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for i in range(steps):
+        one(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    dist_barrier()
+    ms = ev0.elapsed_time(ev1)
+    h2d = (x_host.numel() + w_host.numel()) * 4
+    d2h = y_host.numel() * 4
+    return ms, h2d, d2h
+
+
+def time_sync_api(runner: DeviceRunner, steps: int):
+    torch = runner.torch
+    lat = []
+    for i in range(steps):
+        t0 = time.perf_counter()
+        runner.step(i)
+        torch.cuda.current_stream().synchronize()
+        lat.append(time.perf_counter() - t0)
+    return statistics.median(lat) * 1e6
+
+
+def cpu_oracle_rate(wk: Workload, budget_s: float):
+    """Time the FP64 oracle, as it stands, on this host's cores on a bounded
+    sample of the workload; returns (GB/s, sample description, threads)."""
+    import oracle
+    s = wk.shape
+    h = wk.host
+    x = h["x"].numpy()
+    w = h["w"].numpy()
+    # sample: the first n_b batch items (whole images), grown until the budget
+    if wk.chain:
+        ch = wl.FUSED_CHAIN
+        pairs_all = [(n, G) for n in range(s.N) for G in range(ch.gn_groups)]
+        done = 0
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < budget_s and done < len(pairs_all):
+            nxt = pairs_all[done:done + 8]
+            oracle.chain(x, w, h["b_conv"], h["b_extra"], h["scale"], ch.gn_groups, h["gamma"],
+                         h["beta"], 1e-5, s.stride, s.pad, s.dil, s.groups, pairs=nxt)
+            done += len(nxt)
+        dt = time.perf_counter() - t0
+        frac = done / len(pairs_all)
+        desc = f"{done} of {len(pairs_all)} (n, GroupNorm group) blocks of the full workload"
+    else:
+        per_item = 1
+        t0 = time.perf_counter()
+        done = 0
+        passes = 0
+        while time.perf_counter() - t0 < budget_s:
+            n0 = done % s.N
+            n1 = min(s.N, n0 + per_item)
+            oracle.conv2d(x[n0:n1], w, h.get("bias"), s.stride, s.pad, s.dil, s.groups)
+            done += n1 - n0
+            passes += 1
+            if passes == 1 and time.perf_counter() - t0 < budget_s / 20:
+                per_item = min(s.N, per_item * 4)
+        dt = time.perf_counter() - t0
+        frac = done / s.N
+        desc = f"{done} batch items of N={s.N} (whole images, repeated as needed)"
+    gbs = wk.bytes * frac / dt / 1e9
+    return gbs, desc, oracle.num_threads()
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="depthwise")
+    ap.add_argument("--shapes", action="store_true", help="also time the other page workloads")
+    ap.add_argument("--sweep", action="store_true", help="also time the 80-shape sweep")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, rank)
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    from depthwise_convolution_fp32_b200 import build
+    build.build()
+    import depthwise_convolution_fp32_b200 as gc
+    gc.library()
+
+    props = torch.cuda.get_device_properties(device)
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
+    hbm_peak, peak_kind, _ = peaks()
+
+    wk = Workload(args.workload)
+    runner = DeviceRunner(wk, device, l2)
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        ms, t0, t1 = time_graph(runner, args.steps, args.warmup, barrier)
+        e2e_ms, h2d, d2h = time_e2e(runner, args.steps, args.warmup, barrier)
+        sync_us = time_sync_api(runner, min(args.steps, 200))
+    clocks = sampler.summary(t0, t1)
+
+    # max over ranks
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+
+    per_step_s = ms / 1e3 / args.steps
+    value = wk.bytes * world * args.steps / (ms / 1e3) / 1e9
+    e2e_value = wk.bytes * world * args.steps / (e2e_ms / 1e3) / 1e9
+    gflops = wk.flops * world * args.steps / (ms / 1e3) / 1e9
+
+    # dominant kernel: the conv kernel (the only one for a plain conv)
+    launch_s = per_step_s if not wk.chain else None
+    achieved = wk.bytes / launch_s / 1e9 if launch_s else None
+    roof = None
+    if achieved is not None:
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(achieved / hbm_peak, 4), "traffic": stored_traffic(wk.name),
+                "peak_kind": peak_kind, "kernel": gc.plan_name(
+                    wk.shape.N, wk.shape.C, wk.shape.H, wk.shape.W, wk.shape.K, wk.shape.R,
+                    wk.shape.S, wk.shape.stride, wk.shape.pad, wk.shape.dil, wk.shape.groups)}
+
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded)",
+        "config": dict(wk.config(), **{
+            "l2": f"rotating pool of {runner.n_sets} buffer sets, {runner.pool_bytes / 2**20:.0f} MiB "
+                  f"(L2 {l2 / 2**20:.0f} MiB)",
+            "timing": "CUDA graph of exactly K calls, device events",
+            "parallelism": f"replicas x{world} (batch shards, no collective)"}),
+        "gflops": round(gflops, 2),
+        "sync_api_us": round(sync_us, 2),
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "roofline": roof,
+        "gpu_launches": wk.kernels_per_step * args.steps,
+        "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        "clock_samples": {"n": clocks.get("samples"), "window": clocks.get("window")},
+    }
+
+    if args.shapes or args.sweep:
+        extra = {}
+        names = ["tiny_grouped", "depthwise", "fused_chain", "dense_5x9"] if args.shapes else []
+        if args.sweep:
+            names += [f"sweep{i}" for i in range(80)]
+        for nm in names:
+            if nm == args.workload:
+                continue
+            w2 = Workload(nm)
+            r2 = DeviceRunner(w2, device, l2)
+            k2 = max(3, min(args.steps, 50))
+            ms2, _, _ = time_graph(r2, k2, 3, barrier)
+            sec = ms2 / 1e3 / k2
+            extra[nm] = {"us": round(sec * 1e6, 3), "GB/s": round(w2.bytes / sec / 1e9, 1),
+                         "GFLOP/s": round(w2.flops / sec / 1e9, 1),
+                         "hbm_frac": round(w2.bytes / sec / 1e9 / hbm_peak, 4),
+                         "fp32_frac": round(w2.flops / sec / 1e12 / wl.fp32_fma_peak_tflops(), 4),
+                         "label": w2.shape.label()}
+            del r2
+            torch.cuda.empty_cache()
+        result["shapes"] = extra
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, desc, thr = cpu_oracle_rate(wk, args.cpu_budget)
+        result["cpu_baseline"] = {"value": round(gbs, 4), "unit": UNIT, "cores": thr,
+                                  "kind": "oracle", "sample": desc}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def run_reference(args, rank):
+    """The reference arm: the FP64 CPU oracle, as it stands, on this host."""
+    if rank != 0:
+        return
+    wk = Workload(args.workload)
+    budget = max(2.0, min(20.0, args.cpu_budget))
+    rates = []
+    for _ in range(args.warmup):
+        cpu_oracle_rate(wk, budget / 10)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        r, desc, thr = cpu_oracle_rate(wk, budget / max(1, args.steps))
+        rates.append(r)
+    wall = time.perf_counter() - t0
+    value = statistics.median(rates)
+    ms_per_step = wall * 1e3 / args.steps
+    result = {
+        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "impl": "reference", "config": wk.config(),
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": thr, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(result), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,429 @@
+// Direct grouped / depthwise / dense convolution on the FP32 CUDA cores, with
+// an optional fused epilogue (+bias, *scale, sigmoid, GroupNorm partial
+// statistics).
+//
+// What it computes ("GroupConv Atlas", "Fix the experiment"; POPCORNBENCH
+// "Kimi-K2.6__l1_p62", general index map in_y = out_y*stride - pad + kh*dil):
+//   y[n,k,p,q] = bias[k] + sum_{c,r,s} w[k,c,r,s] * x[n, gi*cpg + c,
+//                                         p*stride - pad + r*dil, q*stride - pad + s*dil]
+// with zero outside the image.
+//
+// Design (B200): the pages' kernels k2 (input tile + halo in shared memory)
+// and k3 (four horizontally adjacent outputs per thread) are combined and
+// extended:
+//  * a CTA owns a tile of TP output rows x TQ output columns x KBtot output
+//    channels; the input rows and columns that tile needs, for cchunk input
+//    channels at a time, are staged into shared memory with 16-byte
+//    cp.async copies whose source size is 0 outside the image, so the zero
+//    padding costs no instructions (4-byte copies when rows are not 16-byte
+//    aligned, e.g. W = 14);
+//  * every staged row is addressed in 16-byte chunks so the window one
+//    thread needs is read with 128-bit shared loads that are bank-conflict
+//    free across a quarter warp (the row pitch is padded so consecutive rows
+//    continue the chunk sequence modulo 8);
+//  * a thread keeps 4 adjacent outputs x RPT rows x KT output channels in
+//    registers: each input value read from shared memory feeds up to
+//    R*S*KT FMAs, each weight (a 128-bit broadcast load over KT channels)
+//    feeds RPT*4 FMAs;
+//  * the epilogue adds the bias, and for the chain applies *scale and the
+//    logistic function and reduces (count, mean, M2) per output channel and
+//    thread in registers (two-pass), then merges them per GroupNorm group in
+//    a fixed order (Chan's parallel-variance update), one partial per CTA and
+//    group, so no atomics are needed and results are deterministic.
+// A generic variant (all geometry at run time, inputs read straight from
+// global memory) serves every shape the specialised variants do not.
+#include "gconv_internal.h"
+
+namespace gconv {
+
+namespace {
+
+__device__ __forceinline__ void cp_async16(float *sdst, const float *gsrc, bool valid) {
+    unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(sdst));
+    int nbytes = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gsrc), "r"(nbytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async4(float *sdst, const float *gsrc, bool valid) {
+    unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(sdst));
+    int nbytes = valid ? 4 : 0;
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(s), "l"(gsrc), "r"(nbytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;\n" ::: "memory");
+}
+
+// Chan et al. pairwise update of (count, mean, M2) -- FP32, used inside a CTA.
+__device__ __forceinline__ void chan_merge(float &na, float &ma, float &m2a, float nb, float mb,
+                                           float m2b) {
+    if (nb == 0.f) return;
+    if (na == 0.f) {
+        na = nb; ma = mb; m2a = m2b;
+        return;
+    }
+    float n = na + nb;
+    float d = mb - ma;
+    float f = nb / n;
+    ma = fmaf(d, f, ma);
+    m2a = m2a + m2b + d * d * na * f;
+    na = n;
+}
+
+template <int KT>
+__device__ __forceinline__ void load_weights(float (&wv)[KT], const float *src) {
+    if constexpr (KT % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < KT / 4; ++i) {
+            float4 t = *reinterpret_cast<const float4 *>(src + 4 * i);
+            wv[4 * i] = t.x; wv[4 * i + 1] = t.y; wv[4 * i + 2] = t.z; wv[4 * i + 3] = t.w;
+        }
+    } else if constexpr (KT == 2) {
+        float2 t = *reinterpret_cast<const float2 *>(src);
+        wv[0] = t.x; wv[1] = t.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < KT; ++i) wv[i] = src[i];
+    }
+}
+
+template <int G> struct Geom;
+template <> struct Geom<kGeom3x3s1p1> { static constexpr int R = 3, S = 3, ST = 1, D = 1, PAD = 1; };
+template <> struct Geom<kGeom3x3s1p0> { static constexpr int R = 3, S = 3, ST = 1, D = 1, PAD = 0; };
+template <> struct Geom<kGeom3x3s2p1> { static constexpr int R = 3, S = 3, ST = 2, D = 1, PAD = 1; };
+template <> struct Geom<kGeom5x9s1p0> { static constexpr int R = 5, S = 9, ST = 1, D = 1, PAD = 0; };
+template <> struct Geom<kGeom1x1s1p0> { static constexpr int R = 1, S = 1, ST = 1, D = 1, PAD = 0; };
+template <> struct Geom<kDirectGeneric> { static constexpr int R = 0, S = 0, ST = 1, D = 1, PAD = 0; };
+
+constexpr int kV = 4;  // adjacent outputs per thread along q
+
+template <int G>
+struct Window {
+    using g = Geom<G>;
+    static constexpr bool FAST = g::R > 0;
+    static constexpr int HL = FAST ? (g::PAD + 3) / 4 : 0;       // halo chunks left of q0
+    static constexpr int OFF = FAST ? 4 * HL - g::PAD : 0;        // first needed float in chunk
+    static constexpr int WIN = FAST ? OFF + (kV - 1) * g::ST + (g::S - 1) * g::D + 1 : 4;
+    static constexpr int NCH = (WIN + 3) / 4;                     // chunks per row per thread
+};
+
+template <int G, int KT, int RPT, bool CHAIN>
+__global__ void __launch_bounds__(256, 2) direct_conv_kernel(const DirectParams p) {
+    extern __shared__ __align__(16) float smem[];
+    using g = Geom<G>;
+    using win = Window<G>;
+    constexpr bool FAST = win::FAST;
+    constexpr int IR = FAST ? (RPT - 1) * g::ST + (g::R - 1) * g::D + 1 : 1;
+
+    const int tid = threadIdx.x;
+    const int qt = blockIdx.x % p.n_qt;
+    const int pt = blockIdx.x / p.n_qt;
+    const int kb = blockIdx.y % p.n_kb;
+    const int gblk = blockIdx.y / p.n_kb;
+    const int n = blockIdx.z;
+    const int q0 = qt * p.TQ, p0 = pt * p.TP;
+    const int g0 = gblk * p.GB;
+    const int kc0 = g0 * p.kpg + kb * p.KB;   // first output channel of the CTA
+
+    int t = tid;
+    const int cx = t % p.CX; t /= p.CX;
+    const int ry = t % p.RY; t /= p.RY;
+    const int kz = t % p.KZ;
+    const int gb = t / p.KZ;
+    const bool active = gb < p.GB;
+    const int kl0 = gb * p.KB + kz * KT;       // local channel of kt = 0
+
+    const int Rr = FAST ? g::R : p.R;
+    const int Ss = FAST ? g::S : p.S;
+    const int RS = Rr * Ss;
+
+    float *sw = smem;                    // [cchunk][R][S][KBtot]
+    float *sx = smem + p.w_floats;       // [GB*cchunk][IHt][pitch]
+
+    float acc[RPT][kV][KT];
+#pragma unroll
+    for (int a = 0; a < RPT; ++a)
+#pragma unroll
+        for (int v = 0; v < kV; ++v)
+#pragma unroll
+            for (int k = 0; k < KT; ++k) acc[a][v][k] = 0.f;
+
+    const int ih0 = p0 * p.stride - p.pad;
+    const int iw0 = q0 * p.stride - 4 * win::HL;
+
+    for (int c0 = 0; c0 < p.cpg; c0 += p.cchunk) {
+        const int cc = min(p.cchunk, p.cpg - c0);
+        __syncthreads();   // the previous pass is done with shared memory
+        // weight slice, transposed to [c][r][s][channel] so KT channels are contiguous
+        const int nw = cc * RS * p.KBtot;
+        for (int e = tid; e < nw; e += blockDim.x) {
+            int kl = e % p.KBtot;
+            int rest = e / p.KBtot;
+            int c = rest / RS, rs = rest - c * RS;
+            sw[e] = __ldg(p.w + ((long long)(kc0 + kl) * p.cpg + c0 + c) * RS + rs);
+        }
+        if constexpr (FAST) {
+            const int planes = p.GB * cc;
+            if (p.vec_in) {
+                const int total = planes * p.IHt * p.PC;
+                for (int e = tid; e < total; e += blockDim.x) {
+                    int ch = e % p.PC;
+                    int rest = e / p.PC;
+                    int row = rest % p.IHt;
+                    int pl = rest / p.IHt;
+                    int gbb = pl / cc, c = pl - gbb * cc;
+                    int ci = (g0 + gbb) * p.cpg + c0 + c;
+                    int ih = ih0 + row, iw = iw0 + 4 * ch;
+                    bool ok = ih >= 0 && ih < p.H && iw >= 0 && iw < p.W;
+                    const float *src = ok ? p.x + (((long long)n * p.C + ci) * p.H + ih) * p.W + iw : p.x;
+                    cp_async16(sx + ((long long)pl * p.IHt + row) * p.pitch + 4 * ch, src, ok);
+                }
+            } else {
+                const int cols = 4 * p.PC;
+                const int total = planes * p.IHt * cols;
+                for (int e = tid; e < total; e += blockDim.x) {
+                    int j = e % cols;
+                    int rest = e / cols;
+                    int row = rest % p.IHt;
+                    int pl = rest / p.IHt;
+                    int gbb = pl / cc, c = pl - gbb * cc;
+                    int ci = (g0 + gbb) * p.cpg + c0 + c;
+                    int ih = ih0 + row, iw = iw0 + j;
+                    bool ok = ih >= 0 && ih < p.H && iw >= 0 && iw < p.W;
+                    const float *src = ok ? p.x + (((long long)n * p.C + ci) * p.H + ih) * p.W + iw : p.x;
+                    cp_async4(sx + ((long long)pl * p.IHt + row) * p.pitch + j, src, ok);
+                }
+            }
+            cp_async_wait_all();
+        }
+        __syncthreads();
+        if (!active) continue;
+
+        if constexpr (FAST) {
+            for (int c = 0; c < cc; ++c) {
+                const float *xs = sx + ((long long)(gb * cc + c) * p.IHt + ry * RPT * g::ST) * p.pitch +
+                                  cx * g::ST * 4;
+                const float *ws = sw + c * RS * p.KBtot + kl0;
+                float xr[IR][win::NCH * 4];
+#pragma unroll
+                for (int ir = 0; ir < IR; ++ir)
+#pragma unroll
+                    for (int ch = 0; ch < win::NCH; ++ch) {
+                        float4 v4 = *reinterpret_cast<const float4 *>(xs + ir * p.pitch + ch * 4);
+                        xr[ir][4 * ch] = v4.x; xr[ir][4 * ch + 1] = v4.y;
+                        xr[ir][4 * ch + 2] = v4.z; xr[ir][4 * ch + 3] = v4.w;
+                    }
+#pragma unroll
+                for (int r = 0; r < g::R; ++r)
+#pragma unroll
+                    for (int s = 0; s < g::S; ++s) {
+                        float wv[KT];
+                        load_weights<KT>(wv, ws + (r * g::S + s) * p.KBtot);
+#pragma unroll
+                        for (int rp = 0; rp < RPT; ++rp)
+#pragma unroll
+                            for (int v = 0; v < kV; ++v) {
+                                const float xv = xr[rp * g::ST + r * g::D][win::OFF + v * g::ST + s * g::D];
+#pragma unroll
+                                for (int k = 0; k < KT; ++k) acc[rp][v][k] = fmaf(wv[k], xv, acc[rp][v][k]);
+                            }
+                    }
+            }
+        } else {
+            // generic geometry: read x straight from global memory (L1/L2 serve the reuse)
+#pragma unroll
+            for (int rp = 0; rp < RPT; ++rp) {
+                const int pp = p0 + ry * RPT + rp;
+#pragma unroll
+                for (int v = 0; v < kV; ++v) {
+                    const int qq = q0 + cx * kV + v;
+                    if (pp >= p.P || qq >= p.Q) continue;
+                    for (int c = 0; c < cc; ++c) {
+                        const int ci = (g0 + gb) * p.cpg + c0 + c;
+                        const float *xp = p.x + ((long long)n * p.C + ci) * p.H * (long long)p.W;
+                        const float *ws = sw + c * RS * p.KBtot + kl0;
+                        for (int r = 0; r < Rr; ++r) {
+                            const int ih = pp * p.stride - p.pad + r * p.dil;
+                            if (ih < 0 || ih >= p.H) continue;
+                            for (int s = 0; s < Ss; ++s) {
+                                const int iw = qq * p.stride - p.pad + s * p.dil;
+                                if (iw < 0 || iw >= p.W) continue;
+                                const float xv = __ldg(xp + (long long)ih * p.W + iw);
+                                const float *wr = ws + (r * Ss + s) * p.KBtot;
+#pragma unroll
+                                for (int k = 0; k < KT; ++k) acc[rp][v][k] = fmaf(wr[k], xv, acc[rp][v][k]);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- epilogue
+    const int qb = q0 + cx * kV;
+    if (active) {
+#pragma unroll
+        for (int k = 0; k < KT; ++k) {
+            const int kk = kc0 + kl0 + k;
+            const float b = p.bias ? __ldg(p.bias + kk) : 0.f;
+            float sc = 1.f;
+            if constexpr (CHAIN) sc = __ldg(p.scale + kk);
+#pragma unroll
+            for (int rp = 0; rp < RPT; ++rp)
+#pragma unroll
+                for (int v = 0; v < kV; ++v) {
+                    float z = acc[rp][v][k] + b;
+                    if constexpr (CHAIN) z = 1.f / (1.f + expf(-(z * sc)));
+                    acc[rp][v][k] = z;
+                }
+        }
+#pragma unroll
+        for (int rp = 0; rp < RPT; ++rp) {
+            const int pp = p0 + ry * RPT + rp;
+            if (pp >= p.P) continue;
+#pragma unroll
+            for (int k = 0; k < KT; ++k) {
+                const int kk = kc0 + kl0 + k;
+                float *yr = p.y + (((long long)n * p.K + kk) * p.P + pp) * (long long)p.Q;
+                if (p.vec_out && qb + kV <= p.Q) {
+                    *reinterpret_cast<float4 *>(yr + qb) =
+                        make_float4(acc[rp][0][k], acc[rp][1][k], acc[rp][2][k], acc[rp][3][k]);
+                } else {
+#pragma unroll
+                    for (int v = 0; v < kV; ++v)
+                        if (qb + v < p.Q) yr[qb + v] = acc[rp][v][k];
+                }
+            }
+        }
+    }
+
+    if constexpr (CHAIN) {
+        // per-thread, per-channel (count, mean, M2) over the thread's valid outputs
+        __syncthreads();   // shared memory is reused for the statistics
+        const int nsp = p.CX * p.RY;
+        float *st_n = smem;
+        float *st_m = smem + p.KBtot * nsp;
+        float *st_q = smem + 2 * p.KBtot * nsp;
+        if (active) {
+            float cnt = 0.f;
+#pragma unroll
+            for (int rp = 0; rp < RPT; ++rp)
+#pragma unroll
+                for (int v = 0; v < kV; ++v)
+                    if (p0 + ry * RPT + rp < p.P && qb + v < p.Q) cnt += 1.f;
+            const int sp = ry * p.CX + cx;
+#pragma unroll
+            for (int k = 0; k < KT; ++k) {
+                float sum = 0.f;
+#pragma unroll
+                for (int rp = 0; rp < RPT; ++rp)
+#pragma unroll
+                    for (int v = 0; v < kV; ++v)
+                        if (p0 + ry * RPT + rp < p.P && qb + v < p.Q) sum += acc[rp][v][k];
+                const float mean = cnt > 0.f ? sum / cnt : 0.f;
+                float m2 = 0.f;
+#pragma unroll
+                for (int rp = 0; rp < RPT; ++rp)
+#pragma unroll
+                    for (int v = 0; v < kV; ++v)
+                        if (p0 + ry * RPT + rp < p.P && qb + v < p.Q) {
+                            float d = acc[rp][v][k] - mean;
+                            m2 = fmaf(d, d, m2);
+                        }
+                const int e = (kl0 + k) * nsp + sp;
+                st_n[e] = cnt; st_m[e] = mean; st_q[e] = m2;
+            }
+        }
+        __syncthreads();
+        // one partial per (CTA, GroupNorm group), merged in a fixed order
+        const int per = min(p.KBtot, p.kgn);         // CTA channels per GN group
+        const int ngc = p.KBtot / per;               // GN groups this CTA touches
+        const int lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+        for (int j = warp; j < ngc; j += nwarps) {
+            float cn = 0.f, mn = 0.f, m2 = 0.f;
+            const int entries = per * nsp;
+            for (int e = lane; e < entries; e += 32) {
+                const int idx = (j * per + e / nsp) * nsp + (e % nsp);
+                chan_merge(cn, mn, m2, st_n[idx], st_m[idx], st_q[idx]);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                float on = __shfl_down_sync(0xffffffffu, cn, off);
+                float om = __shfl_down_sync(0xffffffffu, mn, off);
+                float oq = __shfl_down_sync(0xffffffffu, m2, off);
+                if (lane < off) chan_merge(cn, mn, m2, on, om, oq);
+            }
+            if (lane == 0) {
+                const int kfirst = kc0 + j * per;
+                const int gn_g = kfirst / p.kgn;
+                const int kcb = (p.KBtot < p.kgn) ? (kfirst % p.kgn) / p.KBtot : 0;
+                const int slot = kcb * p.n_sp + blockIdx.x;
+                p.gn_part[((long long)n * p.gn_groups + gn_g) * p.slots + slot] = make_float4(cn, mn, m2, 0.f);
+            }
+        }
+    }
+}
+
+template <int G, int KT, bool CHAIN>
+cudaError_t launch_one(const DirectParams &p, dim3 grid, int threads, size_t smem, cudaStream_t st) {
+    constexpr int RPT = (KT >= 4) ? 2 : 4;
+    auto kern = direct_conv_kernel<G, KT, RPT, CHAIN>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<grid, threads, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <int G, bool CHAIN>
+cudaError_t launch_kt(const DirectParams &p, int KT, dim3 grid, int threads, size_t smem, cudaStream_t st) {
+    switch (KT) {
+        case 1: return launch_one<G, 1, CHAIN>(p, grid, threads, smem, st);
+        case 2: return launch_one<G, 2, CHAIN>(p, grid, threads, smem, st);
+        case 4: return launch_one<G, 4, CHAIN>(p, grid, threads, smem, st);
+        case 8: return launch_one<G, 8, CHAIN>(p, grid, threads, smem, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <bool CHAIN>
+cudaError_t launch_geom(const DirectParams &p, int geom, int KT, dim3 grid, int threads, size_t smem,
+                        cudaStream_t st) {
+    switch (geom) {
+        case kGeom3x3s1p1: return launch_kt<kGeom3x3s1p1, CHAIN>(p, KT, grid, threads, smem, st);
+        case kGeom3x3s1p0: return launch_kt<kGeom3x3s1p0, CHAIN>(p, KT, grid, threads, smem, st);
+        case kGeom3x3s2p1: return launch_kt<kGeom3x3s2p1, CHAIN>(p, KT, grid, threads, smem, st);
+        case kGeom5x9s1p0: return launch_kt<kGeom5x9s1p0, CHAIN>(p, KT, grid, threads, smem, st);
+        case kGeom1x1s1p0: return launch_kt<kGeom1x1s1p0, CHAIN>(p, KT, grid, threads, smem, st);
+        case kDirectGeneric: return launch_kt<kDirectGeneric, CHAIN>(p, KT, grid, threads, smem, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+int direct_rpt(int KT) { return KT >= 4 ? 2 : 4; }
+
+int direct_fast_window_chunks(int geom) {
+    switch (geom) {
+        case kGeom3x3s1p1: return Window<kGeom3x3s1p1>::NCH;
+        case kGeom3x3s1p0: return Window<kGeom3x3s1p0>::NCH;
+        case kGeom3x3s2p1: return Window<kGeom3x3s2p1>::NCH;
+        case kGeom5x9s1p0: return Window<kGeom5x9s1p0>::NCH;
+        case kGeom1x1s1p0: return Window<kGeom1x1s1p0>::NCH;
+        default: return 0;
+    }
+}
+
+cudaError_t launch_direct(const DirectParams &p, int geom, int KT, int chain, dim3 grid, int threads,
+                          size_t smem, cudaStream_t stream) {
+    return chain ? launch_geom<true>(p, geom, KT, grid, threads, smem, stream)
+                 : launch_geom<false>(p, geom, KT, grid, threads, smem, stream);
+}
+
+}  // namespace gconv

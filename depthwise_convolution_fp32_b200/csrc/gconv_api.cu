@@ -1,0 +1,378 @@
+// C ABI of libgconv.so (declared in include/gconv.h): argument validation,
+// geometry, per-shape kernel planning, the GroupNorm workspace, and the two
+// entry points of the FP32 NCHW conv2d forward and the fused
+// conv -> bias -> scale -> sigmoid -> GroupNorm chain.
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "gconv.h"
+#include "gconv_internal.h"
+
+using namespace gconv;
+
+namespace {
+
+constexpr int kMaxThreads = 256;
+constexpr size_t kSmemBudget = 100 * 1024;   // keep two CTAs per SM where possible
+constexpr size_t kSmemMax = 227 * 1024;
+
+enum ForceMode : int { kForceAuto = 0, kForceDirect = 1, kForceGeneric = 2 };
+std::atomic<int> g_force{kForceAuto};
+
+struct Shape {
+    int N, C, H, W, K, R, S, stride, pad, dil, groups;
+    int cpg, kpg, P, Q;
+};
+
+long long out_extent(long long in, long long k, long long s, long long p, long long d) {
+    long long span = in + 2 * p - d * (k - 1) - 1;
+    if (span < 0) return 0;
+    return span / s + 1;
+}
+
+gconv_status_t make_shape(Shape &s, int N, int C, int H, int W, int K, int R, int S, int stride, int pad,
+                          int dil, int groups) {
+    if (N < 1 || C < 1 || H < 1 || W < 1 || K < 1 || R < 1 || S < 1) return GCONV_ERR_INVALID_ARG;
+    if (stride < 1 || pad < 0 || dil < 1 || groups < 1) return GCONV_ERR_INVALID_ARG;
+    if (C % groups != 0 || K % groups != 0) return GCONV_ERR_INVALID_ARG;
+    long long P = out_extent(H, R, stride, pad, dil);
+    long long Q = out_extent(W, S, stride, pad, dil);
+    if (P < 1 || Q < 1 || P > 0x7fffffff || Q > 0x7fffffff) return GCONV_ERR_INVALID_ARG;
+    // index arithmetic: per-plane offsets fit in int64 comfortably; keep the
+    // element counts below 2^62 and the staged-tile arithmetic in int
+    if ((long long)N * C * H * W >= (1LL << 62) || (long long)N * K * P * Q >= (1LL << 62))
+        return GCONV_ERR_INVALID_ARG;
+    if ((long long)H * W >= (1LL << 31) || P * Q >= (1LL << 31)) return GCONV_ERR_UNSUPPORTED;
+    s = {N, C, H, W, K, R, S, stride, pad, dil, groups, C / groups, K / groups, (int)P, (int)Q};
+    return GCONV_OK;
+}
+
+int match_geom(const Shape &s) {
+    if (s.dil != 1) return kDirectGeneric;
+    if (s.R == 3 && s.S == 3 && s.stride == 1 && s.pad == 1) return kGeom3x3s1p1;
+    if (s.R == 3 && s.S == 3 && s.stride == 1 && s.pad == 0) return kGeom3x3s1p0;
+    if (s.R == 3 && s.S == 3 && s.stride == 2 && s.pad == 1) return kGeom3x3s2p1;
+    if (s.R == 5 && s.S == 9 && s.stride == 1 && s.pad == 0) return kGeom5x9s1p0;
+    if (s.R == 1 && s.S == 1 && s.stride == 1 && s.pad == 0) return kGeom1x1s1p0;
+    return kDirectGeneric;
+}
+
+const char *geom_name(int geom) {
+    switch (geom) {
+        case kGeom3x3s1p1: return "direct_3x3s1p1";
+        case kGeom3x3s1p0: return "direct_3x3s1p0";
+        case kGeom3x3s2p1: return "direct_3x3s2p1";
+        case kGeom5x9s1p0: return "direct_5x9s1p0";
+        case kGeom1x1s1p0: return "direct_1x1s1p0";
+        default: return "direct_generic";
+    }
+}
+
+bool compat(int a, int b) { return a % b == 0 || b % a == 0; }
+
+int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// A complete launch plan for the direct kernel.
+struct DirectPlan {
+    DirectParams prm;
+    int geom, KT;
+    dim3 grid;
+    int threads;
+    size_t smem;
+};
+
+// Choose the CTA tile for a direct-kernel launch.  Returns false when no tile
+// fits the shared-memory limit (the shape is then unsupported by this family).
+bool plan_direct(const Shape &s, bool chain, int gn_groups, int geom, DirectPlan &pl) {
+    const bool fast = geom != kDirectGeneric;
+    const int kgn = chain ? s.K / gn_groups : 1;
+    DirectParams &p = pl.prm;
+    std::memset(&p, 0, sizeof(p));
+
+    // channels per thread: largest of 8,4,2,1 dividing kpg (and, for the chain,
+    // nesting with the GroupNorm group width)
+    int KT = 1;
+    if (fast) {
+        for (int c : {8, 4, 2, 1})
+            if (s.kpg % c == 0 && (!chain || compat(kgn, c))) { KT = c; break; }
+    }
+    const int RPT = fast ? direct_rpt(KT) : direct_rpt(1);
+    if (!fast) KT = 1;
+
+    const int qchunks = ceil_div(s.Q, 4);
+    int n_qt = ceil_div(qchunks, 32);
+    int CX = ceil_div(qchunks, n_qt);
+
+    // channel slices per CTA
+    const int m = s.kpg / KT;
+    int KZ = 1;
+    for (int z = 1; z <= m; ++z)
+        if (m % z == 0 && KT * z <= 32 && CX * z <= kMaxThreads && (!chain || compat(kgn, KT * z))) KZ = z;
+    const int KB = KT * KZ;
+    const int n_kb = s.kpg / KB;
+
+    const int strips = ceil_div(s.P, RPT);
+    int ry_max = kMaxThreads / (CX * KZ);
+    if (ry_max < 1) ry_max = 1;
+    int n_pt = ceil_div(strips, ry_max);
+    int RY = ceil_div(strips, n_pt);
+    const int TP = RY * RPT;
+
+    // conv groups per CTA (only when a CTA already holds all channels of a group)
+    int GB = 1;
+    if (n_kb == 1) {
+        const int per = CX * RY * KZ;
+        for (int gcand = 1; gcand <= s.groups; ++gcand) {
+            if (s.groups % gcand) continue;
+            if (per * gcand > kMaxThreads) break;
+            if (chain && !compat(kgn, gcand * s.kpg)) continue;
+            GB = gcand;
+        }
+    }
+    const int KBtot = GB * KB;
+    if (chain && !compat(kgn, KBtot)) return false;
+
+    const int RS = s.R * s.S;
+    int IHt = 0, PC = 0, pitch = 0;
+    if (fast) {
+        IHt = (TP - 1) * s.stride + (s.R - 1) * s.dil + 1;
+        PC = (CX - 1) * s.stride + direct_fast_window_chunks(geom);
+        int pcp = PC;
+        while (((pcp - CX * s.stride) % 8 + 8) % 8 != 0) ++pcp;
+        pitch = 4 * pcp;
+    }
+    auto smem_for = [&](int cc) -> size_t {
+        size_t wf = ((size_t)cc * RS * KBtot + 3) / 4 * 4;
+        size_t xf = fast ? (size_t)GB * cc * IHt * pitch : 0;
+        return (wf + xf) * sizeof(float);
+    };
+    int cchunk = s.cpg;
+    while (cchunk > 1 && smem_for(cchunk) > kSmemBudget) cchunk = (cchunk + 1) / 2;
+    size_t smem = smem_for(cchunk);
+    const int nsp = CX * RY;
+    if (chain) {
+        size_t st = (size_t)3 * KBtot * nsp * sizeof(float);
+        if (st > smem) smem = st;
+    }
+    if (smem > kSmemMax) return false;
+
+    p.N = s.N; p.C = s.C; p.H = s.H; p.W = s.W; p.K = s.K; p.R = s.R; p.S = s.S;
+    p.stride = s.stride; p.pad = s.pad; p.dil = s.dil; p.groups = s.groups;
+    p.cpg = s.cpg; p.kpg = s.kpg; p.P = s.P; p.Q = s.Q;
+    p.CX = CX; p.RY = RY; p.KZ = KZ; p.GB = GB;
+    p.TP = TP; p.TQ = 4 * CX; p.KB = KB; p.KBtot = KBtot;
+    p.n_qt = n_qt; p.n_pt = n_pt; p.n_kb = n_kb;
+    p.IHt = IHt; p.PC = PC; p.pitch = pitch; p.cchunk = cchunk;
+    p.w_floats = (int)(((size_t)cchunk * RS * KBtot + 3) / 4 * 4);
+    p.gn_groups = chain ? gn_groups : 0;
+    p.kgn = kgn;
+    p.n_sp = n_qt * n_pt;
+    p.slots_k = (chain && KBtot < kgn) ? kgn / KBtot : 1;
+    p.slots = p.slots_k * p.n_sp;
+
+    const long long gy = (long long)n_kb * (s.groups / GB);
+    const long long gx = (long long)n_qt * n_pt;
+    if (gx > 0x7fffffffLL || gy > 65535 || s.N > 65535) return false;
+    pl.grid = dim3((unsigned)gx, (unsigned)gy, (unsigned)s.N);
+    pl.threads = (CX * RY * KZ * GB + 31) / 32 * 32;
+    pl.smem = smem;
+    pl.geom = geom;
+    pl.KT = KT;
+    return true;
+}
+
+// Direct-kernel plan for the current forcing mode.
+bool choose_direct(const Shape &s, bool chain, int gn_groups, DirectPlan &pl) {
+    const int force = g_force.load(std::memory_order_relaxed);
+    int geom = (force == kForceGeneric) ? (int)kDirectGeneric : match_geom(s);
+    if (plan_direct(s, chain, gn_groups, geom, pl)) return true;
+    if (geom != kDirectGeneric && force == kForceAuto) return plan_direct(s, chain, gn_groups, kDirectGeneric, pl);
+    return false;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ----------------------------------------------------------------- workspace
+struct Workspace {
+    void *ptr = nullptr;
+    size_t bytes = 0;
+};
+constexpr int kMaxDevices = 64;
+Workspace g_ws[kMaxDevices];
+std::mutex g_ws_mutex;
+
+gconv_status_t ensure_workspace(size_t bytes, cudaStream_t stream, void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GCONV_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return GCONV_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_ws_mutex);
+    Workspace &ws = g_ws[dev];
+    if (ws.bytes >= bytes && ws.ptr) {
+        *out = ws.ptr;
+        return GCONV_OK;
+    }
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return GCONV_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return GCONV_ERR_WORKSPACE;
+    size_t want = bytes < (1u << 20) ? (1u << 20) : bytes;
+    if (ws.ptr) {
+        if (cudaFree(ws.ptr) != cudaSuccess) return GCONV_ERR_CUDA;   // synchronises the device
+        ws.ptr = nullptr;
+        ws.bytes = 0;
+    }
+    void *p = nullptr;
+    if (cudaMalloc(&p, want) != cudaSuccess) {
+        cudaGetLastError();
+        return GCONV_ERR_WORKSPACE;
+    }
+    ws.ptr = p;
+    ws.bytes = want;
+    *out = p;
+    return GCONV_OK;
+}
+
+size_t chain_ws_bytes(const DirectParams &p) {
+    size_t part = (size_t)p.N * p.gn_groups * p.slots * sizeof(float4);
+    size_t stats = (size_t)p.N * p.gn_groups * sizeof(float2);
+    return (part + 255) / 256 * 256 + stats;
+}
+
+gconv_status_t validate_ptrs(const float *x, const float *w, const float *y) {
+    if (!x || !w || !y) return GCONV_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(y)) & 3u)
+        return GCONV_ERR_INVALID_ARG;
+    return GCONV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *gconv_status_string(gconv_status_t status) {
+    switch (status) {
+        case GCONV_OK: return "GCONV_OK";
+        case GCONV_ERR_INVALID_ARG: return "GCONV_ERR_INVALID_ARG: invalid size, pointer or parameter";
+        case GCONV_ERR_UNSUPPORTED: return "GCONV_ERR_UNSUPPORTED: valid shape that no kernel implements";
+        case GCONV_ERR_CUDA: return "GCONV_ERR_CUDA: the CUDA runtime reported an error";
+        case GCONV_ERR_WORKSPACE: return "GCONV_ERR_WORKSPACE: workspace too small and cannot grow now";
+        case GCONV_ERR_TIMEOUT: return "GCONV_ERR_TIMEOUT: a bounded device wait gave up";
+    }
+    return "unknown gconv status";
+}
+
+const char *gconv_version(void) { return "gconv-b200 0.1.0 (sm_100a)"; }
+
+gconv_status_t gconv2d_output_size(int H, int W, int R, int S, int stride, int pad, int dilation, int *P,
+                                   int *Q) {
+    if (!P || !Q) return GCONV_ERR_INVALID_ARG;
+    Shape s;
+    gconv_status_t st = make_shape(s, 1, 1, H, W, 1, R, S, stride, pad, dilation, 1);
+    if (st == GCONV_ERR_UNSUPPORTED) st = GCONV_OK;   // extents are still defined
+    if (st != GCONV_OK) return st;
+    *P = (int)out_extent(H, R, stride, pad, dilation);
+    *Q = (int)out_extent(W, S, stride, pad, dilation);
+    return GCONV_OK;
+}
+
+gconv_status_t gconv_force_kernel(const char *name) {
+    if (!name) return GCONV_ERR_INVALID_ARG;
+    if (!std::strcmp(name, "auto")) g_force = kForceAuto;
+    else if (!std::strcmp(name, "direct")) g_force = kForceDirect;
+    else if (!std::strcmp(name, "generic")) g_force = kForceGeneric;
+    else return GCONV_ERR_INVALID_ARG;
+    return GCONV_OK;
+}
+
+const char *gconv2d_plan_name(int N, int C, int H, int W, int K, int R, int S, int stride, int pad,
+                              int dilation, int groups, int chain) {
+    Shape s;
+    gconv_status_t st = make_shape(s, N, C, H, W, K, R, S, stride, pad, dilation, groups);
+    if (st == GCONV_ERR_INVALID_ARG) return "invalid";
+    if (st != GCONV_OK) return "unsupported";
+    DirectPlan pl;
+    int gn = 1;
+    if (!choose_direct(s, chain != 0, gn, pl)) return "unsupported";
+    return geom_name(pl.geom);
+}
+
+gconv_status_t gconv2d_fwd(const float *x, const float *w, const float *bias, int N, int C, int H, int W, int K,
+                           int R, int S, int stride, int pad, int dilation, int groups, float *y,
+                           cudaStream_t stream) {
+    Shape s;
+    gconv_status_t st = make_shape(s, N, C, H, W, K, R, S, stride, pad, dilation, groups);
+    if (st != GCONV_OK) return st;
+    if ((st = validate_ptrs(x, w, y)) != GCONV_OK) return st;
+    if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) return GCONV_ERR_INVALID_ARG;
+    DirectPlan pl;
+    if (!choose_direct(s, false, 1, pl)) return GCONV_ERR_UNSUPPORTED;
+    DirectParams &p = pl.prm;
+    p.x = x; p.w = w; p.bias = bias; p.y = y;
+    p.vec_in = (s.W % 4 == 0) && aligned16(x);
+    p.vec_out = (s.Q % 4 == 0) && aligned16(y);
+    if (launch_direct(p, pl.geom, pl.KT, 0, pl.grid, pl.threads, pl.smem, stream) != cudaSuccess)
+        return GCONV_ERR_CUDA;
+    return GCONV_OK;
+}
+
+size_t gconv2d_chain_workspace_size(int N, int C, int H, int W, int K, int R, int S, int stride, int pad,
+                                    int dilation, int groups, int gn_groups) {
+    Shape s;
+    if (make_shape(s, N, C, H, W, K, R, S, stride, pad, dilation, groups) != GCONV_OK) return 0;
+    if (gn_groups < 1 || K % gn_groups) return 0;
+    DirectPlan pl;
+    if (!choose_direct(s, true, gn_groups, pl)) return 0;
+    return chain_ws_bytes(pl.prm);
+}
+
+gconv_status_t gconv_reserve_workspace(size_t bytes) {
+    void *p = nullptr;
+    return ensure_workspace(bytes, nullptr, &p);
+}
+
+gconv_status_t gconv2d_bias_scale_sigmoid_groupnorm_fwd(const float *x, const float *w, const float *bias, int N,
+                                                        int C, int H, int W, int K, int R, int S, int stride,
+                                                        int pad, int dilation, int groups, const float *scale,
+                                                        int gn_groups, const float *gamma, const float *beta,
+                                                        float eps, float *y, cudaStream_t stream) {
+    Shape s;
+    gconv_status_t st = make_shape(s, N, C, H, W, K, R, S, stride, pad, dilation, groups);
+    if (st != GCONV_OK) return st;
+    if ((st = validate_ptrs(x, w, y)) != GCONV_OK) return st;
+    if (!scale || !gamma || !beta) return GCONV_ERR_INVALID_ARG;
+    if (gn_groups < 1 || K % gn_groups != 0) return GCONV_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || eps != eps) return GCONV_ERR_INVALID_ARG;
+    for (const void *q : {(const void *)bias, (const void *)scale, (const void *)gamma, (const void *)beta})
+        if (q && (reinterpret_cast<uintptr_t>(q) & 3u)) return GCONV_ERR_INVALID_ARG;
+    DirectPlan pl;
+    if (!choose_direct(s, true, gn_groups, pl)) return GCONV_ERR_UNSUPPORTED;
+    DirectParams &p = pl.prm;
+    void *ws = nullptr;
+    const size_t part_bytes = ((size_t)p.N * p.gn_groups * p.slots * sizeof(float4) + 255) / 256 * 256;
+    if ((st = ensure_workspace(chain_ws_bytes(p), stream, &ws)) != GCONV_OK) return st;
+    p.x = x; p.w = w; p.bias = bias; p.y = y; p.scale = scale;
+    p.gn_part = reinterpret_cast<float4 *>(ws);
+    p.vec_in = (s.W % 4 == 0) && aligned16(x);
+    p.vec_out = (s.Q % 4 == 0) && aligned16(y);
+    if (launch_direct(p, pl.geom, pl.KT, 1, pl.grid, pl.threads, pl.smem, stream) != cudaSuccess)
+        return GCONV_ERR_CUDA;
+
+    GnParams g;
+    g.y = y;
+    g.gn_part = p.gn_part;
+    g.stats = reinterpret_cast<float2 *>(reinterpret_cast<char *>(ws) + part_bytes);
+    g.gamma = gamma; g.beta = beta;
+    g.N = s.N; g.K = s.K; g.gn_groups = gn_groups; g.kgn = s.K / gn_groups; g.slots = p.slots;
+    g.PQ = (long long)s.P * s.Q;
+    g.eps = eps;
+    g.vec = (g.PQ % 4 == 0) && aligned16(y);
+    const long long per_cta = g.vec ? 4LL * 256 * 8 : 256LL * 8;
+    g.chunks = (int)((g.PQ + per_cta - 1) / per_cta);
+    if (g.chunks < 1) g.chunks = 1;
+    if (launch_gn_finalize(g, stream) != cudaSuccess) return GCONV_ERR_CUDA;
+    if (launch_gn_normalize(g, stream) != cudaSuccess) return GCONV_ERR_CUDA;
+    return GCONV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,73 @@
+// Internal declarations shared by the host dispatcher and the kernels of
+// libgconv.so.  Not part of the public ABI (include/gconv.h is).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gconv {
+
+// Compile-time geometry a fast direct-kernel variant is specialised for.
+// The generic variant (id kDirectGeneric) takes every size at run time.
+enum DirectVariantGeom : int {
+    kGeom3x3s1p1 = 0,   // 3x3, stride 1, pad 1, dilation 1 (Atlas sweep, depthwise)
+    kGeom3x3s1p0 = 1,   // 3x3, stride 1, pad 0, dilation 1 (fused-chain conv)
+    kGeom3x3s2p1 = 2,   // 3x3, stride 2, pad 1, dilation 1 (downsampling depthwise)
+    kGeom5x9s1p0 = 3,   // 5x9, stride 1, pad 0, dilation 1 (dense asymmetric conv)
+    kGeom1x1s1p0 = 4,   // pointwise
+    kGeomCount = 5,
+    kDirectGeneric = 99
+};
+
+// Everything one launch of the direct kernel needs.  The host fills it; the
+// kernel derives its tile from blockIdx / threadIdx.
+struct DirectParams {
+    const float *x, *w, *bias;  // inputs (bias may be null)
+    float *y;                   // output [N,K,P,Q]
+    const float *scale;         // chain only: [K]
+    float4 *gn_part;            // chain only: [N*gn_groups][slots] (count, mean, M2, 0)
+
+    int N, C, H, W, K, R, S, stride, pad, dil, groups;
+    int cpg, kpg, P, Q;
+
+    // CTA tile: CX chunk-columns of 4 outputs, RY row strips of RPT rows,
+    // KZ channel slices of KT channels, GB conv groups.
+    int CX, RY, KZ, GB;
+    int TP, TQ;       // output rows / cols per CTA
+    int KB;           // output channels per CTA inside one conv group (KZ*KT)
+    int KBtot;        // channels per CTA (GB*KB; GB > 1 only when KB == kpg)
+    int n_qt, n_pt, n_kb;
+    int IHt;          // staged input rows per plane
+    int PC;           // staged 16-byte chunks per row
+    int pitch;        // floats per staged row (>= 4*PC)
+    int cchunk;       // input channels staged per pass
+    int w_floats;     // floats reserved for the weight slice (multiple of 4)
+    int vec_in;       // x rows are 16-byte aligned (16-byte cp.async staging)
+    int vec_out;      // y rows are 16-byte aligned (float4 stores)
+
+    // chain bookkeeping
+    int gn_groups, kgn, slots, slots_k, n_sp;
+};
+
+struct GnParams {
+    float *y;
+    const float4 *gn_part;
+    float2 *stats;    // [N*gn_groups] (mean, rstd)
+    const float *gamma, *beta;
+    int N, K, gn_groups, kgn, slots;
+    long long PQ;
+    float eps;
+    int chunks;       // CTAs per channel plane in the normalise pass
+    int vec;          // float4 path allowed
+};
+
+// Launch one direct-kernel variant; returns cudaGetLastError() of the launch.
+cudaError_t launch_direct(const DirectParams &p, int geom, int KT, int chain,
+                          dim3 grid, int threads, size_t smem, cudaStream_t stream);
+int direct_rpt(int KT);   // rows per thread the variant with KT uses
+int direct_fast_window_chunks(int geom);   // 16-byte chunks one thread reads per row
+
+cudaError_t launch_gn_finalize(const GnParams &p, cudaStream_t stream);
+cudaError_t launch_gn_normalize(const GnParams &p, cudaStream_t stream);
+
+}  // namespace gconv

@@ -1,0 +1,115 @@
+// GroupNorm statistics merge and normalisation for the fused chain
+// (POPCORNBENCH "Kimi-K2.6__l2_p21", Model forward: GroupNorm with
+// population variance, eps inside the square root, affine weight/bias):
+//   mu  = mean(a) over the K/gn_groups channels of group G and all P*Q
+//   var = mean((a - mu)^2)
+//   y   = (a - mu) / sqrt(var + eps) * gamma[k] + beta[k]
+//
+// The conv kernel leaves one (count, mean, M2) partial per CTA and group.
+// gn_finalize merges a group's partials in double precision with Chan's
+// update, in slot order through a fixed binary tree, so the statistics are
+// deterministic and free of the E[a^2] - mu^2 cancellation the transcript's
+// kernels use (a sits near 0.5 after the logistic function while var can be
+// ~1e-6).  gn_normalize then streams y once (read + write, float4 when rows
+// are 16-byte aligned), one channel plane slice per CTA.
+#include "gconv_internal.h"
+
+namespace gconv {
+
+namespace {
+
+__device__ __forceinline__ void chan_merge64(double &na, double &ma, double &m2a, double nb, double mb,
+                                             double m2b) {
+    if (nb == 0.0) return;
+    if (na == 0.0) {
+        na = nb; ma = mb; m2a = m2b;
+        return;
+    }
+    double n = na + nb;
+    double d = mb - ma;
+    double f = nb / n;
+    ma += d * f;
+    m2a += m2b + d * d * na * f;
+    na = n;
+}
+
+constexpr int kFinThreads = 128;
+
+__global__ void __launch_bounds__(kFinThreads) gn_finalize_kernel(const GnParams p) {
+    __shared__ double sn[kFinThreads], sm[kFinThreads], sq[kFinThreads];
+    const int ng = blockIdx.x;
+    const int tid = threadIdx.x;
+    double cn = 0.0, mn = 0.0, m2 = 0.0;
+    const float4 *part = p.gn_part + (long long)ng * p.slots;
+    for (int i = tid; i < p.slots; i += kFinThreads) {
+        float4 v = part[i];
+        chan_merge64(cn, mn, m2, (double)v.x, (double)v.y, (double)v.z);
+    }
+    sn[tid] = cn; sm[tid] = mn; sq[tid] = m2;
+    __syncthreads();
+    for (int h = kFinThreads / 2; h > 0; h >>= 1) {
+        if (tid < h) {
+            double a = sn[tid], b = sm[tid], c = sq[tid];
+            chan_merge64(a, b, c, sn[tid + h], sm[tid + h], sq[tid + h]);
+            sn[tid] = a; sm[tid] = b; sq[tid] = c;
+        }
+        __syncthreads();
+    }
+    if (tid == 0) {
+        double var = sn[0] > 0.0 ? sq[0] / sn[0] : 0.0;
+        double rstd = 1.0 / sqrt(var + (double)p.eps);
+        p.stats[ng] = make_float2((float)sm[0], (float)rstd);
+    }
+}
+
+constexpr int kNormThreads = 256;
+
+__global__ void __launch_bounds__(kNormThreads) gn_normalize_kernel(const GnParams p) {
+    const long long plane = blockIdx.x / p.chunks;        // n*K + k
+    const int chunk = blockIdx.x % p.chunks;
+    const int k = (int)(plane % p.K);
+    const int n = (int)(plane / p.K);
+    const int G = k / p.kgn;
+    const float2 st = p.stats[(long long)n * p.gn_groups + G];
+    const float mean = st.x;
+    const float mul = (float)((double)st.y * (double)__ldg(p.gamma + k));
+    const float add = __ldg(p.beta + k);
+    float *yp = p.y + plane * p.PQ;
+    if (p.vec) {
+        const long long nv = p.PQ / 4;
+        const long long per = (nv + p.chunks - 1) / p.chunks;
+        const long long beg = chunk * per;
+        const long long end = min(nv, beg + per);
+        float4 *y4 = reinterpret_cast<float4 *>(yp);
+        for (long long i = beg + threadIdx.x; i < end; i += kNormThreads) {
+            float4 v = y4[i];
+            v.x = fmaf(v.x - mean, mul, add);
+            v.y = fmaf(v.y - mean, mul, add);
+            v.z = fmaf(v.z - mean, mul, add);
+            v.w = fmaf(v.w - mean, mul, add);
+            y4[i] = v;
+        }
+    } else {
+        const long long per = (p.PQ + p.chunks - 1) / p.chunks;
+        const long long beg = chunk * per;
+        const long long end = min(p.PQ, beg + per);
+        for (long long i = beg + threadIdx.x; i < end; i += kNormThreads)
+            yp[i] = fmaf(yp[i] - mean, mul, add);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_gn_finalize(const GnParams &p, cudaStream_t stream) {
+    gn_finalize_kernel<<<p.N * p.gn_groups, kFinThreads, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gn_normalize(const GnParams &p, cudaStream_t stream) {
+    long long blocks = (long long)p.N * p.K * p.chunks;
+    if (blocks <= 0 || blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    gn_normalize_kernel<<<(unsigned)blocks, kNormThreads, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace gconv

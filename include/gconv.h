@@ -1,0 +1,141 @@
+/*
+ * gconv.h -- C ABI of libgconv.so: FP32 contiguous-NCHW 2D convolution forward
+ * (grouped, depthwise, dense, asymmetric kernels) and the fused
+ * conv -> +bias -> *scale -> sigmoid -> GroupNorm chain, on NVIDIA B200
+ * (sm_100a).
+ *
+ * Sources for the operations (web pages on the subject):
+ *  - "GroupConv Atlas" (xiangguozhang.com/projects/groupconv-atlas), section
+ *    "Fix the experiment": FP32, contiguous NCHW grouped convolution with
+ *    general geometry (the direct-mapping kernel "supports general convolution
+ *    geometry").
+ *  - POPCORNBENCH "Kimi-K2.6__l2_p21" transcript: the Model
+ *    Conv2d(8->32, 3x3) -> x + bias[K,1,1] -> x * scale[K,1,1] -> sigmoid ->
+ *    GroupNorm(8 groups, eps 1e-5, affine weight/bias), and the final design's
+ *    folding of the conv bias and the extra bias into one per-channel vector.
+ *  - POPCORNBENCH "Kimi-K2.6__l1_p62" transcript: the asymmetric Conv2d with a
+ *    (5, 9) kernel, the output size (H + 2p - d(R-1) - 1)/s + 1 and the index
+ *    map in_y = out_y*stride - pad + kh*dilation.
+ *
+ * Conventions shared by every entry point:
+ *  - Tensors are FP32, contiguous, row-major: x[N][C][H][W], w[K][C/groups][R][S],
+ *    y[N][K][P][Q].  Offsets are computed in 64-bit.  Pointers need only
+ *    4-byte alignment; 16-byte alignment enables the vector paths.
+ *  - x, w, bias, scale, gamma, beta and y are DEVICE pointers owned by the
+ *    caller.  The library never frees or retains them.
+ *  - The operation is a cross-correlation (no kernel flip): output channel k
+ *    belongs to group k / (K/groups) and reads input channels
+ *    [gi*C/groups, (gi+1)*C/groups); taps outside the image read zero.
+ *  - Stride, padding and dilation are the same along H and W; the kernel may
+ *    be non-square (R != S).
+ *  - Every call is asynchronous on `stream` (0 = legacy default stream).  It
+ *    performs no host synchronisation and no device allocation, except the
+ *    one-time workspace allocation described at gconv_reserve_workspace.
+ *  - Errors: arguments are validated on the host first; on any error nothing
+ *    is launched and y is untouched.  A launch failure reported by the CUDA
+ *    runtime returns GCONV_ERR_CUDA.  Shapes that are valid but outside what
+ *    the kernels implement return GCONV_ERR_UNSUPPORTED (never a fallback).
+ *  - y must not overlap x, w or any parameter vector.
+ */
+#ifndef GCONV_H_
+#define GCONV_H_
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define GCONV_API __attribute__((visibility("default")))
+#else
+#define GCONV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gconv_status {
+    GCONV_OK = 0,
+    GCONV_ERR_INVALID_ARG = 1,   /* a size, pointer or parameter is invalid */
+    GCONV_ERR_UNSUPPORTED = 2,   /* valid shape that no kernel implements */
+    GCONV_ERR_CUDA = 3,          /* the CUDA runtime reported an error */
+    GCONV_ERR_WORKSPACE = 4,     /* workspace too small and cannot grow now */
+    GCONV_ERR_TIMEOUT = 5        /* reserved: a bounded device wait gave up */
+} gconv_status_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+GCONV_API const char *gconv_status_string(gconv_status_t status);
+
+/* Output extents P, Q of a convolution: P = floor((H + 2*pad - dilation*(R-1) - 1)/stride) + 1
+ * and likewise Q from W and S ("Kimi-K2.6__l1_p62", output-size formula).
+ * Returns GCONV_ERR_INVALID_ARG when an argument is out of range or the
+ * kernel does not fit (P or Q < 1).  P and Q are host pointers. */
+GCONV_API gconv_status_t gconv2d_output_size(int H, int W, int R, int S, int stride, int pad,
+                                   int dilation, int *P, int *Q);
+
+/* Grouped / depthwise / dense convolution forward:
+ *   y[n,k,p,q] = bias[k] + sum_{c<C/g, r<R, s<S} w[k,c,r,s] * x[n, gi*C/g + c,
+ *                                    p*stride - pad + r*dilation, q*stride - pad + s*dilation]
+ * ("GroupConv Atlas", "Fix the experiment"; "Kimi-K2.6__l1_p62", index map).
+ * bias: [K] device pointer or NULL for none.
+ * Requires N >= 1, C, K, R, S, stride, dilation >= 1, pad >= 0,
+ * groups >= 1 dividing C and K, P, Q >= 1, and every tensor smaller than
+ * 2^31 elements per sample plane product (N*C*H*W, N*K*P*Q < 2^62). */
+GCONV_API gconv_status_t gconv2d_fwd(const float *x, const float *w, const float *bias,
+                           int N, int C, int H, int W, int K, int R, int S,
+                           int stride, int pad, int dilation, int groups,
+                           float *y, cudaStream_t stream);
+
+/* Fused chain ("Kimi-K2.6__l2_p21", Model forward):
+ *   z = conv(x, w) + bias[k]          (bias [K] or NULL; the caller folds the
+ *                                       conv bias and the extra [K,1,1] bias)
+ *   a = 1 / (1 + exp(-(z * scale[k])))
+ *   per (n, G) with G < gn_groups, over channels [G*K/gn_groups, (G+1)*K/gn_groups)
+ *   and all P*Q positions: mu = mean(a), var = mean((a - mu)^2)
+ *   y = (a - mu) / sqrt(var + eps) * gamma[k] + beta[k]
+ * scale, gamma, beta: [K] device pointers (required).  gn_groups must divide K;
+ * eps >= 0.  y receives the result (it also holds a between the two passes).
+ * GroupNorm statistics are merged deterministically (fixed order), so equal
+ * inputs give bit-identical outputs.
+ * Scratch: per-tile partial statistics live in a library-owned workspace on
+ * the current device (see gconv_reserve_workspace).  Calls on different
+ * streams that overlap on the GPU share that workspace and must not run
+ * concurrently. */
+GCONV_API gconv_status_t gconv2d_bias_scale_sigmoid_groupnorm_fwd(
+    const float *x, const float *w, const float *bias,
+    int N, int C, int H, int W, int K, int R, int S,
+    int stride, int pad, int dilation, int groups,
+    const float *scale, int gn_groups, const float *gamma, const float *beta,
+    float eps, float *y, cudaStream_t stream);
+
+/* Bytes of workspace the fused chain needs for this shape (0 on invalid input). */
+GCONV_API size_t gconv2d_chain_workspace_size(int N, int C, int H, int W, int K, int R, int S,
+                                    int stride, int pad, int dilation, int groups,
+                                    int gn_groups);
+
+/* Make sure the current device's workspace holds at least `bytes`.  The chain
+ * grows the workspace on demand (cudaMalloc) the first time a shape needs more;
+ * growing is impossible while `stream` capture is active, in which case the
+ * chain returns GCONV_ERR_WORKSPACE.  Call this (or one un-captured chain call)
+ * before capturing a CUDA graph.  The workspace lives until process exit. */
+GCONV_API gconv_status_t gconv_reserve_workspace(size_t bytes);
+
+/* Name of the kernel variant the dispatcher selects for a convolution shape
+ * (for records and A/B measurements); "unsupported" / "invalid" otherwise.
+ * `chain` != 0 asks about the fused chain's conv stage. */
+GCONV_API const char *gconv2d_plan_name(int N, int C, int H, int W, int K, int R, int S,
+                              int stride, int pad, int dilation, int groups, int chain);
+
+/* Force a kernel family for subsequent calls on this process, by name
+ * ("auto" restores per-shape dispatch).  A forced family that cannot run a
+ * shape makes that call return GCONV_ERR_UNSUPPORTED.  Returns
+ * GCONV_ERR_INVALID_ARG for an unknown name.  Intended for measurement. */
+GCONV_API gconv_status_t gconv_force_kernel(const char *name);
+
+/* Library version string. */
+GCONV_API const char *gconv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GCONV_H_ */

@@ -1,0 +1,318 @@
+"""GPU parity: every kernel path against the FP64 oracle on the same seeded
+inputs, element by element, through the C ABI (via the ctypes binding).
+
+Small and medium shapes are compared in full; the full-size workloads are
+compared on sampled outputs the oracle computes one by one (and whole
+GroupNorm groups for the chain).  Output buffers are NaN-prefilled and
+surrounded by canary guards, so a missed store or a stray one fails."""
+import math
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import depthwise_convolution_fp32_b200 as gc
+from depthwise_convolution_fp32_b200 import build, inputs
+from depthwise_convolution_fp32_b200 import workloads as wl
+
+from tolerance import assert_chain_close, assert_conv_close
+
+pytestmark = pytest.mark.gpu
+
+CANARY = 1234.5678
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build.build()
+    gc.library()
+    gc.force_kernel("auto")
+    yield
+    gc.force_kernel("auto")
+
+
+class Guarded:
+    """A NaN-prefilled output with canary regions on both sides; `misalign`
+    shifts the output start by that many floats (4-byte aligned only)."""
+
+    def __init__(self, shape, guard=1024, misalign=0):
+        self.n = int(np.prod(shape))
+        self.g = guard + misalign
+        self.buf = torch.full((self.n + 2 * guard + misalign,), CANARY, device="cuda")
+        self.buf[self.g:self.g + self.n] = float("nan")
+        self.y = self.buf[self.g:self.g + self.n].view(*shape)
+
+    def check(self):
+        lo = self.buf[:self.g]
+        hi = self.buf[self.g + self.n:]
+        assert bool((lo == CANARY).all()) and bool((hi == CANARY).all()), "write outside y"
+
+
+def _to_dev(t, misalign=0):
+    if misalign == 0:
+        return t.cuda()
+    buf = torch.empty(t.numel() + misalign, device="cuda")
+    v = buf[misalign:misalign + t.numel()].view(t.shape)
+    v.copy_(t)
+    return v
+
+
+def run_conv(d, stride, pad, dil, groups, misalign=0):
+    x = _to_dev(d["x"], misalign)
+    w = d["w"].cuda()
+    b = d["bias"].cuda() if "bias" in d else None
+    N, C, H, W = d["x"].shape
+    K, _, R, S = d["w"].shape
+    P, Q = gc.output_size(H, W, R, S, stride, pad, dil)
+    out = Guarded((N, K, P, Q), misalign=misalign)
+    gc.conv2d(x, w, b, stride, pad, dil, groups, out=out.y)
+    torch.cuda.synchronize()
+    out.check()
+    return out.y
+
+
+def full_check(oracle_mod, d, stride, pad, dil, groups, what, misalign=0):
+    y = run_conv(d, stride, pad, dil, groups, misalign).cpu().numpy()
+    ref, acc = oracle_mod.conv2d(d["x"], d["w"], d.get("bias"), stride, pad, dil, groups,
+                                 return_absacc=True)
+    return assert_conv_close(y, ref, acc, what)
+
+
+def sampled_idx(shape, n_random, seed):
+    """Random flat indices plus every border position of a few output planes."""
+    N, K, P, Q = shape
+    rng = np.random.default_rng(seed)
+    idx = set(rng.integers(0, N * K * P * Q, n_random).tolist())
+    for (n, k) in [(0, 0), (N - 1, K - 1), (N // 2, K // 2)]:
+        base = (n * K + k) * P * Q
+        for p in range(P):
+            for q in (0, 1, Q - 2, Q - 1):
+                if 0 <= q < Q:
+                    idx.add(base + p * Q + q)
+        for q in range(Q):
+            for p in (0, P - 1):
+                idx.add(base + p * Q + q)
+    return np.array(sorted(idx), dtype=np.int64)
+
+
+def sampled_check(oracle_mod, d, y_dev, stride, pad, dil, groups, what, n_random=4000, seed=0):
+    idx = sampled_idx(tuple(y_dev.shape), n_random, seed)
+    got = y_dev.reshape(-1)[torch.from_numpy(idx).cuda()].cpu().numpy()
+    ref, acc = oracle_mod.conv2d_at(d["x"], d["w"], idx, d.get("bias"), stride, pad, dil, groups)
+    return assert_conv_close(got, ref, acc, what)
+
+
+# ------------------------------------------------------------------ workloads
+
+def test_tiny_grouped_full(oracle_mod):
+    s = wl.TINY_GROUPED
+    d = inputs.conv_inputs(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.groups, wl.SEEDS["tiny_grouped"],
+                           x_dist="uniform11", w_bound=1 / math.sqrt(18))
+    full_check(oracle_mod, d, 1, 1, 1, s.groups, "tiny grouped")
+
+
+def test_depthwise_mobilenet_full(oracle_mod):
+    s = wl.DEPTHWISE
+    d = inputs.conv_inputs(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.groups, wl.SEEDS["depthwise"],
+                           x_dist="normal", w_bound=1 / 3)
+    full_check(oracle_mod, d, 1, 1, 1, s.groups, "depthwise 4x144x56x56")
+
+
+@pytest.mark.parametrize("i", range(80))
+def test_sweep80(oracle_mod, i):
+    s = wl.sweep80()[i]
+    d = inputs.conv_inputs(s.N, s.C, s.H, s.W, s.K, 3, 3, s.groups, wl.sweep_seed(i),
+                           x_dist="normal", w_bound=1 / math.sqrt(9 * s.cpg))
+    if s.macs <= 4e8:
+        full_check(oracle_mod, d, 1, 1, 1, s.groups, s.label())
+    else:
+        y = run_conv(d, 1, 1, 1, s.groups)
+        sampled_check(oracle_mod, d, y, 1, 1, 1, s.groups, s.label(), seed=i)
+
+
+def test_dense_5x9_full_size_sampled(oracle_mod):
+    s = wl.DENSE_5X9
+    d = inputs.conv_inputs(s.N, s.C, s.H, s.W, s.K, s.R, s.S, 1, wl.SEEDS["dense_5x9"],
+                           x_dist="uniform01", w_bound=1 / math.sqrt(1440))
+    y = run_conv(d, 1, 0, 1, 1)
+    assert tuple(y.shape) == (8, 64, 508, 504)
+    sampled_check(oracle_mod, d, y, 1, 0, 1, 1, "dense 5x9 full size", n_random=3000)
+
+
+def test_dense_5x9_small_full(oracle_mod):
+    d = inputs.conv_inputs(1, 32, 37, 70, 64, 5, 9, 1, 77, x_dist="uniform01",
+                           w_bound=1 / math.sqrt(1440))
+    full_check(oracle_mod, d, 1, 0, 1, 1, "dense 5x9 ragged")
+
+
+# ------------------------------------------------------------------ geometry
+
+GEOMS = [
+    # N, C, H, W, K, R, S, stride, pad, dil, groups, bias
+    (2, 16, 14, 14, 16, 3, 3, 1, 1, 1, 16, False),   # W=14: 4-byte staging path
+    (1, 32, 28, 28, 32, 3, 3, 1, 1, 1, 8, True),
+    (3, 12, 17, 23, 12, 3, 3, 1, 1, 1, 12, True),     # odd sizes, ragged tiles
+    (2, 8, 33, 130, 8, 3, 3, 1, 1, 1, 8, False),     # Q > 128: two column tiles
+    (1, 16, 56, 56, 32, 3, 3, 1, 1, 1, 16, False),   # channel multiplier 2
+    (2, 24, 20, 20, 48, 3, 3, 1, 1, 1, 3, True),     # cpg 8, kpg 16
+    (1, 8, 29, 31, 8, 3, 3, 2, 1, 1, 8, False),      # stride 2 depthwise
+    (2, 16, 56, 56, 16, 3, 3, 2, 1, 1, 16, True),
+    (1, 8, 19, 21, 16, 3, 3, 1, 0, 1, 1, True),      # pad 0 dense
+    (1, 16, 12, 40, 16, 1, 1, 1, 0, 1, 4, True),     # pointwise grouped
+    (1, 8, 15, 15, 8, 3, 3, 1, 2, 2, 8, False),      # dilation 2 (generic)
+    (2, 6, 11, 13, 9, 5, 3, 1, 2, 1, 3, True),       # R != S (generic)
+    (1, 4, 9, 9, 8, 7, 7, 1, 3, 1, 2, False),        # 7x7 (generic)
+    (1, 6, 10, 12, 6, 3, 3, 3, 1, 1, 6, False),      # stride 3 (generic)
+    (1, 4, 1, 17, 4, 1, 3, 1, 0, 1, 4, False),       # H = 1
+    (1, 4, 5, 1, 4, 3, 1, 1, 1, 1, 2, False),        # W = 1
+    (1, 3, 3, 3, 5, 3, 3, 1, 0, 1, 1, True),         # P = Q = 1
+    (1, 8, 6, 6, 8, 3, 3, 1, 4, 1, 8, False),        # padding larger than the halo chunk
+    (1, 64, 9, 9, 64, 3, 3, 1, 1, 1, 1, False),      # dense 3x3, cpg 64 (channel chunks)
+    (1, 96, 7, 8, 12, 5, 9, 1, 0, 1, 1, False),      # dense 5x9 with many channels
+]
+
+
+@pytest.mark.parametrize("geo", GEOMS, ids=lambda g: "x".join(map(str, g[:11])))
+def test_geometry_full(oracle_mod, geo):
+    N, C, H, W, K, R, S, st, pad, dil, g, bias = geo
+    d = inputs.conv_inputs(N, C, H, W, K, R, S, g, seed=zlib.crc32(repr(geo).encode()) % 10000, x_dist="normal",
+                           bias=bias)
+    full_check(oracle_mod, d, st, pad, dil, g, str(geo))
+
+
+@pytest.mark.parametrize("geo", GEOMS[:10], ids=lambda g: "x".join(map(str, g[:11])))
+def test_forced_generic_matches_oracle(oracle_mod, geo):
+    N, C, H, W, K, R, S, st, pad, dil, g, bias = geo
+    d = inputs.conv_inputs(N, C, H, W, K, R, S, g, seed=7 + zlib.crc32(repr(geo).encode()) % 1000, x_dist="normal",
+                           bias=bias)
+    gc.force_kernel("generic")
+    try:
+        full_check(oracle_mod, d, st, pad, dil, g, "generic " + str(geo))
+    finally:
+        gc.force_kernel("auto")
+
+
+@pytest.mark.parametrize("mis", [1, 2, 3])
+def test_misaligned_pointers(oracle_mod, mis):
+    d = inputs.conv_inputs(2, 16, 28, 28, 16, 3, 3, 16, seed=40 + mis, x_dist="normal", bias=True)
+    full_check(oracle_mod, d, 1, 1, 1, 16, f"misaligned by {mis}", misalign=mis)
+
+
+def test_bias_null_equals_zero_bias():
+    d = inputs.conv_inputs(2, 8, 20, 20, 8, 3, 3, 8, seed=50)
+    x, w = d["x"].cuda(), d["w"].cuda()
+    y0 = gc.conv2d(x, w, None, 1, 1, 1, 8)
+    yz = gc.conv2d(x, w, torch.zeros(8, device="cuda"), 1, 1, 1, 8)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, yz)
+
+
+def test_delta_kernel_is_exact_identity():
+    d = inputs.conv_inputs(2, 32, 56, 56, 32, 3, 3, 32, seed=51)
+    w = torch.zeros(32, 1, 3, 3)
+    w[:, 0, 1, 1] = 1.0
+    y = gc.conv2d(d["x"].cuda(), w.cuda(), None, 1, 1, 1, 32)
+    torch.cuda.synchronize()
+    assert torch.equal(y.cpu(), d["x"])
+
+
+def test_stream_ordering():
+    """The call runs on torch's current stream (a side stream here)."""
+    d = inputs.conv_inputs(4, 64, 56, 56, 64, 3, 3, 64, seed=52)
+    s = torch.cuda.Stream()
+    x = d["x"].cuda()
+    w = d["w"].cuda()
+    ref = gc.conv2d(x, w, None, 1, 1, 1, 64)
+    with torch.cuda.stream(s):
+        x2 = x * 1.0
+        y = gc.conv2d(x2, w, None, 1, 1, 1, 64)
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref)
+
+
+# ------------------------------------------------------------------ fused chain
+
+def _chain_dev(d, stride, pad, dil, groups, eps):
+    x = d["x"].cuda()
+    w = d["w"].cuda()
+    bias = (d["b_conv"] + d["b_extra"]).cuda()
+    N, C, H, W = d["x"].shape
+    K, _, R, S = d["w"].shape
+    P, Q = gc.output_size(H, W, R, S, stride, pad, dil)
+    out = Guarded((N, K, P, Q))
+    gc.conv2d_bias_scale_sigmoid_groupnorm(x, w, bias, d["scale"].cuda(), d["gn_groups"],
+                                           d["gamma"].cuda(), d["beta"].cuda(), eps, stride, pad,
+                                           dil, groups, out=out.y)
+    torch.cuda.synchronize()
+    out.check()
+    return out.y
+
+
+def _chain_ref(oracle_mod, d, stride, pad, dil, groups, eps, pairs=None):
+    return oracle_mod.chain(d["x"], d["w"], d["b_conv"], d["b_extra"], d["scale"], d["gn_groups"],
+                            d["gamma"], d["beta"], eps, stride, pad, dil, groups, pairs)
+
+
+CHAINS = [
+    # N, C, H, W, K, R, S, stride, pad, dil, groups, gn_groups, bias/scale std, affine
+    (2, 8, 40, 40, 32, 3, 3, 1, 0, 1, 1, 8, 0.02, "identity"),   # the workload's geometry, small
+    (2, 8, 40, 40, 32, 3, 3, 1, 0, 1, 1, 8, 1.0, "random"),      # stressed statistics
+    (3, 8, 37, 45, 32, 3, 3, 1, 0, 1, 1, 8, 1.0, "random"),      # ragged tiles
+    (2, 8, 24, 24, 32, 3, 3, 1, 0, 1, 1, 2, 1.0, "random"),      # 16 channels per GN group
+    (2, 8, 24, 24, 32, 3, 3, 1, 0, 1, 1, 32, 1.0, "random"),     # 1 channel per GN group
+    (2, 16, 30, 30, 16, 3, 3, 1, 1, 1, 16, 4, 1.0, "random"),    # depthwise conv in the chain
+    (2, 12, 21, 19, 24, 3, 3, 1, 1, 1, 3, 6, 1.0, "random"),     # grouped conv, GN crosses groups
+    (1, 8, 17, 17, 24, 3, 3, 2, 1, 1, 1, 3, 1.0, "random"),      # stride 2
+    (1, 6, 15, 16, 12, 5, 3, 1, 1, 1, 2, 4, 1.0, "random"),      # generic geometry
+    (2, 8, 40, 40, 32, 3, 3, 1, 0, 1, 1, 8, 3.0, "random"),      # saturating logistic
+]
+
+
+@pytest.mark.parametrize("cfg", CHAINS, ids=lambda c: "x".join(map(str, c[:12])) + f"_{c[12]}")
+def test_chain_full(oracle_mod, cfg):
+    N, C, H, W, K, R, S, st, pad, dil, g, gn, std, affine = cfg
+    d = inputs.chain_inputs(N, C, H, W, K, R, S, g, gn, seed=60 + zlib.crc32(repr(cfg).encode()) % 1000,
+                            bias_scale_std=std, affine=affine)
+    eps = 1e-5
+    y = _chain_dev(d, st, pad, dil, g, eps).cpu().numpy()
+    ref = _chain_ref(oracle_mod, d, st, pad, dil, g, eps)
+    assert_chain_close(y, ref, d["scale"].numpy(), d["gamma"].numpy(), eps, K // gn, str(cfg))
+
+
+def test_chain_workload_full_size_sampled_groups(oracle_mod):
+    ch = wl.FUSED_CHAIN
+    s = ch.conv
+    d = inputs.chain_inputs(s.N, s.C, s.H, s.W, s.K, s.R, s.S, 1, ch.gn_groups,
+                            seed=wl.SEEDS["fused_chain"])
+    eps = 1e-5
+    y = _chain_dev(d, 1, 0, 1, 1, eps)
+    assert tuple(y.shape) == (128, 32, 254, 254)
+    kgn = s.K // ch.gn_groups
+    pairs = [(0, 0), (127, 7), (64, 3), (5, 6)]
+    ref = _chain_ref(oracle_mod, d, 1, 0, 1, 1, eps, pairs=pairs)
+    got = np.stack([y[n, G * kgn:(G + 1) * kgn].cpu().numpy() for n, G in pairs])
+    sc = np.stack([d["scale"].numpy()[G * kgn:(G + 1) * kgn] for _, G in pairs])
+    ga = np.stack([d["gamma"].numpy()[G * kgn:(G + 1) * kgn] for _, G in pairs])
+    assert_chain_close(got, ref, sc, ga, eps, kgn, "fused chain full size")
+    # every group is normalised: per (n, G) mean ~ 0 and mean square ~ var/(var+eps)
+    yy = y.view(128, 8, -1).double()
+    m = yy.mean(dim=2)
+    assert float(m.abs().max()) < 1e-3
+
+
+def test_chain_deterministic():
+    d = inputs.chain_inputs(4, 8, 64, 64, 32, 3, 3, 1, 8, seed=70, bias_scale_std=1.0)
+    y1 = _chain_dev(d, 1, 0, 1, 1, 1e-5).clone()
+    y2 = _chain_dev(d, 1, 0, 1, 1, 1e-5)
+    assert torch.equal(y1, y2)
+
+
+def test_chain_scale_zero_gives_beta():
+    d = inputs.chain_inputs(2, 8, 20, 20, 32, 3, 3, 1, 8, seed=71, affine="random")
+    d["scale"] = torch.zeros(32)
+    y = _chain_dev(d, 1, 0, 1, 1, 1e-5)
+    want = d["beta"].view(1, 32, 1, 1).expand_as(y.cpu())
+    assert torch.equal(y.cpu(), want.contiguous())
