@@ -73,6 +73,8 @@ def library():
         lib.gconv2d_plan_name.argtypes = geo + [i]
         lib.gconv_force_kernel.restype = i
         lib.gconv_force_kernel.argtypes = [s]
+        lib.gconv_device_error_status.restype = i
+        lib.gconv_device_error_status.argtypes = []
         _lib = lib
         return lib
 

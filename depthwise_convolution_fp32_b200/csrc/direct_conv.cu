@@ -12,15 +12,18 @@
 // and k3 (four horizontally adjacent outputs per thread) are combined and
 // extended:
 //  * a CTA owns a tile of TP output rows x TQ output columns x KBtot output
-//    channels; the input rows and columns that tile needs, for cchunk input
-//    channels at a time, are staged into shared memory with 16-byte
-//    cp.async copies whose source size is 0 outside the image, so the zero
-//    padding costs no instructions (4-byte copies when rows are not 16-byte
-//    aligned, e.g. W = 14);
+//    channels.  The input rows and columns that tile needs are staged into
+//    shared memory either
+//      - by TMA: one elected warp issues 3-D tiled loads (one per row band
+//        and input plane); out-of-bounds elements arrive as zeros, so the
+//        padding costs nothing, and each band completes on its own mbarrier
+//        so threads whose rows have arrived start computing while later
+//        bands are still in flight; or
+//      - by 16-byte (or, for rows that are not 16-byte aligned, 4-byte)
+//        cp.async copies with a zero source size outside the image, for
+//        shapes TMA cannot describe or that need several channel passes;
 //  * every staged row is addressed in 16-byte chunks so the window one
-//    thread needs is read with 128-bit shared loads that are bank-conflict
-//    free across a quarter warp (the row pitch is padded so consecutive rows
-//    continue the chunk sequence modulo 8);
+//    thread needs is read with 128-bit shared loads;
 //  * a thread keeps 4 adjacent outputs x RPT rows x KT output channels in
 //    registers: each input value read from shared memory feeds up to
 //    R*S*KT FMAs, each weight (a 128-bit broadcast load over KT channels)
@@ -29,32 +32,23 @@
 //    logistic function and reduces (count, mean, M2) per output channel and
 //    thread in registers (two-pass), then merges them per GroupNorm group in
 //    a fixed order (Chan's parallel-variance update), one partial per CTA and
-//    group, so no atomics are needed and results are deterministic.
+//    group, so no atomics are needed and results are deterministic;
+//  * launches use programmatic dependent launch: a kernel's CTAs are
+//    scheduled while the previous kernel in the stream drains and wait
+//    (griddepcontrol.wait) before their first global access.
 // A generic variant (all geometry at run time, inputs read straight from
 // global memory) serves every shape the specialised variants do not.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "device_utils.cuh"
 #include "gconv_internal.h"
 
 namespace gconv {
 
 namespace {
 
-__device__ __forceinline__ void cp_async16(float *sdst, const float *gsrc, bool valid) {
-    unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(sdst));
-    int nbytes = valid ? 16 : 0;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gsrc), "r"(nbytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void cp_async4(float *sdst, const float *gsrc, bool valid) {
-    unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(sdst));
-    int nbytes = valid ? 4 : 0;
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(s), "l"(gsrc), "r"(nbytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.wait_all;\n" ::: "memory");
-}
+__device__ int g_device_error = 0;
 
 // Chan et al. pairwise update of (count, mean, M2) -- FP32, used inside a CTA.
 __device__ __forceinline__ void chan_merge(float &na, float &ma, float &m2a, float nb, float mb,
@@ -97,7 +91,8 @@ template <> struct Geom<kGeom5x9s1p0> { static constexpr int R = 5, S = 9, ST = 
 template <> struct Geom<kGeom1x1s1p0> { static constexpr int R = 1, S = 1, ST = 1, D = 1, PAD = 0; };
 template <> struct Geom<kDirectGeneric> { static constexpr int R = 0, S = 0, ST = 1, D = 1, PAD = 0; };
 
-constexpr int kV = 4;  // adjacent outputs per thread along q
+constexpr int kV = 4;           // adjacent outputs per thread along q
+constexpr int kBarFloats = 32;  // shared memory reserved for mbarriers (128 B)
 
 template <int G>
 struct Window {
@@ -109,9 +104,10 @@ struct Window {
     static constexpr int NCH = (WIN + 3) / 4;                     // chunks per row per thread
 };
 
-template <int G, int KT, int RPT, bool CHAIN>
-__global__ void __launch_bounds__(256, 2) direct_conv_kernel(const DirectParams p) {
-    extern __shared__ __align__(16) float smem[];
+template <int G, int KT, int RPT, bool CHAIN, bool TMA>
+__global__ void __launch_bounds__(256, 2)
+    direct_conv_kernel(const __grid_constant__ TensorMap tm, const DirectParams p) {
+    extern __shared__ __align__(128) float smem[];
     using g = Geom<G>;
     using win = Window<G>;
     constexpr bool FAST = win::FAST;
@@ -139,8 +135,23 @@ __global__ void __launch_bounds__(256, 2) direct_conv_kernel(const DirectParams 
     const int Ss = FAST ? g::S : p.S;
     const int RS = Rr * Ss;
 
-    float *sw = smem;                    // [cchunk][R][S][KBtot]
-    float *sx = smem + p.w_floats;       // [GB*cchunk][IHt][pitch]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
+    float *sw = smem + kBarFloats;       // [cchunk][R][S][KBtot]
+    float *sx = smem + p.x_off;          // [planes][rows][pitch]
+
+    const int ih0 = p0 * p.stride - p.pad;
+    const int iw0 = q0 * p.stride - 4 * win::HL;
+    bool ok_wait = true;
+
+    if constexpr (TMA) {
+        if (tid == 0) {
+            for (int b = 0; b < p.nb; ++b) dev::mbar_init(&bars[b], 1);
+            dev::fence_mbar_init();
+        }
+        __syncthreads();
+    }
+    dev::griddep_wait();
+    dev::griddep_launch_dependents();
 
     float acc[RPT][kV][KT];
 #pragma unroll
@@ -150,12 +161,27 @@ __global__ void __launch_bounds__(256, 2) direct_conv_kernel(const DirectParams 
 #pragma unroll
             for (int k = 0; k < KT; ++k) acc[a][v][k] = 0.f;
 
-    const int ih0 = p0 * p.stride - p.pad;
-    const int iw0 = q0 * p.stride - 4 * win::HL;
-
     for (int c0 = 0; c0 < p.cpg; c0 += p.cchunk) {
         const int cc = min(p.cchunk, p.cpg - c0);
-        __syncthreads();   // the previous pass is done with shared memory
+        if constexpr (TMA) {
+            // one pass (cchunk == cpg): warp 0 issues every band of every plane
+            if (tid < 32) {
+                const int planes = p.GB * cc;
+                const int box_w = 4 * p.PC;
+                if (tid == 0)
+                    for (int b = 0; b < p.nb; ++b)
+                        dev::mbar_arrive_expect_tx(&bars[b], (uint32_t)(planes * p.bh * box_w * 4));
+                __syncwarp();
+                const int zbase = n * p.C + g0 * p.cpg;
+                for (int j = tid; j < p.nb * planes; j += 32) {
+                    const int b = j / planes, pl = j - b * planes;
+                    dev::tma_load_3d(sx + (long long)pl * p.pstride + b * p.bh * box_w, &tm, &bars[b], iw0,
+                                     ih0 + b * p.bh, zbase + pl);
+                }
+            }
+        } else {
+            __syncthreads();   // the previous pass is done with shared memory
+        }
         // weight slice, transposed to [c][r][s][channel] so KT channels are contiguous
         const int nw = cc * RS * p.KBtot;
         for (int e = tid; e < nw; e += blockDim.x) {
@@ -164,7 +190,7 @@ __global__ void __launch_bounds__(256, 2) direct_conv_kernel(const DirectParams 
             int c = rest / RS, rs = rest - c * RS;
             sw[e] = __ldg(p.w + ((long long)(kc0 + kl) * p.cpg + c0 + c) * RS + rs);
         }
-        if constexpr (FAST) {
+        if constexpr (FAST && !TMA) {
             const int planes = p.GB * cc;
             if (p.vec_in) {
                 const int total = planes * p.IHt * p.PC;
@@ -178,7 +204,7 @@ __global__ void __launch_bounds__(256, 2) direct_conv_kernel(const DirectParams 
                     int ih = ih0 + row, iw = iw0 + 4 * ch;
                     bool ok = ih >= 0 && ih < p.H && iw >= 0 && iw < p.W;
                     const float *src = ok ? p.x + (((long long)n * p.C + ci) * p.H + ih) * p.W + iw : p.x;
-                    cp_async16(sx + ((long long)pl * p.IHt + row) * p.pitch + 4 * ch, src, ok);
+                    dev::cp_async16(sx + (long long)pl * p.pstride + row * p.pitch + 4 * ch, src, ok);
                 }
             } else {
                 const int cols = 4 * p.PC;
@@ -193,17 +219,28 @@ __global__ void __launch_bounds__(256, 2) direct_conv_kernel(const DirectParams 
                     int ih = ih0 + row, iw = iw0 + j;
                     bool ok = ih >= 0 && ih < p.H && iw >= 0 && iw < p.W;
                     const float *src = ok ? p.x + (((long long)n * p.C + ci) * p.H + ih) * p.W + iw : p.x;
-                    cp_async4(sx + ((long long)pl * p.IHt + row) * p.pitch + j, src, ok);
+                    dev::cp_async4(sx + (long long)pl * p.pstride + row * p.pitch + j, src, ok);
                 }
             }
-            cp_async_wait_all();
+            dev::cp_async_wait_all();
         }
         __syncthreads();
         if (!active) continue;
 
         if constexpr (FAST) {
+            if constexpr (TMA) {
+                // wait for the bands holding this thread's input rows
+                const int r_first = ry * RPT * g::ST;
+                const int b_last = min(p.nb - 1, (r_first + IR - 1) / p.bh);
+                for (int b = r_first / p.bh; b <= b_last; ++b)
+                    if (!dev::mbar_wait_bounded(&bars[b], 0)) ok_wait = false;
+                if (!ok_wait) {
+                    atomicExch(&g_device_error, 1);
+                    continue;
+                }
+            }
             for (int c = 0; c < cc; ++c) {
-                const float *xs = sx + ((long long)(gb * cc + c) * p.IHt + ry * RPT * g::ST) * p.pitch +
+                const float *xs = sx + (long long)(gb * cc + c) * p.pstride + (ry * RPT * g::ST) * p.pitch +
                                   cx * g::ST * 4;
                 const float *ws = sw + c * RS * p.KBtot + kl0;
                 float xr[IR][win::NCH * 4];
@@ -264,7 +301,7 @@ __global__ void __launch_bounds__(256, 2) direct_conv_kernel(const DirectParams 
 
     // ---------------------------------------------------------------- epilogue
     const int qb = q0 + cx * kV;
-    if (active) {
+    if (active && ok_wait) {
 #pragma unroll
         for (int k = 0; k < KT; ++k) {
             const int kk = kc0 + kl0 + k;
@@ -302,18 +339,20 @@ __global__ void __launch_bounds__(256, 2) direct_conv_kernel(const DirectParams 
 
     if constexpr (CHAIN) {
         // per-thread, per-channel (count, mean, M2) over the thread's valid outputs
-        __syncthreads();   // shared memory is reused for the statistics
+        __syncthreads();   // shared memory (past the barriers) is reused for the statistics
         const int nsp = p.CX * p.RY;
-        float *st_n = smem;
-        float *st_m = smem + p.KBtot * nsp;
-        float *st_q = smem + 2 * p.KBtot * nsp;
+        float *st_n = smem + kBarFloats;
+        float *st_m = st_n + p.KBtot * nsp;
+        float *st_q = st_m + p.KBtot * nsp;
         if (active) {
             float cnt = 0.f;
+            if (ok_wait) {
 #pragma unroll
-            for (int rp = 0; rp < RPT; ++rp)
+                for (int rp = 0; rp < RPT; ++rp)
 #pragma unroll
-                for (int v = 0; v < kV; ++v)
-                    if (p0 + ry * RPT + rp < p.P && qb + v < p.Q) cnt += 1.f;
+                    for (int v = 0; v < kV; ++v)
+                        if (p0 + ry * RPT + rp < p.P && qb + v < p.Q) cnt += 1.f;
+            }
             const int sp = ry * p.CX + cx;
 #pragma unroll
             for (int k = 0; k < KT; ++k) {
@@ -334,7 +373,7 @@ __global__ void __launch_bounds__(256, 2) direct_conv_kernel(const DirectParams 
                             m2 = fmaf(d, d, m2);
                         }
                 const int e = (kl0 + k) * nsp + sp;
-                st_n[e] = cnt; st_m[e] = mean; st_q[e] = m2;
+                st_n[e] = cnt; st_m[e] = mean; st_q[e] = cnt > 0.f ? m2 : 0.f;
             }
         }
         __syncthreads();
@@ -367,42 +406,75 @@ __global__ void __launch_bounds__(256, 2) direct_conv_kernel(const DirectParams 
     }
 }
 
-template <int G, int KT, bool CHAIN>
-cudaError_t launch_one(const DirectParams &p, dim3 grid, int threads, size_t smem, cudaStream_t st) {
-    constexpr int RPT = (KT >= 4) ? 2 : 4;
-    auto kern = direct_conv_kernel<G, KT, RPT, CHAIN>;
+template <typename Kern>
+cudaError_t launch_pdl(Kern kern, dim3 grid, int threads, size_t smem, cudaStream_t st, const TensorMap &tm,
+                       const DirectParams &p) {
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
     }
-    kern<<<grid, threads, smem, st>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tm, p);
+}
+
+template <int G, int KT, bool CHAIN>
+cudaError_t launch_one(const DirectParams &p, const TensorMap &tm, dim3 grid, int threads, size_t smem,
+                       cudaStream_t st) {
+    constexpr int RPT = (KT >= 4) ? 2 : 4;
+    if constexpr (Window<G>::FAST) {
+        if (p.tma) return launch_pdl(direct_conv_kernel<G, KT, RPT, CHAIN, true>, grid, threads, smem, st, tm, p);
+    }
+    return launch_pdl(direct_conv_kernel<G, KT, RPT, CHAIN, false>, grid, threads, smem, st, tm, p);
 }
 
 template <int G, bool CHAIN>
-cudaError_t launch_kt(const DirectParams &p, int KT, dim3 grid, int threads, size_t smem, cudaStream_t st) {
+cudaError_t launch_kt(const DirectParams &p, const TensorMap &tm, int KT, dim3 grid, int threads, size_t smem,
+                      cudaStream_t st) {
     switch (KT) {
-        case 1: return launch_one<G, 1, CHAIN>(p, grid, threads, smem, st);
-        case 2: return launch_one<G, 2, CHAIN>(p, grid, threads, smem, st);
-        case 4: return launch_one<G, 4, CHAIN>(p, grid, threads, smem, st);
-        case 8: return launch_one<G, 8, CHAIN>(p, grid, threads, smem, st);
+        case 1: return launch_one<G, 1, CHAIN>(p, tm, grid, threads, smem, st);
+        case 2: return launch_one<G, 2, CHAIN>(p, tm, grid, threads, smem, st);
+        case 4: return launch_one<G, 4, CHAIN>(p, tm, grid, threads, smem, st);
+        case 8: return launch_one<G, 8, CHAIN>(p, tm, grid, threads, smem, st);
         default: return cudaErrorInvalidValue;
     }
 }
 
 template <bool CHAIN>
-cudaError_t launch_geom(const DirectParams &p, int geom, int KT, dim3 grid, int threads, size_t smem,
-                        cudaStream_t st) {
+cudaError_t launch_geom(const DirectParams &p, const TensorMap &tm, int geom, int KT, dim3 grid, int threads,
+                        size_t smem, cudaStream_t st) {
     switch (geom) {
-        case kGeom3x3s1p1: return launch_kt<kGeom3x3s1p1, CHAIN>(p, KT, grid, threads, smem, st);
-        case kGeom3x3s1p0: return launch_kt<kGeom3x3s1p0, CHAIN>(p, KT, grid, threads, smem, st);
-        case kGeom3x3s2p1: return launch_kt<kGeom3x3s2p1, CHAIN>(p, KT, grid, threads, smem, st);
-        case kGeom5x9s1p0: return launch_kt<kGeom5x9s1p0, CHAIN>(p, KT, grid, threads, smem, st);
-        case kGeom1x1s1p0: return launch_kt<kGeom1x1s1p0, CHAIN>(p, KT, grid, threads, smem, st);
-        case kDirectGeneric: return launch_kt<kDirectGeneric, CHAIN>(p, KT, grid, threads, smem, st);
+        case kGeom3x3s1p1: return launch_kt<kGeom3x3s1p1, CHAIN>(p, tm, KT, grid, threads, smem, st);
+        case kGeom3x3s1p0: return launch_kt<kGeom3x3s1p0, CHAIN>(p, tm, KT, grid, threads, smem, st);
+        case kGeom3x3s2p1: return launch_kt<kGeom3x3s2p1, CHAIN>(p, tm, KT, grid, threads, smem, st);
+        case kGeom5x9s1p0: return launch_kt<kGeom5x9s1p0, CHAIN>(p, tm, KT, grid, threads, smem, st);
+        case kGeom1x1s1p0: return launch_kt<kGeom1x1s1p0, CHAIN>(p, tm, KT, grid, threads, smem, st);
+        case kDirectGeneric: return launch_kt<kDirectGeneric, CHAIN>(p, tm, KT, grid, threads, smem, st);
         default: return cudaErrorInvalidValue;
     }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+        }
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }();
+    return fn;
 }
 
 }  // namespace
@@ -420,10 +492,31 @@ int direct_fast_window_chunks(int geom) {
     }
 }
 
-cudaError_t launch_direct(const DirectParams &p, int geom, int KT, int chain, dim3 grid, int threads,
-                          size_t smem, cudaStream_t stream) {
-    return chain ? launch_geom<true>(p, geom, KT, grid, threads, smem, stream)
-                 : launch_geom<false>(p, geom, KT, grid, threads, smem, stream);
+bool make_x_tensor_map(TensorMap *tm, const float *x, long long planes, int H, int W, int box_w, int box_h) {
+    static_assert(sizeof(TensorMap) == sizeof(CUtensorMap), "tensor map size");
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)planes};
+    cuuint64_t strides[2] = {(cuuint64_t)W * 4, (cuuint64_t)W * H * 4};
+    cuuint32_t box[3] = {(cuuint32_t)box_w, (cuuint32_t)box_h, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(reinterpret_cast<CUtensorMap *>(tm), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(x),
+                    dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+cudaError_t launch_direct(const DirectParams &p, const TensorMap &tm, int geom, int KT, int chain, dim3 grid,
+                          int threads, size_t smem, cudaStream_t stream) {
+    return chain ? launch_geom<true>(p, tm, geom, KT, grid, threads, smem, stream)
+                 : launch_geom<false>(p, tm, geom, KT, grid, threads, smem, stream);
+}
+
+int read_and_clear_device_error() {
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return -1;
+    if (v) cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+    return v;
 }
 
 }  // namespace gconv

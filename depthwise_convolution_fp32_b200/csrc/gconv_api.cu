@@ -2,6 +2,7 @@
 // geometry, per-shape kernel planning, the GroupNorm workspace, and the two
 // entry points of the FP32 NCHW conv2d forward and the fused
 // conv -> bias -> scale -> sigmoid -> GroupNorm chain.
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -17,8 +18,9 @@ namespace {
 constexpr int kMaxThreads = 256;
 constexpr size_t kSmemBudget = 100 * 1024;   // keep two CTAs per SM where possible
 constexpr size_t kSmemMax = 227 * 1024;
+constexpr int kBarFloats = 32;               // shared memory reserved for mbarriers
 
-enum ForceMode : int { kForceAuto = 0, kForceDirect = 1, kForceGeneric = 2 };
+enum ForceMode : int { kForceAuto = 0, kForceDirect = 1, kForceGeneric = 2, kForceCpAsync = 3 };
 std::atomic<int> g_force{kForceAuto};
 
 struct Shape {
@@ -70,7 +72,20 @@ const char *geom_name(int geom) {
     }
 }
 
+const char *geom_name_tma(int geom) {
+    switch (geom) {
+        case kGeom3x3s1p1: return "direct_tma_3x3s1p1";
+        case kGeom3x3s1p0: return "direct_tma_3x3s1p0";
+        case kGeom3x3s2p1: return "direct_tma_3x3s2p1";
+        case kGeom5x9s1p0: return "direct_tma_5x9s1p0";
+        case kGeom1x1s1p0: return "direct_tma_1x1s1p0";
+        default: return "direct_generic";
+    }
+}
+
 bool compat(int a, int b) { return a % b == 0 || b % a == 0; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 
@@ -85,7 +100,7 @@ struct DirectPlan {
 
 // Choose the CTA tile for a direct-kernel launch.  Returns false when no tile
 // fits the shared-memory limit (the shape is then unsupported by this family).
-bool plan_direct(const Shape &s, bool chain, int gn_groups, int geom, DirectPlan &pl) {
+bool plan_direct(const Shape &s, bool chain, int gn_groups, int geom, bool x_vec, DirectPlan &pl) {
     const bool fast = geom != kDirectGeneric;
     const int kgn = chain ? s.K / gn_groups : 1;
     DirectParams &p = pl.prm;
@@ -143,19 +158,41 @@ bool plan_direct(const Shape &s, bool chain, int gn_groups, int geom, DirectPlan
         while (((pcp - CX * s.stride) % 8 + 8) % 8 != 0) ++pcp;
         pitch = 4 * pcp;
     }
+    auto w_floats_for = [&](int cc) -> size_t { return ((size_t)cc * RS * KBtot + 3) / 4 * 4; };
+    auto x_off_for = [&](int cc) -> size_t { return kBarFloats + (w_floats_for(cc) + 31) / 32 * 32; };
     auto smem_for = [&](int cc) -> size_t {
-        size_t wf = ((size_t)cc * RS * KBtot + 3) / 4 * 4;
         size_t xf = fast ? (size_t)GB * cc * IHt * pitch : 0;
-        return (wf + xf) * sizeof(float);
+        return (x_off_for(cc) + xf) * sizeof(float);
     };
     int cchunk = s.cpg;
     while (cchunk > 1 && smem_for(cchunk) > kSmemBudget) cchunk = (cchunk + 1) / 2;
     size_t smem = smem_for(cchunk);
     const int nsp = CX * RY;
-    if (chain) {
-        size_t st = (size_t)3 * KBtot * nsp * sizeof(float);
-        if (st > smem) smem = st;
+    const size_t st_bytes = chain ? (kBarFloats + (size_t)3 * KBtot * nsp) * sizeof(float) : 0;
+
+    // TMA staging: one pass over all input channels, aligned rows, boxes
+    // within the 256-element limit; rows fetched in bands of ~16.
+    int tma = 0, nb = 1, bh = IHt;
+    size_t pstride = (size_t)IHt * pitch;
+    const int planes = GB * s.cpg;
+    // box rows padded to 128 bytes so every TMA destination is 128-byte aligned
+    const int tpc = (PC + 7) / 8 * 8;
+    if (fast && x_vec && cchunk == s.cpg && 4 * tpc <= 256 && planes <= 256) {
+        nb = std::min(8, std::max(1, (IHt + 15) / 16));
+        bh = (IHt + nb - 1) / nb;
+        nb = (IHt + bh - 1) / bh;
+        const size_t tpitch = 4 * (size_t)tpc;
+        const size_t tps = (size_t)nb * bh * tpitch;
+        const size_t tsmem = (x_off_for(cchunk) + planes * tps) * sizeof(float);
+        if (bh <= 256 && tsmem <= kSmemMax) {
+            tma = 1;
+            PC = tpc;
+            pitch = (int)tpitch;
+            pstride = tps;
+            smem = tsmem;
+        }
     }
+    if (st_bytes > smem) smem = st_bytes;
     if (smem > kSmemMax) return false;
 
     p.N = s.N; p.C = s.C; p.H = s.H; p.W = s.W; p.K = s.K; p.R = s.R; p.S = s.S;
@@ -165,7 +202,12 @@ bool plan_direct(const Shape &s, bool chain, int gn_groups, int geom, DirectPlan
     p.TP = TP; p.TQ = 4 * CX; p.KB = KB; p.KBtot = KBtot;
     p.n_qt = n_qt; p.n_pt = n_pt; p.n_kb = n_kb;
     p.IHt = IHt; p.PC = PC; p.pitch = pitch; p.cchunk = cchunk;
-    p.w_floats = (int)(((size_t)cchunk * RS * KBtot + 3) / 4 * 4);
+    p.w_floats = (int)w_floats_for(cchunk);
+    p.x_off = (int)x_off_for(cchunk);
+    p.pstride = (int)pstride;
+    p.tma = tma;
+    p.nb = nb;
+    p.bh = bh;
     p.gn_groups = chain ? gn_groups : 0;
     p.kgn = kgn;
     p.n_sp = n_qt * n_pt;
@@ -184,15 +226,33 @@ bool plan_direct(const Shape &s, bool chain, int gn_groups, int geom, DirectPlan
 }
 
 // Direct-kernel plan for the current forcing mode.
-bool choose_direct(const Shape &s, bool chain, int gn_groups, DirectPlan &pl) {
+bool choose_direct(const Shape &s, bool chain, int gn_groups, bool x_vec, DirectPlan &pl) {
     const int force = g_force.load(std::memory_order_relaxed);
     int geom = (force == kForceGeneric) ? (int)kDirectGeneric : match_geom(s);
-    if (plan_direct(s, chain, gn_groups, geom, pl)) return true;
-    if (geom != kDirectGeneric && force == kForceAuto) return plan_direct(s, chain, gn_groups, kDirectGeneric, pl);
+    if (force == kForceCpAsync) x_vec = false;
+    if (plan_direct(s, chain, gn_groups, geom, x_vec, pl)) return true;
+    if (geom != kDirectGeneric && force == kForceAuto)
+        return plan_direct(s, chain, gn_groups, kDirectGeneric, x_vec, pl);
     return false;
 }
 
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// Fill the pointer-dependent fields and the TMA descriptor of a plan; a map
+// the driver rejects falls back to cp.async staging.
+bool finish_plan(const Shape &s, bool chain, int gn_groups, const float *x, float *y, DirectPlan &pl,
+                 TensorMap &tm) {
+    DirectParams &p = pl.prm;
+    p.vec_in = (s.W % 4 == 0) && aligned16(x);
+    p.vec_out = (s.Q % 4 == 0) && aligned16(y);
+    std::memset(&tm, 0, sizeof(tm));
+    if (p.tma && !make_x_tensor_map(&tm, x, (long long)s.N * s.C, s.H, s.W, 4 * p.PC, p.bh)) {
+        DirectPlan again;
+        if (!plan_direct(s, chain, gn_groups, pl.geom, false, again)) return false;
+        again.prm.vec_in = p.vec_in;
+        again.prm.vec_out = p.vec_out;
+        pl = again;
+    }
+    return true;
+}
 
 // ----------------------------------------------------------------- workspace
 struct Workspace {
@@ -262,7 +322,13 @@ const char *gconv_status_string(gconv_status_t status) {
     return "unknown gconv status";
 }
 
-const char *gconv_version(void) { return "gconv-b200 0.1.0 (sm_100a)"; }
+const char *gconv_version(void) { return "gconv-b200 0.2.0 (sm_100a)"; }
+
+gconv_status_t gconv_device_error_status(void) {
+    int v = read_and_clear_device_error();
+    if (v < 0) return GCONV_ERR_CUDA;
+    return v ? GCONV_ERR_TIMEOUT : GCONV_OK;
+}
 
 gconv_status_t gconv2d_output_size(int H, int W, int R, int S, int stride, int pad, int dilation, int *P,
                                    int *Q) {
@@ -281,6 +347,7 @@ gconv_status_t gconv_force_kernel(const char *name) {
     if (!std::strcmp(name, "auto")) g_force = kForceAuto;
     else if (!std::strcmp(name, "direct")) g_force = kForceDirect;
     else if (!std::strcmp(name, "generic")) g_force = kForceGeneric;
+    else if (!std::strcmp(name, "direct_cpasync")) g_force = kForceCpAsync;
     else return GCONV_ERR_INVALID_ARG;
     return GCONV_OK;
 }
@@ -293,8 +360,8 @@ const char *gconv2d_plan_name(int N, int C, int H, int W, int K, int R, int S, i
     if (st != GCONV_OK) return "unsupported";
     DirectPlan pl;
     int gn = 1;
-    if (!choose_direct(s, chain != 0, gn, pl)) return "unsupported";
-    return geom_name(pl.geom);
+    if (!choose_direct(s, chain != 0, gn, s.W % 4 == 0, pl)) return "unsupported";
+    return pl.prm.tma ? geom_name_tma(pl.geom) : geom_name(pl.geom);
 }
 
 gconv_status_t gconv2d_fwd(const float *x, const float *w, const float *bias, int N, int C, int H, int W, int K,
@@ -306,12 +373,13 @@ gconv_status_t gconv2d_fwd(const float *x, const float *w, const float *bias, in
     if ((st = validate_ptrs(x, w, y)) != GCONV_OK) return st;
     if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) return GCONV_ERR_INVALID_ARG;
     DirectPlan pl;
-    if (!choose_direct(s, false, 1, pl)) return GCONV_ERR_UNSUPPORTED;
+    const bool x_vec = (s.W % 4 == 0) && aligned16(x);
+    if (!choose_direct(s, false, 1, x_vec, pl)) return GCONV_ERR_UNSUPPORTED;
+    TensorMap tm;
+    if (!finish_plan(s, false, 1, x, y, pl, tm)) return GCONV_ERR_UNSUPPORTED;
     DirectParams &p = pl.prm;
     p.x = x; p.w = w; p.bias = bias; p.y = y;
-    p.vec_in = (s.W % 4 == 0) && aligned16(x);
-    p.vec_out = (s.Q % 4 == 0) && aligned16(y);
-    if (launch_direct(p, pl.geom, pl.KT, 0, pl.grid, pl.threads, pl.smem, stream) != cudaSuccess)
+    if (launch_direct(p, tm, pl.geom, pl.KT, 0, pl.grid, pl.threads, pl.smem, stream) != cudaSuccess)
         return GCONV_ERR_CUDA;
     return GCONV_OK;
 }
@@ -322,7 +390,7 @@ size_t gconv2d_chain_workspace_size(int N, int C, int H, int W, int K, int R, in
     if (make_shape(s, N, C, H, W, K, R, S, stride, pad, dilation, groups) != GCONV_OK) return 0;
     if (gn_groups < 1 || K % gn_groups) return 0;
     DirectPlan pl;
-    if (!choose_direct(s, true, gn_groups, pl)) return 0;
+    if (!choose_direct(s, true, gn_groups, s.W % 4 == 0, pl)) return 0;
     return chain_ws_bytes(pl.prm);
 }
 
@@ -346,16 +414,17 @@ gconv_status_t gconv2d_bias_scale_sigmoid_groupnorm_fwd(const float *x, const fl
     for (const void *q : {(const void *)bias, (const void *)scale, (const void *)gamma, (const void *)beta})
         if (q && (reinterpret_cast<uintptr_t>(q) & 3u)) return GCONV_ERR_INVALID_ARG;
     DirectPlan pl;
-    if (!choose_direct(s, true, gn_groups, pl)) return GCONV_ERR_UNSUPPORTED;
+    const bool x_vec = (s.W % 4 == 0) && aligned16(x);
+    if (!choose_direct(s, true, gn_groups, x_vec, pl)) return GCONV_ERR_UNSUPPORTED;
+    TensorMap tm;
+    if (!finish_plan(s, true, gn_groups, x, y, pl, tm)) return GCONV_ERR_UNSUPPORTED;
     DirectParams &p = pl.prm;
     void *ws = nullptr;
     const size_t part_bytes = ((size_t)p.N * p.gn_groups * p.slots * sizeof(float4) + 255) / 256 * 256;
     if ((st = ensure_workspace(chain_ws_bytes(p), stream, &ws)) != GCONV_OK) return st;
     p.x = x; p.w = w; p.bias = bias; p.y = y; p.scale = scale;
     p.gn_part = reinterpret_cast<float4 *>(ws);
-    p.vec_in = (s.W % 4 == 0) && aligned16(x);
-    p.vec_out = (s.Q % 4 == 0) && aligned16(y);
-    if (launch_direct(p, pl.geom, pl.KT, 1, pl.grid, pl.threads, pl.smem, stream) != cudaSuccess)
+    if (launch_direct(p, tm, pl.geom, pl.KT, 1, pl.grid, pl.threads, pl.smem, stream) != cudaSuccess)
         return GCONV_ERR_CUDA;
 
     GnParams g;

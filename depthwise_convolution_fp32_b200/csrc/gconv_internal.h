@@ -45,6 +45,14 @@ struct DirectParams {
     int vec_in;       // x rows are 16-byte aligned (16-byte cp.async staging)
     int vec_out;      // y rows are 16-byte aligned (float4 stores)
 
+    // TMA staging (tma != 0): the tile's rows are fetched as nb bands of bh
+    // rows, one 3-D box (4*PC columns x bh rows x 1 plane) per band and plane,
+    // each band completing on its own mbarrier.  Requires cchunk == cpg.
+    int tma;
+    int nb, bh;
+    int x_off;        // float offset of the x tile in shared memory
+    int pstride;      // floats between staged planes
+
     // chain bookkeeping
     int gn_groups, kgn, slots, slots_k, n_sp;
 };
@@ -61,9 +69,24 @@ struct GnParams {
     int vec;          // float4 path allowed
 };
 
-// Launch one direct-kernel variant; returns cudaGetLastError() of the launch.
-cudaError_t launch_direct(const DirectParams &p, int geom, int KT, int chain,
+// Opaque 128-byte TMA descriptor (CUtensorMap) storage.
+struct alignas(64) TensorMap {
+    unsigned char bytes[128];
+};
+
+// Encode a 3-D tensor map over x viewed as [N*C][H][W] with a box of
+// box_w x box_h x 1 elements (zero fill out of bounds).  Returns false when
+// the driver entry point is unavailable or rejects the map.
+bool make_x_tensor_map(TensorMap *tm, const float *x, long long planes, int H, int W, int box_w, int box_h);
+
+// Launch one direct-kernel variant (programmatic dependent launch enabled);
+// returns the launch status.
+cudaError_t launch_direct(const DirectParams &p, const TensorMap &tm, int geom, int KT, int chain,
                           dim3 grid, int threads, size_t smem, cudaStream_t stream);
+
+// Device error flag raised by bounded waits that gave up (0 = none); reading
+// clears it.  Synchronises with the device.
+int read_and_clear_device_error();
 int direct_rpt(int KT);   // rows per thread the variant with KT uses
 int direct_fast_window_chunks(int geom);   // 16-byte chunks one thread reads per row
 

@@ -12,6 +12,7 @@
 // kernels use (a sits near 0.5 after the logistic function while var can be
 // ~1e-6).  gn_normalize then streams y once (read + write, float4 when rows
 // are 16-byte aligned), one channel plane slice per CTA.
+#include "device_utils.cuh"
 #include "gconv_internal.h"
 
 namespace gconv {
@@ -37,6 +38,8 @@ constexpr int kFinThreads = 128;
 
 __global__ void __launch_bounds__(kFinThreads) gn_finalize_kernel(const GnParams p) {
     __shared__ double sn[kFinThreads], sm[kFinThreads], sq[kFinThreads];
+    dev::griddep_wait();
+    dev::griddep_launch_dependents();
     const int ng = blockIdx.x;
     const int tid = threadIdx.x;
     double cn = 0.0, mn = 0.0, m2 = 0.0;
@@ -65,6 +68,8 @@ __global__ void __launch_bounds__(kFinThreads) gn_finalize_kernel(const GnParams
 constexpr int kNormThreads = 256;
 
 __global__ void __launch_bounds__(kNormThreads) gn_normalize_kernel(const GnParams p) {
+    dev::griddep_wait();
+    dev::griddep_launch_dependents();
     const long long plane = blockIdx.x / p.chunks;        // n*K + k
     const int chunk = blockIdx.x % p.chunks;
     const int k = (int)(plane % p.K);
@@ -100,16 +105,35 @@ __global__ void __launch_bounds__(kNormThreads) gn_normalize_kernel(const GnPara
 
 }  // namespace
 
+namespace {
+
+template <typename Kern>
+cudaError_t launch_pdl(Kern kern, unsigned blocks, int threads, cudaStream_t st, const GnParams &p) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+}  // namespace
+
 cudaError_t launch_gn_finalize(const GnParams &p, cudaStream_t stream) {
-    gn_finalize_kernel<<<p.N * p.gn_groups, kFinThreads, 0, stream>>>(p);
-    return cudaGetLastError();
+    long long blocks = (long long)p.N * p.gn_groups;
+    if (blocks <= 0 || blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    return launch_pdl(gn_finalize_kernel, (unsigned)blocks, kFinThreads, stream, p);
 }
 
 cudaError_t launch_gn_normalize(const GnParams &p, cudaStream_t stream) {
     long long blocks = (long long)p.N * p.K * p.chunks;
     if (blocks <= 0 || blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    gn_normalize_kernel<<<(unsigned)blocks, kNormThreads, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(gn_normalize_kernel, (unsigned)blocks, kNormThreads, stream, p);
 }
 
 }  // namespace gconv

@@ -131,6 +131,12 @@ GCONV_API const char *gconv2d_plan_name(int N, int C, int H, int W, int K, int R
  * GCONV_ERR_INVALID_ARG for an unknown name.  Intended for measurement. */
 GCONV_API gconv_status_t gconv_force_kernel(const char *name);
 
+/* Status of the bounded waits inside the kernels since the last query:
+ * GCONV_ERR_TIMEOUT when a kernel gave up waiting for its own asynchronous
+ * copies (its outputs for that tile were not written), GCONV_OK otherwise.
+ * Reading clears the flag.  Synchronises with the current device. */
+GCONV_API gconv_status_t gconv_device_error_status(void);
+
 /* Library version string. */
 GCONV_API const char *gconv_version(void);
 

@@ -101,7 +101,8 @@ def test_chain_rejects_invalid_arguments(lib):
 
 
 def test_plan_names(lib):
-    assert gc.plan_name(4, 144, 56, 56, 144, 3, 3, 1, 1, 1, 144) == "direct_3x3s1p1"
+    assert gc.plan_name(4, 144, 56, 56, 144, 3, 3, 1, 1, 1, 144) == "direct_tma_3x3s1p1"
+    assert gc.plan_name(2, 16, 14, 14, 16, 3, 3, 1, 1, 1, 16) == "direct_3x3s1p1"
     assert gc.plan_name(1, 8, 16, 16, 8, 3, 3, 1, 1, 2, 4) == "direct_generic"
     assert gc.plan_name(1, 8, 16, 16, 8, 3, 3, 1, 1, 1, 3) == "invalid"
     assert gc.chain_workspace_size(128, 8, 256, 256, 32, 3, 3, 1, 0, 1, 1, 8) > 0
@@ -109,7 +110,7 @@ def test_plan_names(lib):
 
 
 def test_force_kernel_names(lib):
-    for n in ("generic", "direct", "auto"):
+    for n in ("generic", "direct", "direct_cpasync", "auto"):
         gc.force_kernel(n)
     with pytest.raises(gc.GconvError):
         gc.force_kernel("cudnn")

@@ -171,7 +171,7 @@ GEOMS = [
     (1, 3, 3, 3, 5, 3, 3, 1, 0, 1, 1, True),         # P = Q = 1
     (1, 8, 6, 6, 8, 3, 3, 1, 4, 1, 8, False),        # padding larger than the halo chunk
     (1, 64, 9, 9, 64, 3, 3, 1, 1, 1, 1, False),      # dense 3x3, cpg 64 (channel chunks)
-    (1, 96, 7, 8, 12, 5, 9, 1, 0, 1, 1, False),      # dense 5x9 with many channels
+    (1, 96, 7, 12, 12, 5, 9, 1, 0, 1, 1, False),     # dense 5x9 with many channels
 ]
 
 
@@ -193,6 +193,34 @@ def test_forced_generic_matches_oracle(oracle_mod, geo):
         full_check(oracle_mod, d, st, pad, dil, g, "generic " + str(geo))
     finally:
         gc.force_kernel("auto")
+
+
+@pytest.mark.parametrize("geo", GEOMS[:10], ids=lambda g: "x".join(map(str, g[:11])))
+def test_forced_cpasync_staging_matches_oracle(oracle_mod, geo):
+    """The cp.async staging path on shapes that would otherwise use TMA."""
+    N, C, H, W, K, R, S, st, pad, dil, g, bias = geo
+    d = inputs.conv_inputs(N, C, H, W, K, R, S, g, seed=11 + zlib.crc32(repr(geo).encode()) % 1000,
+                           x_dist="normal", bias=bias)
+    gc.force_kernel("direct_cpasync")
+    try:
+        full_check(oracle_mod, d, st, pad, dil, g, "cp.async " + str(geo))
+    finally:
+        gc.force_kernel("auto")
+
+
+def test_forced_cpasync_chain(oracle_mod):
+    d = inputs.chain_inputs(2, 8, 40, 40, 32, 3, 3, 1, 8, seed=64, bias_scale_std=1.0, affine="random")
+    gc.force_kernel("direct_cpasync")
+    try:
+        y = _chain_dev(d, 1, 0, 1, 1, 1e-5).cpu().numpy()
+    finally:
+        gc.force_kernel("auto")
+    ref = _chain_ref(oracle_mod, d, 1, 0, 1, 1, 1e-5)
+    assert_chain_close(y, ref, d["scale"].numpy(), d["gamma"].numpy(), 1e-5, 4, "cp.async chain")
+
+
+def test_no_device_error_flag():
+    assert gc.library().gconv_device_error_status() == gc.OK
 
 
 @pytest.mark.parametrize("mis", [1, 2, 3])
