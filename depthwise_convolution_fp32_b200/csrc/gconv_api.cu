@@ -445,3 +445,93 @@ gconv_status_t gconv2d_bias_scale_sigmoid_groupnorm_fwd(const float *x, const fl
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------
+// Allocation-free variant of the fused chain (gconv2d_bias_scale_sigmoid_
+// groupnorm_fwd_noalloc).  Its GroupNorm partials live in a fixed array in
+// device memory that every GPU loading this library reserves until process
+// exit, instead of the workspace the regular entry point grows with
+// cudaMalloc.  Host code must not hand the array's name to a kernel: on the
+// host that name is only a stand-in, so the device address is looked up with
+// cudaGetSymbolAddress once per device (with that device current) and passed
+// as a pointer.
+static constexpr size_t kNoAllocScratchBytes = 4u << 20;   // 4 MiB per GPU
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+void *g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mutex;
+
+// Device address of the scratch array on the current device; the first call
+// per device performs the lookup.
+gconv_status_t noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GCONV_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return GCONV_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+            cudaGetLastError();
+            return GCONV_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return GCONV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gconv_noalloc_scratch_capacity(void) { return kNoAllocScratchBytes; }
+
+gconv_status_t gconv2d_bias_scale_sigmoid_groupnorm_fwd_noalloc(
+    const float *x, const float *w, const float *bias, int N, int C, int H, int W, int K, int R, int S,
+    int stride, int pad, int dilation, int groups, const float *scale, int gn_groups, const float *gamma,
+    const float *beta, float eps, float *y, cudaStream_t stream) {
+    Shape s;
+    gconv_status_t st = make_shape(s, N, C, H, W, K, R, S, stride, pad, dilation, groups);
+    if (st != GCONV_OK) return st;
+    if ((st = validate_ptrs(x, w, y)) != GCONV_OK) return st;
+    if (!scale || !gamma || !beta) return GCONV_ERR_INVALID_ARG;
+    if (gn_groups < 1 || K % gn_groups != 0) return GCONV_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || eps != eps) return GCONV_ERR_INVALID_ARG;
+    for (const void *q : {(const void *)bias, (const void *)scale, (const void *)gamma, (const void *)beta})
+        if (q && (reinterpret_cast<uintptr_t>(q) & 3u)) return GCONV_ERR_INVALID_ARG;
+    DirectPlan pl;
+    const bool x_vec = (s.W % 4 == 0) && aligned16(x);
+    if (!choose_direct(s, true, gn_groups, x_vec, pl)) return GCONV_ERR_UNSUPPORTED;
+    TensorMap tm;
+    if (!finish_plan(s, true, gn_groups, x, y, pl, tm)) return GCONV_ERR_UNSUPPORTED;
+    DirectParams &p = pl.prm;
+    // every partial slot and every statistics entry is written by this call
+    // before it is read, so stale contents from an earlier call never leak
+    if (chain_ws_bytes(p) > kNoAllocScratchBytes) return GCONV_ERR_WORKSPACE;
+    void *ws = nullptr;
+    if ((st = noalloc_scratch(&ws)) != GCONV_OK) return st;
+    const size_t part_bytes = ((size_t)p.N * p.gn_groups * p.slots * sizeof(float4) + 255) / 256 * 256;
+    p.x = x; p.w = w; p.bias = bias; p.y = y; p.scale = scale;
+    p.gn_part = reinterpret_cast<float4 *>(ws);
+    if (launch_direct(p, tm, pl.geom, pl.KT, 1, pl.grid, pl.threads, pl.smem, stream) != cudaSuccess)
+        return GCONV_ERR_CUDA;
+    GnParams g;
+    g.y = y;
+    g.gn_part = p.gn_part;
+    g.stats = reinterpret_cast<float2 *>(reinterpret_cast<char *>(ws) + part_bytes);
+    g.gamma = gamma; g.beta = beta;
+    g.N = s.N; g.K = s.K; g.gn_groups = gn_groups; g.kgn = s.K / gn_groups; g.slots = p.slots;
+    g.PQ = (long long)s.P * s.Q;
+    g.eps = eps;
+    g.vec = (g.PQ % 4 == 0) && aligned16(y);
+    const long long per_cta = g.vec ? 4LL * 256 * 8 : 256LL * 8;
+    g.chunks = (int)((g.PQ + per_cta - 1) / per_cta);
+    if (g.chunks < 1) g.chunks = 1;
+    if (launch_gn_finalize(g, stream) != cudaSuccess) return GCONV_ERR_CUDA;
+    if (launch_gn_normalize(g, stream) != cudaSuccess) return GCONV_ERR_CUDA;
+    return GCONV_OK;
+}
+
+}  // extern "C"

@@ -107,6 +107,40 @@ GCONV_API gconv_status_t gconv2d_bias_scale_sigmoid_groupnorm_fwd(
     const float *scale, int gn_groups, const float *gamma, const float *beta,
     float eps, float *y, cudaStream_t stream);
 
+/* Allocation-free variant of gconv2d_bias_scale_sigmoid_groupnorm_fwd (the
+ * pages have no counterpart: this is an addition for callers of this
+ * library).  Same arguments, same result, same kernels; the only difference
+ * is where the GroupNorm partial statistics live.  The regular entry point
+ * keeps them in a workspace it grows with cudaMalloc; this one uses a
+ * fixed-size scratch array in device memory that every GPU loading the
+ * library reserves until process exit (gconv_noalloc_scratch_capacity()
+ * bytes, 4 MiB), so it never calls cudaMalloc, cudaFree or any other
+ * allocator.  It is meant for callers that cannot allocate device memory at
+ * call time: code recording a CUDA graph (allocation is not allowed while a
+ * stream is being captured), engines that must not stall on an implicit
+ * device synchronisation or must keep a fixed memory budget after start-up,
+ * and hosts whose allocator is owned by another framework.
+ * - Shapes whose partial statistics need more than the capacity
+ *   (gconv2d_chain_workspace_size() > capacity) return GCONV_ERR_WORKSPACE
+ *   and launch nothing; use the regular entry point for them.
+ * - The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ * - Every call on a device shares the one array and leaves its contents
+ *   behind; each call writes every entry it later reads, so nothing needs to
+ *   start at zero.  Calls whose kernels overlap on the GPU (for example on two
+ *   streams without ordering between them) race on the array and must be
+ *   serialised by the caller. */
+GCONV_API gconv_status_t gconv2d_bias_scale_sigmoid_groupnorm_fwd_noalloc(
+    const float *x, const float *w, const float *bias,
+    int N, int C, int H, int W, int K, int R, int S,
+    int stride, int pad, int dilation, int groups,
+    const float *scale, int gn_groups, const float *gamma, const float *beta,
+    float eps, float *y, cudaStream_t stream);
+
+/* Bytes of the fixed scratch array the allocation-free chain may use. */
+GCONV_API size_t gconv_noalloc_scratch_capacity(void);
+
 /* Bytes of workspace the fused chain needs for this shape (0 on invalid input). */
 GCONV_API size_t gconv2d_chain_workspace_size(int N, int C, int H, int W, int K, int R, int S,
                                     int stride, int pad, int dilation, int groups,
