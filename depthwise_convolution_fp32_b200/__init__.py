@@ -25,7 +25,8 @@ __all__ = [
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR_TIMEOUT = range(6)
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_PKG, "libgconv.so")
+# GCONV_LIBRARY may point at another build of the same library (A/B measurements).
+_LIB_PATH = os.environ.get("GCONV_LIBRARY") or os.path.join(_PKG, "libgconv.so")
 _lock = threading.Lock()
 _lib = None
 

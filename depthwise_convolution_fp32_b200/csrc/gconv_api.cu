@@ -20,7 +20,7 @@ constexpr size_t kSmemBudget = 100 * 1024;   // keep two CTAs per SM where possi
 constexpr size_t kSmemMax = 227 * 1024;
 constexpr int kBarFloats = 32;               // shared memory reserved for mbarriers
 
-enum ForceMode : int { kForceAuto = 0, kForceDirect = 1, kForceGeneric = 2, kForceCpAsync = 3 };
+enum ForceMode : int { kForceAuto = 0, kForceDirect = 1, kForceGeneric = 2, kForceCpAsync = 3, kForceIgemm = 4 };
 std::atomic<int> g_force{kForceAuto};
 
 struct Shape {
@@ -299,6 +299,139 @@ size_t chain_ws_bytes(const DirectParams &p) {
     return (part + 255) / 256 * 256 + stats;
 }
 
+// ----------------------------------------------------------------- implicit GEMM
+struct IgemmPlan {
+    IgemmParams prm;
+    dim3 grid;
+    size_t smem;
+    size_t off_xl, off_wh, off_wl, off_part, off_stats, ws_bytes;
+};
+
+size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+int env_int(const char *name) {
+    const char *e = std::getenv(name);
+    return e ? std::atoi(e) : 0;
+}
+
+// Stride-1 convolutions whose groups hold a multiple of 8 input channels and
+// 32/64/128/256 output channels run as an implicit GEMM on the tensor cores.
+bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
+    if (s.stride != 1 || s.cpg % 8 != 0 || !igemm_supported_nt(s.kpg)) return false;
+    const int kgn = chain ? s.K / gn_groups : 1;
+    if (chain && s.kpg % kgn != 0) return false;
+    const int NT = s.kpg;
+    int COLS = 128 + (s.S - 1) * s.dil;
+    COLS = (COLS + 3) / 4 * 4;
+    if (COLS > 256) return false;
+    static const int force_th = env_int("GCONV_IGEMM_TH");
+    static const int force_st = env_int("GCONV_IGEMM_STAGES");
+    // output rows per CTA: accumulators of two CTAs fit the 512 TMEM columns
+    int TH = std::max(1, 256 / NT);
+    TH = std::min(TH, 8);
+    if (force_th > 0) TH = force_th;
+    TH = std::min(TH, s.P);
+    int tmem_cols = 32;
+    while (tmem_cols < TH * NT) tmem_cols *= 2;
+    if (tmem_cols > 512) return false;
+    const int a_bytes = 32 * COLS * TH;
+    const int b_bytes = 32 * s.S * NT;
+    const size_t stage = 2 * (size_t)a_bytes + 2 * (size_t)b_bytes;
+    const int num_k = (s.cpg / 8) * s.R;
+    int stages = std::min(4, num_k);
+    if (force_st > 0) stages = std::min(force_st, num_k);
+    const size_t limit = 227 * 1024 - igemm_header_bytes();
+    while (stages > 1 && stages * stage > limit) --stages;
+    if (stages * stage > limit) return false;
+    const size_t st_bytes = chain ? (size_t)NT * 4 * 3 * sizeof(float) : 0;
+    if (st_bytes > stages * stage) return false;
+
+    IgemmParams &p = pl.prm;
+    std::memset(&p, 0, sizeof(p));
+    p.N = s.N; p.C = s.C; p.H = s.H; p.W = s.W; p.K = s.K; p.R = s.R; p.S = s.S;
+    p.pad = s.pad; p.dil = s.dil; p.groups = s.groups; p.cpg = s.cpg; p.kpg = s.kpg; p.P = s.P; p.Q = s.Q;
+    p.CC8 = s.cpg / 8;
+    p.TH = TH;
+    p.COLS = COLS;
+    p.n_qt = (s.Q + 127) / 128;
+    p.n_pt = (s.P + TH - 1) / TH;
+    p.stages = stages;
+    p.a_bytes = a_bytes;
+    p.b_bytes = b_bytes;
+    p.tmem_cols = tmem_cols;
+    p.gn_groups = chain ? gn_groups : 0;
+    p.kgn = kgn;
+    p.slots = p.n_qt * p.n_pt;
+    const long long gx = (long long)p.n_qt * p.n_pt;
+    if (gx > 0x7fffffffLL || s.groups > 65535 || s.N > 65535) return false;
+    pl.grid = dim3((unsigned)gx, (unsigned)s.groups, (unsigned)s.N);
+    pl.smem = igemm_header_bytes() + stages * stage;
+
+    const size_t xbytes = (size_t)s.N * s.C * s.H * s.W * sizeof(float);
+    const size_t wbytes = (size_t)s.K * s.cpg * s.R * s.S * sizeof(float);
+    pl.off_xl = align256(xbytes);
+    pl.off_wh = pl.off_xl + align256(xbytes);
+    pl.off_wl = pl.off_wh + align256(wbytes);
+    pl.off_part = pl.off_wl + align256(wbytes);
+    const size_t part = chain ? (size_t)s.N * gn_groups * p.slots * sizeof(float4) : 0;
+    pl.off_stats = pl.off_part + align256(part);
+    pl.ws_bytes = pl.off_stats + (chain ? (size_t)s.N * gn_groups * sizeof(float2) : 0);
+    return true;
+}
+
+// Whether the dispatcher sends a shape to the implicit GEMM.
+bool use_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
+    const int force = g_force.load(std::memory_order_relaxed);
+    if (force == kForceDirect || force == kForceGeneric || force == kForceCpAsync) return false;
+    if (!plan_igemm(s, chain, gn_groups, pl)) return false;
+    if (force == kForceIgemm) return true;
+    // auto: enough reduction depth and output channels for the tensor cores to win
+    return s.cpg * s.R * s.S >= 64;
+}
+
+// Launch the split passes and the GEMM; chain additionally runs the GroupNorm
+// finalize and normalize passes.
+gconv_status_t run_igemm(const Shape &s, IgemmPlan &pl, const float *x, const float *w, const float *bias,
+                         const float *scale, int gn_groups, const float *gamma, const float *beta, float eps,
+                         float *y, void *ws, cudaStream_t stream) {
+    char *base = reinterpret_cast<char *>(ws);
+    float *xh = reinterpret_cast<float *>(base);
+    float *xl = reinterpret_cast<float *>(base + pl.off_xl);
+    float *wh = reinterpret_cast<float *>(base + pl.off_wh);
+    float *wl = reinterpret_cast<float *>(base + pl.off_wl);
+    IgemmParams &p = pl.prm;
+    const long long quads = (long long)s.N * (s.C / 4);
+    TensorMap tmh, tml;
+    if (!make_nc4hw4_tensor_map(&tmh, xh, quads, s.H, s.W, p.COLS, p.TH) ||
+        !make_nc4hw4_tensor_map(&tml, xl, quads, s.H, s.W, p.COLS, p.TH))
+        return GCONV_ERR_UNSUPPORTED;
+    p.wh = reinterpret_cast<const float4 *>(wh);
+    p.wl = reinterpret_cast<const float4 *>(wl);
+    p.bias = bias;
+    p.scale = scale;
+    p.y = y;
+    const bool chain = scale != nullptr;
+    p.gn_part = chain ? reinterpret_cast<float4 *>(base + pl.off_part) : nullptr;
+    if (launch_split_x(x, xh, xl, s.N, s.C, s.H, s.W, stream) != cudaSuccess) return GCONV_ERR_CUDA;
+    if (launch_split_w(w, wh, wl, s.K, s.cpg, s.R, s.S, s.groups, stream) != cudaSuccess) return GCONV_ERR_CUDA;
+    if (launch_igemm(p, tmh, tml, chain ? 1 : 0, pl.grid, pl.smem, stream) != cudaSuccess) return GCONV_ERR_CUDA;
+    if (!chain) return GCONV_OK;
+    GnParams g;
+    g.y = y;
+    g.gn_part = p.gn_part;
+    g.stats = reinterpret_cast<float2 *>(base + pl.off_stats);
+    g.gamma = gamma; g.beta = beta;
+    g.N = s.N; g.K = s.K; g.gn_groups = gn_groups; g.kgn = s.K / gn_groups; g.slots = p.slots;
+    g.PQ = (long long)s.P * s.Q;
+    g.eps = eps;
+    g.vec = (g.PQ % 4 == 0) && aligned16(y);
+    const long long per_cta = g.vec ? 4LL * 256 * 8 : 256LL * 8;
+    g.chunks = (int)std::max<long long>(1, (g.PQ + per_cta - 1) / per_cta);
+    if (launch_gn_finalize(g, stream) != cudaSuccess) return GCONV_ERR_CUDA;
+    if (launch_gn_normalize(g, stream) != cudaSuccess) return GCONV_ERR_CUDA;
+    return GCONV_OK;
+}
+
 gconv_status_t validate_ptrs(const float *x, const float *w, const float *y) {
     if (!x || !w || !y) return GCONV_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(y)) & 3u)
@@ -326,8 +459,9 @@ const char *gconv_version(void) { return "gconv-b200 0.2.0 (sm_100a)"; }
 
 gconv_status_t gconv_device_error_status(void) {
     int v = read_and_clear_device_error();
-    if (v < 0) return GCONV_ERR_CUDA;
-    return v ? GCONV_ERR_TIMEOUT : GCONV_OK;
+    int u = read_and_clear_igemm_error();
+    if (v < 0 || u < 0) return GCONV_ERR_CUDA;
+    return (v || u) ? GCONV_ERR_TIMEOUT : GCONV_OK;
 }
 
 gconv_status_t gconv2d_output_size(int H, int W, int R, int S, int stride, int pad, int dilation, int *P,
@@ -348,6 +482,7 @@ gconv_status_t gconv_force_kernel(const char *name) {
     else if (!std::strcmp(name, "direct")) g_force = kForceDirect;
     else if (!std::strcmp(name, "generic")) g_force = kForceGeneric;
     else if (!std::strcmp(name, "direct_cpasync")) g_force = kForceCpAsync;
+    else if (!std::strcmp(name, "igemm")) g_force = kForceIgemm;
     else return GCONV_ERR_INVALID_ARG;
     return GCONV_OK;
 }
@@ -358,6 +493,8 @@ const char *gconv2d_plan_name(int N, int C, int H, int W, int K, int R, int S, i
     gconv_status_t st = make_shape(s, N, C, H, W, K, R, S, stride, pad, dilation, groups);
     if (st == GCONV_ERR_INVALID_ARG) return "invalid";
     if (st != GCONV_OK) return "unsupported";
+    IgemmPlan ig;
+    if (use_igemm(s, chain != 0, chain ? s.K : 1, ig)) return "igemm_tf32x3";
     DirectPlan pl;
     int gn = 1;
     if (!choose_direct(s, chain != 0, gn, s.W % 4 == 0, pl)) return "unsupported";
@@ -372,6 +509,13 @@ gconv_status_t gconv2d_fwd(const float *x, const float *w, const float *bias, in
     if (st != GCONV_OK) return st;
     if ((st = validate_ptrs(x, w, y)) != GCONV_OK) return st;
     if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) return GCONV_ERR_INVALID_ARG;
+    IgemmPlan ig;
+    if (use_igemm(s, false, 1, ig)) {
+        void *ws = nullptr;
+        if ((st = ensure_workspace(ig.ws_bytes, stream, &ws)) != GCONV_OK) return st;
+        return run_igemm(s, ig, x, w, bias, nullptr, 0, nullptr, nullptr, 0.f, y, ws, stream);
+    }
+    if (g_force.load(std::memory_order_relaxed) == kForceIgemm) return GCONV_ERR_UNSUPPORTED;
     DirectPlan pl;
     const bool x_vec = (s.W % 4 == 0) && aligned16(x);
     if (!choose_direct(s, false, 1, x_vec, pl)) return GCONV_ERR_UNSUPPORTED;
@@ -389,6 +533,8 @@ size_t gconv2d_chain_workspace_size(int N, int C, int H, int W, int K, int R, in
     Shape s;
     if (make_shape(s, N, C, H, W, K, R, S, stride, pad, dilation, groups) != GCONV_OK) return 0;
     if (gn_groups < 1 || K % gn_groups) return 0;
+    IgemmPlan ig;
+    if (use_igemm(s, true, gn_groups, ig)) return ig.ws_bytes;
     DirectPlan pl;
     if (!choose_direct(s, true, gn_groups, s.W % 4 == 0, pl)) return 0;
     return chain_ws_bytes(pl.prm);
@@ -413,6 +559,13 @@ gconv_status_t gconv2d_bias_scale_sigmoid_groupnorm_fwd(const float *x, const fl
     if (!(eps >= 0.f) || eps != eps) return GCONV_ERR_INVALID_ARG;
     for (const void *q : {(const void *)bias, (const void *)scale, (const void *)gamma, (const void *)beta})
         if (q && (reinterpret_cast<uintptr_t>(q) & 3u)) return GCONV_ERR_INVALID_ARG;
+    IgemmPlan ig;
+    if (use_igemm(s, true, gn_groups, ig)) {
+        void *ws = nullptr;
+        if ((st = ensure_workspace(ig.ws_bytes, stream, &ws)) != GCONV_OK) return st;
+        return run_igemm(s, ig, x, w, bias, scale, gn_groups, gamma, beta, eps, y, ws, stream);
+    }
+    if (g_force.load(std::memory_order_relaxed) == kForceIgemm) return GCONV_ERR_UNSUPPORTED;
     DirectPlan pl;
     const bool x_vec = (s.W % 4 == 0) && aligned16(x);
     if (!choose_direct(s, true, gn_groups, x_vec, pl)) return GCONV_ERR_UNSUPPORTED;

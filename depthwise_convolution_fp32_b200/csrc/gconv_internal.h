@@ -90,6 +90,36 @@ int read_and_clear_device_error();
 int direct_rpt(int KT);   // rows per thread the variant with KT uses
 int direct_fast_window_chunks(int geom);   // 16-byte chunks one thread reads per row
 
+// ---- implicit GEMM on tcgen05 (3xTF32) -------------------------------------
+struct IgemmParams {
+    const float4 *wh, *wl;     // split weights [g][cpg/8][r][s][2][kpg][4]
+    const float *bias, *scale; // bias may be null; scale only for the chain
+    float *y;
+    float4 *gn_part;           // chain only
+    int N, C, H, W, K, R, S, pad, dil, groups, cpg, kpg, P, Q;
+    int CC8;                   // cpg / 8 (K-steps of 8 channels)
+    int TH;                    // output rows per CTA (one 128-pixel M tile each)
+    int COLS;                  // staged columns per row (>= 128 + (S-1)*dil, multiple of 4)
+    int n_qt, n_pt;
+    int stages;                // shared-memory pipeline depth
+    int a_bytes, b_bytes;      // one x operand (hi or lo) / one w operand per stage
+    int tmem_cols;
+    int gn_groups, kgn, slots;
+};
+
+int igemm_supported_nt(int kpg);
+size_t igemm_header_bytes();
+// 4-D tensor map over an NC4HW4 tensor [quads][H][W][4] with a box of
+// 4 x box_cols x box_rows x 2 quads.
+bool make_nc4hw4_tensor_map(TensorMap *tm, const float *base, long long quads, int H, int W, int box_cols,
+                            int box_rows);
+cudaError_t launch_split_x(const float *x, float *xh, float *xl, int N, int C, int H, int W, cudaStream_t st);
+cudaError_t launch_split_w(const float *w, float *wh, float *wl, int K, int cpg, int R, int S, int groups,
+                           cudaStream_t st);
+cudaError_t launch_igemm(const IgemmParams &p, const TensorMap &tmh, const TensorMap &tml, int chain, dim3 grid,
+                         size_t smem, cudaStream_t st);
+int read_and_clear_igemm_error();
+
 cudaError_t launch_gn_finalize(const GnParams &p, cudaStream_t stream);
 cudaError_t launch_gn_normalize(const GnParams &p, cudaStream_t stream);
 

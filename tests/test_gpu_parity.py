@@ -344,3 +344,57 @@ def test_chain_scale_zero_gives_beta():
     y = _chain_dev(d, 1, 0, 1, 1, 1e-5)
     want = d["beta"].view(1, 32, 1, 1).expand_as(y.cpu())
     assert torch.equal(y.cpu(), want.contiguous())
+
+
+# ------------------------------------------------------------------ implicit GEMM (tcgen05)
+
+IGEMM_GEOMS = [
+    # N, C, H, W, K, R, S, stride, pad, dil, groups, bias
+    (1, 8, 20, 150, 32, 3, 3, 1, 0, 1, 1, True),      # Q > 128: two M tiles along q, ragged
+    (2, 8, 19, 33, 32, 3, 3, 1, 1, 1, 1, False),      # padding, ragged rows
+    (1, 16, 12, 40, 64, 5, 9, 1, 0, 1, 1, True),      # the dense asymmetric kernel
+    (1, 32, 9, 137, 64, 5, 9, 1, 2, 1, 1, False),     # 5x9 with padding, Q = 133
+    (1, 16, 17, 29, 32, 3, 3, 1, 2, 2, 1, True),      # dilation 2
+    (2, 16, 10, 20, 64, 3, 3, 1, 1, 1, 2, True),      # two groups of 8 -> 32
+    (1, 8, 9, 18, 128, 3, 3, 1, 1, 1, 1, False),      # N = 128
+    (1, 8, 6, 10, 256, 3, 3, 1, 1, 1, 1, True),       # N = 256
+    (1, 24, 11, 21, 32, 3, 5, 1, 1, 1, 1, False),     # R != S, three channel steps
+    (1, 8, 1, 140, 32, 1, 3, 1, 0, 1, 1, True),       # single output row
+]
+
+
+@pytest.mark.parametrize("geo", IGEMM_GEOMS, ids=lambda g: "x".join(map(str, g[:11])))
+def test_igemm_matches_oracle(oracle_mod, geo):
+    N, C, H, W, K, R, S, st, pad, dil, g, bias = geo
+    d = inputs.conv_inputs(N, C, H, W, K, R, S, g, seed=zlib.crc32(repr(geo).encode()) % 10000,
+                           x_dist="normal", bias=bias)
+    gc.force_kernel("igemm")
+    try:
+        assert gc.plan_name(N, C, H, W, K, R, S, st, pad, dil, g) == "igemm_tf32x3"
+        full_check(oracle_mod, d, st, pad, dil, g, "igemm " + str(geo))
+    finally:
+        gc.force_kernel("auto")
+    assert gc.library().gconv_device_error_status() == gc.OK
+
+
+def test_dense_5x9_direct_path_small(oracle_mod):
+    """The CUDA-core direct path on the dense asymmetric shape (the dispatcher's alternative)."""
+    d = inputs.conv_inputs(1, 32, 37, 70, 64, 5, 9, 1, 78, x_dist="uniform01",
+                           w_bound=1 / math.sqrt(1440))
+    gc.force_kernel("direct")
+    try:
+        full_check(oracle_mod, d, 1, 0, 1, 1, "direct dense 5x9 ragged")
+    finally:
+        gc.force_kernel("auto")
+
+
+@pytest.mark.parametrize("mode", ["igemm", "direct"])
+def test_chain_paths_agree_with_oracle(oracle_mod, mode):
+    d = inputs.chain_inputs(2, 8, 45, 140, 32, 3, 3, 1, 8, seed=81, bias_scale_std=1.0, affine="random")
+    gc.force_kernel(mode)
+    try:
+        y = _chain_dev(d, 1, 0, 1, 1, 1e-5).cpu().numpy()
+    finally:
+        gc.force_kernel("auto")
+    ref = _chain_ref(oracle_mod, d, 1, 0, 1, 1, 1e-5)
+    assert_chain_close(y, ref, d["scale"].numpy(), d["gamma"].numpy(), 1e-5, 4, f"{mode} chain")
