@@ -394,6 +394,8 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="also time the 80-shape sweep")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--force-kernel", default="auto",
+                    help="kernel family for A/B runs: auto, direct, direct_cpasync, generic, igemm")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -421,6 +423,7 @@ def main():
     build.build()
     import depthwise_convolution_fp32_b200 as gc
     gc.library()
+    gc.force_kernel(args.force_kernel)
 
     props = torch.cuda.get_device_properties(device)
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
@@ -466,7 +469,8 @@ def main():
             "l2": f"rotating pool of {runner.n_sets} buffer sets, {runner.pool_bytes / 2**20:.0f} MiB "
                   f"(L2 {l2 / 2**20:.0f} MiB)",
             "timing": "CUDA graph of exactly K calls, device events",
-            "parallelism": f"replicas x{world} (batch shards, no collective)"}),
+            "parallelism": f"replicas x{world} (batch shards, no collective)",
+            "kernel_family": args.force_kernel}),
         "gflops": round(gflops, 2),
         "sync_api_us": round(sync_us, 2),
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,

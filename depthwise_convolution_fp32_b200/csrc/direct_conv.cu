@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
                 for (int v = 0; v < kV; ++v) {
                     float z = acc[rp][v][k] + b;
-                    if constexpr (CHAIN) z = 1.f / (1.f + expf(-(z * sc)));
+                    if constexpr (CHAIN) z = __frcp_rn(1.f + __expf(-(z * sc)));
                     acc[rp][v][k] = z;
                 }
         }

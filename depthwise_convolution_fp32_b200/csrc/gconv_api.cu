@@ -178,7 +178,11 @@ bool plan_direct(const Shape &s, bool chain, int gn_groups, int geom, bool x_vec
     // box rows padded to 128 bytes so every TMA destination is 128-byte aligned
     const int tpc = (PC + 7) / 8 * 8;
     if (fast && x_vec && cchunk == s.cpg && 4 * tpc <= 256 && planes <= 256) {
-        nb = std::min(8, std::max(1, (IHt + 15) / 16));
+        static const int band_rows = [] {
+            const char *e = std::getenv("GCONV_DIRECT_BAND_ROWS");
+            return e ? std::max(1, std::atoi(e)) : 16;
+        }();
+        nb = std::min(8, std::max(1, (IHt + band_rows - 1) / band_rows));
         bh = (IHt + nb - 1) / nb;
         nb = (IHt + bh - 1) / bh;
         const size_t tpitch = 4 * (size_t)tpc;
@@ -309,6 +313,19 @@ struct IgemmPlan {
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
+int sm_count() {
+    static const int n = [] {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+            cudaGetLastError();
+            return 148;
+        }
+        return v;
+    }();
+    return n;
+}
+
 int env_int(const char *name) {
     const char *e = std::getenv(name);
     return e ? std::atoi(e) : 0;
@@ -319,32 +336,29 @@ int env_int(const char *name) {
 bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     if (s.stride != 1 || s.cpg % 8 != 0 || !igemm_supported_nt(s.kpg)) return false;
     const int kgn = chain ? s.K / gn_groups : 1;
-    if (chain && s.kpg % kgn != 0) return false;
+    // chain epilogue: groups nest inside a conv group, widths 1..16 or multiples of 16
+    if (chain && (s.kpg > 64 || s.kpg % kgn != 0 || (kgn > 16 && kgn % 16 != 0))) return false;
     const int NT = s.kpg;
     int COLS = 128 + (s.S - 1) * s.dil;
-    COLS = (COLS + 3) / 4 * 4;
+    COLS = (COLS + 7) / 8 * 8;   // 128-byte aligned row segments
     if (COLS > 256) return false;
     static const int force_th = env_int("GCONV_IGEMM_TH");
     static const int force_st = env_int("GCONV_IGEMM_STAGES");
-    // output rows per CTA: accumulators of two CTAs fit the 512 TMEM columns
-    int TH = std::max(1, 256 / NT);
-    TH = std::min(TH, 8);
+    // output rows per tile: two accumulator buffers of TH*NT columns fit TMEM
+    int TH = std::max(1, std::min(8, 256 / NT));
     if (force_th > 0) TH = force_th;
     TH = std::min(TH, s.P);
     int tmem_cols = 32;
-    while (tmem_cols < TH * NT) tmem_cols *= 2;
+    while (tmem_cols < 2 * TH * NT) tmem_cols *= 2;
     if (tmem_cols > 512) return false;
     const int a_bytes = 32 * COLS * TH;
     const int b_bytes = 32 * s.S * NT;
     const size_t stage = 2 * (size_t)a_bytes + 2 * (size_t)b_bytes;
-    const int num_k = (s.cpg / 8) * s.R;
-    int stages = std::min(4, num_k);
-    if (force_st > 0) stages = std::min(force_st, num_k);
-    const size_t limit = 227 * 1024 - igemm_header_bytes();
+    int stages = 4;
+    if (force_st > 0) stages = std::min(force_st, 8);
+    const size_t limit = 227 * 1024 - igemm_header_bytes(NT, chain);
     while (stages > 1 && stages * stage > limit) --stages;
     if (stages * stage > limit) return false;
-    const size_t st_bytes = chain ? (size_t)NT * 4 * 3 * sizeof(float) : 0;
-    if (st_bytes > stages * stage) return false;
 
     IgemmParams &p = pl.prm;
     std::memset(&p, 0, sizeof(p));
@@ -355,6 +369,9 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     p.COLS = COLS;
     p.n_qt = (s.Q + 127) / 128;
     p.n_pt = (s.P + TH - 1) / TH;
+    const long long n_tiles = (long long)s.N * s.groups * p.n_qt * p.n_pt;
+    if (n_tiles > 0x7fffffffLL) return false;
+    p.n_tiles = (int)n_tiles;
     p.stages = stages;
     p.a_bytes = a_bytes;
     p.b_bytes = b_bytes;
@@ -362,10 +379,8 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     p.gn_groups = chain ? gn_groups : 0;
     p.kgn = kgn;
     p.slots = p.n_qt * p.n_pt;
-    const long long gx = (long long)p.n_qt * p.n_pt;
-    if (gx > 0x7fffffffLL || s.groups > 65535 || s.N > 65535) return false;
-    pl.grid = dim3((unsigned)gx, (unsigned)s.groups, (unsigned)s.N);
-    pl.smem = igemm_header_bytes() + stages * stage;
+    pl.grid = dim3((unsigned)std::min<long long>(n_tiles, sm_count()));
+    pl.smem = igemm_header_bytes(NT, chain) + stages * stage;
 
     const size_t xbytes = (size_t)s.N * s.C * s.H * s.W * sizeof(float);
     const size_t wbytes = (size_t)s.K * s.cpg * s.R * s.S * sizeof(float);
@@ -402,8 +417,7 @@ gconv_status_t run_igemm(const Shape &s, IgemmPlan &pl, const float *x, const fl
     IgemmParams &p = pl.prm;
     const long long quads = (long long)s.N * (s.C / 4);
     TensorMap tmh, tml;
-    if (!make_nc4hw4_tensor_map(&tmh, xh, quads, s.H, s.W, p.COLS, p.TH) ||
-        !make_nc4hw4_tensor_map(&tml, xl, quads, s.H, s.W, p.COLS, p.TH))
+    if (!make_nc4hw4_tensor_map(&tmh, xh, quads, s.H, s.W) || !make_nc4hw4_tensor_map(&tml, xl, quads, s.H, s.W))
         return GCONV_ERR_UNSUPPORTED;
     p.wh = reinterpret_cast<const float4 *>(wh);
     p.wl = reinterpret_cast<const float4 *>(wl);

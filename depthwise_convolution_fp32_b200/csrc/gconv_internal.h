@@ -99,8 +99,9 @@ struct IgemmParams {
     int N, C, H, W, K, R, S, pad, dil, groups, cpg, kpg, P, Q;
     int CC8;                   // cpg / 8 (K-steps of 8 channels)
     int TH;                    // output rows per CTA (one 128-pixel M tile each)
-    int COLS;                  // staged columns per row (>= 128 + (S-1)*dil, multiple of 4)
+    int COLS;                  // staged columns per row (>= 128 + (S-1)*dil, multiple of 8)
     int n_qt, n_pt;
+    int n_tiles;               // N * groups * n_pt * n_qt
     int stages;                // shared-memory pipeline depth
     int a_bytes, b_bytes;      // one x operand (hi or lo) / one w operand per stage
     int tmem_cols;
@@ -108,11 +109,11 @@ struct IgemmParams {
 };
 
 int igemm_supported_nt(int kpg);
-size_t igemm_header_bytes();
-// 4-D tensor map over an NC4HW4 tensor [quads][H][W][4] with a box of
-// 4 x box_cols x box_rows x 2 quads.
-bool make_nc4hw4_tensor_map(TensorMap *tm, const float *base, long long quads, int H, int W, int box_cols,
-                            int box_rows);
+size_t igemm_header_bytes(int nt, bool chain);
+int igemm_threads();
+// 3-D tensor map over an NC4HW4 tensor viewed as [quads][H][W*4] floats with
+// a box of 256 floats (64 pixels of one row of one channel quad).
+bool make_nc4hw4_tensor_map(TensorMap *tm, const float *base, long long quads, int H, int W);
 cudaError_t launch_split_x(const float *x, float *xh, float *xl, int N, int C, int H, int W, cudaStream_t st);
 cudaError_t launch_split_w(const float *w, float *wh, float *wl, int K, int cpg, int R, int S, int groups,
                            cudaStream_t st);

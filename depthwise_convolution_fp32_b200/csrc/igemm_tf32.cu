@@ -100,51 +100,81 @@ __global__ void __launch_bounds__(256) split_w_kernel(const float *__restrict__ 
     }
 }
 
-// Chan et al. pairwise update of (count, mean, M2).
-__device__ __forceinline__ void chan_merge(float &na, float &ma, float &m2a, float nb, float mb, float m2b) {
-    if (nb == 0.f) return;
-    if (na == 0.f) {
-        na = nb; ma = mb; m2a = m2b;
-        return;
-    }
-    float n = na + nb;
-    float d = mb - ma;
-    float f = nb / n;
-    ma = fmaf(d, f, ma);
-    m2a = m2a + m2b + d * d * na * f;
-    na = n;
+constexpr int kIgEpiWarps = 8;                      // epilogue warps (2 per TMEM lane quarter)
+constexpr int kIgThreads = 64 + 32 * kIgEpiWarps;    // + producer warp + MMA warp
+// shared memory ahead of the stage ring: barriers, TMEM slot and, for the
+// chain, per-fragment statistics [NT fragments at most][4 lane quarters][3 doubles]
+__host__ __device__ constexpr int ig_header(int NT, bool chain) {
+    return chain ? (256 + 96 * NT + 1023) / 1024 * 1024 : 1024;
 }
 
-constexpr int kIgThreads = 256;
-constexpr int kIgHeader = 1024;   // barriers and the TMEM address slot
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(dev::smem_addr(bar)) : "memory");
+}
+
+// Named barrier over the epilogue warps only.
+__device__ __forceinline__ void epi_sync() {
+    asm volatile("bar.sync 1, %0;\n" ::"r"(32 * kIgEpiWarps) : "memory");
+}
+
+// Output tile t -> (n, g, row tile, column tile); column tiles vary fastest so
+// CTAs running side by side share input rows in L2.
+struct IgTile {
+    int n, g, p0, q0, sp;
+};
+
+__device__ __forceinline__ IgTile ig_tile(const IgemmParams &p, int t) {
+    IgTile r;
+    const int nsp = p.n_qt * p.n_pt;
+    r.sp = t % nsp;
+    const int rest = t / nsp;
+    r.g = rest % p.groups;
+    r.n = rest / p.groups;
+    r.q0 = (r.sp % p.n_qt) * 128;
+    r.p0 = (r.sp / p.n_qt) * p.TH;
+    return r;
+}
 
 // ------------------------------------------------------------------ main kernel
-template <int NT, bool CHAIN>
-__global__ void __launch_bounds__(kIgThreads, 2)
+// Persistent: CTA b processes tiles b, b + gridDim.x, ...  The producer and
+// the MMA issuer run ahead through a ring of shared-memory stages; the MMA
+// issuer alternates between two TMEM accumulator buffers so the epilogue of
+// tile j overlaps the MMAs of tile j+1.
+// KGN: 0 = plain convolution; otherwise the GroupNorm group width of the
+// chain (1, 2, 4, 8, 16, or 32 standing for any multiple of 16).
+template <int NT, int KGN>
+__global__ void __launch_bounds__(kIgThreads, 1)
     igemm_tf32x3_kernel(const __grid_constant__ TensorMap tmh, const __grid_constant__ TensorMap tml,
                         const IgemmParams p) {
     extern __shared__ __align__(1024) unsigned char smem[];
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem);        // [stages]
-    uint64_t *empty = full + 8;                                  // [stages]
-    uint64_t *accf = full + 16;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(full + 17);
-    int *abort_flag = reinterpret_cast<int *>(full + 18);
-    unsigned char *stages = smem + kIgHeader;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);   // [stages]
+    uint64_t *empty = full + 8;                             // [stages]
+    uint64_t *accf = full + 16;                             // [2] accumulator ready
+    uint64_t *acce = full + 18;                             // [2] accumulator drained
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(full + 20);
+    int *abort_flag = reinterpret_cast<int *>(full + 21);
+    constexpr bool CHAIN = KGN > 0;
+    double *st_n = reinterpret_cast<double *>(smem + 256);   // [fragment][4] chain statistics
+    double *st_1 = st_n + NT * 4;
+    double *st_2 = st_1 + NT * 4;
+    unsigned char *stages = smem + ig_header(NT, CHAIN);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int qt = blockIdx.x % p.n_qt, pt = blockIdx.x / p.n_qt;
-    const int g = blockIdx.y, n = blockIdx.z;
-    const int q0 = qt * 128, p0 = pt * p.TH;
     const int num_k = p.CC8 * p.R;
+    const int num_tiles = p.n_tiles;
     const uint32_t stage_bytes = 2u * p.a_bytes + 2u * p.b_bytes;
+    const uint32_t acc_cols = (uint32_t)(p.TH * NT);
 
     if (tid == 0) {
         for (int s = 0; s < p.stages; ++s) {
             dev::mbar_init(&full[s], 1);
             dev::mbar_init(&empty[s], 1);
         }
-        dev::mbar_init(accf, 1);
+        for (int b = 0; b < 2; ++b) {
+            dev::mbar_init(&accf[b], 1);
+            dev::mbar_init(&acce[b], kIgEpiWarps);
+        }
         *abort_flag = 0;
         dev::fence_mbar_init();
     }
@@ -160,166 +190,246 @@ __global__ void __launch_bounds__(kIgThreads, 2)
     dev::griddep_wait();
     dev::griddep_launch_dependents();
 
-    if (warp == 0 && lane == 0) {
+    if (warp == 0) {
         // ---------------------------------------------------------- producer
-        const int z0 = n * (p.C / 4) + g * (p.cpg / 4);
-        for (int kt = 0; kt < num_k; ++kt) {
-            const int slot = kt % p.stages;
-            const int use = kt / p.stages;
-            if (use > 0 && !dev::mbar_wait_bounded(&empty[slot], (use - 1) & 1)) {
-                *abort_flag = 1;
-                atomicExch(&g_igemm_error, 1);
-                break;
-            }
-            const int cc8 = kt / p.R, r = kt - cc8 * p.R;
-            unsigned char *st = stages + (size_t)slot * stage_bytes;
-            dev::mbar_arrive_expect_tx(&full[slot], stage_bytes);
-            const int cw = q0 - p.pad, ch = p0 - p.pad + r * p.dil, cz = z0 + cc8 * 2;
-            dev::tma_load_4d(st, &tmh, &full[slot], 0, cw, ch, cz);
-            dev::tma_load_4d(st + p.a_bytes, &tml, &full[slot], 0, cw, ch, cz);
-            const long long woff = (((long long)g * p.CC8 + cc8) * p.R + r) * (p.b_bytes / 16);
-            dev::bulk_load(st + 2 * p.a_bytes, p.wh + woff, p.b_bytes, &full[slot]);
-            dev::bulk_load(st + 2 * p.a_bytes + p.b_bytes, p.wl + woff, p.b_bytes, &full[slot]);
-        }
-    } else if (warp == 1 && lane == 0) {
-        // ---------------------------------------------------------- MMA issuer
-        constexpr uint32_t idesc = dev::idesc_tf32(128, NT);
-        const uint32_t a_lbo = (uint32_t)p.TH * p.COLS * 16;
-        const uint32_t b_lbo = NT * 16;
+        // Each staged row segment of one channel quad is contiguous in the
+        // NC4HW4 tensor; it is fetched as boxes of 64 pixels (1 KB), the last
+        // one aligned to the row end (overlapping the previous box), so the
+        // whole warp issues a few dozen 1 KB TMA loads per stage.
+        const int nseg = (p.COLS + 63) / 64;
+        const int per_op = 2 * p.TH * nseg;                 // boxes per x operand
+        const uint32_t tx = (uint32_t)(2 * per_op * 1024 + 2 * p.b_bytes);
+        int it = 0;
         bool ok = true;
-        for (int kt = 0; kt < num_k && ok; ++kt) {
-            const int slot = kt % p.stages;
-            if (!dev::mbar_wait_bounded(&full[slot], (kt / p.stages) & 1)) {
-                ok = false;
-                *abort_flag = 1;
-                atomicExch(&g_igemm_error, 1);
-                break;
-            }
-            dev::tc_fence_after();
-            const unsigned char *st = stages + (size_t)slot * stage_bytes;
-            const unsigned char *ah = st, *al = st + p.a_bytes;
-            const unsigned char *bh = st + 2 * p.a_bytes, *bl = bh + p.b_bytes;
-            for (int i = 0; i < p.TH; ++i) {
-                const uint32_t d = tmem + (uint32_t)(i * NT);
-                for (int s = 0; s < p.S; ++s) {
-                    const uint32_t ao = (uint32_t)(i * p.COLS + s * p.dil) * 16;
-                    const uint32_t bo = (uint32_t)(s * 2 * NT) * 16;
-                    const uint32_t acc = (kt > 0 || s > 0) ? 1u : 0u;
-                    dev::mma_tf32(d, dev::smem_desc(al + ao, a_lbo, 128), dev::smem_desc(bh + bo, b_lbo, 128),
-                                  idesc, acc);
-                    dev::mma_tf32(d, dev::smem_desc(ah + ao, a_lbo, 128), dev::smem_desc(bl + bo, b_lbo, 128),
-                                  idesc, 1u);
-                    dev::mma_tf32(d, dev::smem_desc(ah + ao, a_lbo, 128), dev::smem_desc(bh + bo, b_lbo, 128),
-                                  idesc, 1u);
+        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            const IgTile tl = ig_tile(p, t);
+            const int z0 = tl.n * (p.C / 4) + tl.g * (p.cpg / 4);
+            for (int kt = 0; kt < num_k; ++kt, ++it) {
+                const int slot = it % p.stages;
+                const int use = it / p.stages;
+                if (lane == 0) {
+                    if (use > 0 && !dev::mbar_wait_bounded(&empty[slot], (use - 1) & 1)) ok = false;
+                    if (*(volatile int *)abort_flag) ok = false;
+                    if (ok) dev::mbar_arrive_expect_tx(&full[slot], tx);
                 }
-            }
-            dev::mma_commit(&empty[slot]);
-        }
-        dev::mma_commit(accf);   // fires once every MMA above has completed
-    }
-    __syncwarp();
-
-    // -------------------------------------------------------------- epilogue
-    const bool have_acc = dev::mbar_wait_bounded(accf, 0);
-    if (!have_acc) atomicExch(&g_igemm_error, 1);
-    dev::tc_fence_after();
-    const bool ok = have_acc && (*(volatile int *)abort_flag == 0);
-
-    const int lq = warp & 3;            // TMEM lane quarter
-    const int chalf = warp >> 2;        // column half
-    constexpr int HALF = NT / 2;
-    const int m = lq * 32 + lane;
-    const int q = q0 + m;
-    const bool qvalid = q < p.Q;
-    const long long plane = (long long)p.P * p.Q;
-    float *ybase = p.y + ((long long)n * p.K + (long long)g * p.kpg) * plane + q;
-
-    // per-channel statistics of this warp (chain): [NT][4 lane quarters]
-    float *st_n = reinterpret_cast<float *>(stages);
-    float *st_m = st_n + NT * 4;
-    float *st_q = st_m + NT * 4;
-
-#pragma unroll 1
-    for (int c0 = chalf * HALF; c0 < (chalf + 1) * HALF; c0 += 16) {
-        float bias_v[16], sc_v[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const int k = g * p.kpg + c0 + j;
-            bias_v[j] = p.bias ? __ldg(p.bias + k) : 0.f;
-            sc_v[j] = CHAIN ? __ldg(p.scale + k) : 1.f;
-        }
-        float shift[16], s1[16], s2[16];
-        float cnt = 0.f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) { shift[j] = 0.f; s1[j] = 0.f; s2[j] = 0.f; }
-#pragma unroll 1
-        for (int i = 0; i < p.TH; ++i) {
-            float v[16];
-            dev::tmem_ld16(tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)(i * NT + c0), v);
-            const int pp = p0 + i;
-            const bool valid = ok && qvalid && pp < p.P;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                float z = v[j] + bias_v[j];
-                if constexpr (CHAIN) z = 1.f / (1.f + expf(-(z * sc_v[j])));
-                v[j] = z;
-            }
-            if (valid) {
-                float *yr = ybase + (long long)c0 * plane + (long long)pp * p.Q;
-#pragma unroll
-                for (int j = 0; j < 16; ++j) yr[(long long)j * plane] = v[j];
-                if constexpr (CHAIN) {
-                    if (cnt == 0.f) {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) shift[j] = v[j];
-                    }
-                    cnt += 1.f;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float d = v[j] - shift[j];
-                        s1[j] += d;
-                        s2[j] = fmaf(d, d, s2[j]);
-                    }
-                }
-            }
-        }
-        if constexpr (CHAIN) {
-            // per channel: thread (cnt, mean, M2) -> warp (fixed shuffle tree) -> shared memory
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                float cn = cnt, mn = 0.f, m2 = 0.f;
-                if (cnt > 0.f) {
-                    const float a = s1[j] / cnt;
-                    mn = shift[j] + a;
-                    m2 = fmaxf(s2[j] - s1[j] * a, 0.f);
-                }
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) {
-                    const float on = __shfl_down_sync(0xffffffffu, cn, off);
-                    const float om = __shfl_down_sync(0xffffffffu, mn, off);
-                    const float oq = __shfl_down_sync(0xffffffffu, m2, off);
-                    if (lane < off) chan_merge(cn, mn, m2, on, om, oq);
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) break;
+                const int cc8 = kt / p.R, r = kt - cc8 * p.R;
+                unsigned char *st = stages + (size_t)slot * stage_bytes;
+                const int x0 = tl.q0 - p.pad, y0 = tl.p0 - p.pad + r * p.dil, cz = z0 + cc8 * 2;
+                for (int b = lane; b < 2 * per_op; b += 32) {
+                    const int lo = b >= per_op;
+                    const int bb = b - lo * per_op;
+                    const int seg = bb % nseg;
+                    const int row = (bb / nseg) % p.TH;
+                    const int quad = bb / (nseg * p.TH);
+                    const int px = seg < nseg - 1 ? seg * 64 : p.COLS - 64;
+                    unsigned char *dst = st + lo * p.a_bytes + ((size_t)(quad * p.TH + row) * p.COLS + px) * 16;
+                    dev::tma_load_3d(dst, lo ? &tml : &tmh, &full[slot], (x0 + px) * 4, y0 + row, cz + quad);
                 }
                 if (lane == 0) {
-                    // stage memory is free: every MMA reading it has completed
-                    st_n[(c0 + j) * 4 + lq] = cn;
-                    st_m[(c0 + j) * 4 + lq] = mn;
-                    st_q[(c0 + j) * 4 + lq] = m2;
+                    const long long woff = (((long long)tl.g * p.CC8 + cc8) * p.R + r) * (p.b_bytes / 16);
+                    dev::bulk_load(st + 2 * p.a_bytes, p.wh + woff, p.b_bytes, &full[slot]);
+                    dev::bulk_load(st + 2 * p.a_bytes + p.b_bytes, p.wl + woff, p.b_bytes, &full[slot]);
                 }
             }
         }
-    }
-
-    if constexpr (CHAIN) {
-        __syncthreads();
-        const int ngroups = NT / p.kgn;
-        if (tid < ngroups) {
-            float cn = 0.f, mn = 0.f, m2 = 0.f;
-            for (int c = tid * p.kgn; c < (tid + 1) * p.kgn; ++c)
-                for (int l = 0; l < 4; ++l) chan_merge(cn, mn, m2, st_n[c * 4 + l], st_m[c * 4 + l], st_q[c * 4 + l]);
-            const int G = (g * p.kpg) / p.kgn + tid;
-            const int slot = pt * p.n_qt + qt;
-            p.gn_part[((long long)n * p.gn_groups + G) * p.slots + slot] = make_float4(cn, mn, m2, 0.f);
+        if (!ok && lane == 0) {
+            *abort_flag = 1;
+            atomicExch(&g_igemm_error, 1);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------------ MMA issuer
+            constexpr uint32_t idesc = dev::idesc_tf32(128, NT);
+            const uint32_t a_lbo = (uint32_t)p.TH * p.COLS * 16;
+            const uint32_t b_lbo = NT * 16;
+            int it = 0, j = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++j) {
+                const int buf = j & 1, ub = j >> 1;
+                if (ub > 0 && !dev::mbar_wait_bounded(&acce[buf], (ub - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                dev::tc_fence_after();
+                const uint32_t dbase = tmem + (uint32_t)buf * acc_cols;
+                for (int kt = 0; kt < num_k; ++kt, ++it) {
+                    const int slot = it % p.stages;
+                    if (!dev::mbar_wait_bounded(&full[slot], (it / p.stages) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    dev::tc_fence_after();
+                    const unsigned char *st = stages + (size_t)slot * stage_bytes;
+                    const uint64_t dah = dev::smem_desc(st, a_lbo, 128);
+                    const uint64_t dal = dev::smem_desc(st + p.a_bytes, a_lbo, 128);
+                    const uint64_t dbh = dev::smem_desc(st + 2 * p.a_bytes, b_lbo, 128);
+                    const uint64_t dbl = dev::smem_desc(st + 2 * p.a_bytes + p.b_bytes, b_lbo, 128);
+                    for (int i = 0; i < p.TH; ++i) {
+                        const uint32_t d = dbase + (uint32_t)(i * NT);
+                        for (int s = 0; s < p.S; ++s) {
+                            const uint64_t ao = (uint64_t)((i * p.COLS + s * p.dil));   // 16-byte units
+                            const uint64_t bo = (uint64_t)(s * 2 * NT);
+                            const uint32_t acc = (kt > 0 || s > 0) ? 1u : 0u;
+                            dev::mma_tf32(d, dal + ao, dbh + bo, idesc, acc);
+                            dev::mma_tf32(d, dah + ao, dbl + bo, idesc, 1u);
+                            dev::mma_tf32(d, dah + ao, dbh + bo, idesc, 1u);
+                        }
+                    }
+                    dev::mma_commit(&empty[slot]);
+                }
+                dev::mma_commit(&accf[buf]);   // fires once this tile's MMAs have completed
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicExch(&g_igemm_error, 1);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------- epilogue
+        // chain: GroupNorm groups per 16-channel chunk and their width in it
+        constexpr int GPC = CHAIN ? (KGN >= 16 ? 1 : 16 / KGN) : 1;
+        constexpr int GW = CHAIN ? (KGN >= 16 ? 16 : KGN) : 16;
+        const int ew = warp - 2;                 // 0..7
+        const int lq = warp & 3;                 // TMEM lane quarter this warp may access
+        const int chalf = ew >> 2;               // column half
+        constexpr int HALF = NT / 2;
+        const int m = lq * 32 + lane;
+        const long long plane = (long long)p.P * p.Q;
+        int j = 0;
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++j) {
+            const IgTile tl = ig_tile(p, t);
+            const int buf = j & 1;
+            // after an abort nothing more will be committed: do not wait for it
+            const bool have = !*(volatile int *)abort_flag && dev::mbar_wait_bounded(&accf[buf], (j >> 1) & 1);
+            if (!have) atomicExch(&g_igemm_error, 1);
+            dev::tc_fence_after();
+            const bool ok = have && !*(volatile int *)abort_flag;
+            const int q = tl.q0 + m;
+            const bool qvalid = q < p.Q;
+            float *ybase = p.y + ((long long)tl.n * p.K + (long long)tl.g * p.kpg) * plane + q;
+            const uint32_t tbase = tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)buf * acc_cols;
+#pragma unroll 1
+            for (int c0 = chalf * HALF; c0 < (chalf + 1) * HALF; c0 += 16) {
+                // z = acc * mul + add: plain (mul 1, add bias) or chain (scale, bias*scale)
+                float mul[16], add[16];
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int k = tl.g * p.kpg + c0 + jj;
+                    const float b = p.bias ? __ldg(p.bias + k) : 0.f;
+                    mul[jj] = CHAIN ? __ldg(p.scale + k) : 1.f;
+                    add[jj] = CHAIN ? b * mul[jj] : b;
+                }
+                float shift[16], s1[16], s2[16];
+                float cnt = 0.f;
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) { shift[jj] = 0.f; s1[jj] = 0.f; s2[jj] = 0.f; }
+                // rows are processed two at a time so one TMEM load latency covers both
+#pragma unroll 1
+                for (int i = 0; i < p.TH; i += 2) {
+                    float vv[2][16];
+                    const bool two = i + 1 < p.TH;
+                    dev::tmem_ld16_pair(tbase + (uint32_t)(i * NT + c0), tbase + (uint32_t)((i + (two ? 1 : 0)) * NT + c0),
+                                        vv[0], vv[1]);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (h == 1 && !two) break;
+                        float *v = vv[h];
+                        const int pp = tl.p0 + i + h;
+                        const bool valid = ok && qvalid && pp < p.P;
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj) {
+                            float z = fmaf(v[jj], mul[jj], add[jj]);
+                            // logistic; the clamp keeps 1 + e finite (e^80 < 2^126)
+                            if constexpr (CHAIN) z = __fdividef(1.f, 1.f + __expf(fminf(-z, 80.f)));
+                            v[jj] = z;
+                        }
+                        if (valid) {
+                            float *yr = ybase + (long long)c0 * plane + (long long)pp * p.Q;
+#pragma unroll
+                            for (int jj = 0; jj < 16; ++jj) yr[(long long)jj * plane] = v[jj];
+                            if constexpr (CHAIN) {
+                                if (cnt == 0.f) {
+#pragma unroll
+                                    for (int jj = 0; jj < 16; ++jj) shift[jj] = v[jj];
+                                }
+                                cnt += 1.f;
+#pragma unroll
+                                for (int jj = 0; jj < 16; ++jj) {
+                                    const float d = v[jj] - shift[jj];
+                                    s1[jj] += d;
+                                    s2[jj] = fmaf(d, d, s2[jj]);
+                                }
+                            }
+                        }
+                    }
+                }
+                if (c0 + 16 >= (chalf + 1) * HALF) {
+                    // last TMEM read of this tile by this warp: hand the buffer back
+                    dev::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&acce[buf]);
+                }
+                if constexpr (CHAIN) {
+                    // per GroupNorm group in this chunk: raw sums (n, sum a, sum a^2) in
+                    // double, combined over the thread's channels, then a fixed
+                    // shuffle tree over the warp's 32 pixels
+#pragma unroll
+                    for (int gg = 0; gg < GPC; ++gg) {
+                        double S1 = 0.0, S2 = 0.0;
+                        if (cnt > 0.f) {
+#pragma unroll
+                            for (int jj = gg * GW; jj < (gg + 1) * GW; ++jj) {
+                                const double a1 = (double)s1[jj];
+                                const double mu = (double)shift[jj] + a1 / cnt;
+                                const double m2 = fmax((double)s2[jj] - a1 * a1 / cnt, 0.0);
+                                S1 += cnt * mu;
+                                S2 += m2 + cnt * mu * mu;
+                            }
+                        }
+                        double Nn = (double)cnt * GW;
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1) {
+                            const double o1 = __shfl_down_sync(0xffffffffu, S1, off);
+                            const double o2 = __shfl_down_sync(0xffffffffu, S2, off);
+                            const double on = __shfl_down_sync(0xffffffffu, Nn, off);
+                            if (lane < off) { S1 += o1; S2 += o2; Nn += on; }
+                        }
+                        if (lane == 0) {
+                            const int fr = (c0 >> 4) * GPC + gg;
+                            st_n[fr * 4 + lq] = Nn;
+                            st_1[fr * 4 + lq] = S1;
+                            st_2[fr * 4 + lq] = S2;
+                        }
+                    }
+                }
+            }
+            if constexpr (CHAIN) {
+                epi_sync();
+                const int et = tid - 64;
+                const int ngroups = NT / p.kgn;
+                if (et < ngroups) {
+                    // fragments of group et: one per group (width <= 16) or kgn/16 chunks
+                    const int f0 = KGN >= 16 ? et * (p.kgn / 16) : et;
+                    const int f1 = KGN >= 16 ? (et + 1) * (p.kgn / 16) : et + 1;
+                    double Nn = 0.0, S1 = 0.0, S2 = 0.0;
+                    for (int fr = f0; fr < f1; ++fr)
+                        for (int l = 0; l < 4; ++l) {
+                            Nn += st_n[fr * 4 + l];
+                            S1 += st_1[fr * 4 + l];
+                            S2 += st_2[fr * 4 + l];
+                        }
+                    const double mean = Nn > 0.0 ? S1 / Nn : 0.0;
+                    const double m2 = Nn > 0.0 ? fmax(S2 - S1 * mean, 0.0) : 0.0;
+                    const int G = (tl.g * p.kpg) / p.kgn + et;
+                    p.gn_part[((long long)tl.n * p.gn_groups + G) * p.slots + tl.sp] =
+                        make_float4((float)Nn, (float)mean, (float)m2, 0.f);
+                }
+                epi_sync();   // statistics scratch free for the next tile
+            }
         }
     }
 
@@ -343,13 +453,28 @@ cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-template <int NT, bool CHAIN>
+template <int NT, int KGN>
 cudaError_t launch_nt(const IgemmParams &p, const TensorMap &tmh, const TensorMap &tml, dim3 grid, size_t smem,
                       cudaStream_t st) {
-    auto kern = igemm_tf32x3_kernel<NT, CHAIN>;
+    auto kern = igemm_tf32x3_kernel<NT, KGN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     return launch_ex(kern, grid, dim3(kIgThreads), smem, st, tmh, tml, p);
+}
+
+template <int NT>
+cudaError_t launch_chain_nt(const IgemmParams &p, const TensorMap &tmh, const TensorMap &tml, dim3 grid,
+                            size_t smem, cudaStream_t st) {
+    switch (p.kgn) {
+        case 1: return launch_nt<NT, 1>(p, tmh, tml, grid, smem, st);
+        case 2: return launch_nt<NT, 2>(p, tmh, tml, grid, smem, st);
+        case 4: return launch_nt<NT, 4>(p, tmh, tml, grid, smem, st);
+        case 8: return launch_nt<NT, 8>(p, tmh, tml, grid, smem, st);
+        case 16: return launch_nt<NT, 16>(p, tmh, tml, grid, smem, st);
+        default:
+            if (p.kgn % 16 == 0) return launch_nt<NT, 32>(p, tmh, tml, grid, smem, st);
+            return cudaErrorInvalidValue;
+    }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -370,17 +495,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 int igemm_supported_nt(int kpg) { return kpg == 32 || kpg == 64 || kpg == 128 || kpg == 256; }
 
-size_t igemm_header_bytes() { return kIgHeader; }
+size_t igemm_header_bytes(int nt, bool chain) { return ig_header(nt, chain); }
 
-bool make_nc4hw4_tensor_map(TensorMap *tm, const float *base, long long quads, int H, int W, int box_cols,
-                            int box_rows) {
+int igemm_threads() { return kIgThreads; }
+
+bool make_nc4hw4_tensor_map(TensorMap *tm, const float *base, long long quads, int H, int W) {
     auto fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[4] = {4, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)quads};
-    cuuint64_t strides[3] = {16, (cuuint64_t)W * 16, (cuuint64_t)W * H * 16};
-    cuuint32_t box[4] = {4, (cuuint32_t)box_cols, (cuuint32_t)box_rows, 2};
-    cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(reinterpret_cast<CUtensorMap *>(tm), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+    // [quads][H][W*4] floats; box = 64 pixels x 4 channels of one row of one quad
+    cuuint64_t dims[3] = {(cuuint64_t)W * 4, (cuuint64_t)H, (cuuint64_t)quads};
+    cuuint64_t strides[2] = {(cuuint64_t)W * 16, (cuuint64_t)W * H * 16};
+    cuuint32_t box[3] = {256, 1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(reinterpret_cast<CUtensorMap *>(tm), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
                     const_cast<float *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -404,15 +531,18 @@ cudaError_t launch_split_w(const float *w, float *wh, float *wl, int K, int cpg,
 
 cudaError_t launch_igemm(const IgemmParams &p, const TensorMap &tmh, const TensorMap &tml, int chain, dim3 grid,
                          size_t smem, cudaStream_t st) {
+    if (chain) {
+        switch (p.kpg) {
+            case 32: return launch_chain_nt<32>(p, tmh, tml, grid, smem, st);
+            case 64: return launch_chain_nt<64>(p, tmh, tml, grid, smem, st);
+            default: return cudaErrorInvalidValue;
+        }
+    }
     switch (p.kpg) {
-        case 32: return chain ? launch_nt<32, true>(p, tmh, tml, grid, smem, st)
-                              : launch_nt<32, false>(p, tmh, tml, grid, smem, st);
-        case 64: return chain ? launch_nt<64, true>(p, tmh, tml, grid, smem, st)
-                              : launch_nt<64, false>(p, tmh, tml, grid, smem, st);
-        case 128: return chain ? launch_nt<128, true>(p, tmh, tml, grid, smem, st)
-                               : launch_nt<128, false>(p, tmh, tml, grid, smem, st);
-        case 256: return chain ? launch_nt<256, true>(p, tmh, tml, grid, smem, st)
-                               : launch_nt<256, false>(p, tmh, tml, grid, smem, st);
+        case 32: return launch_nt<32, 0>(p, tmh, tml, grid, smem, st);
+        case 64: return launch_nt<64, 0>(p, tmh, tml, grid, smem, st);
+        case 128: return launch_nt<128, 0>(p, tmh, tml, grid, smem, st);
+        case 256: return launch_nt<256, 0>(p, tmh, tml, grid, smem, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -296,6 +296,10 @@ CHAINS = [
     (1, 8, 17, 17, 24, 3, 3, 2, 1, 1, 1, 3, 1.0, "random"),      # stride 2
     (1, 6, 15, 16, 12, 5, 3, 1, 1, 1, 2, 4, 1.0, "random"),      # generic geometry
     (2, 8, 40, 40, 32, 3, 3, 1, 0, 1, 1, 8, 3.0, "random"),      # saturating logistic
+    (2, 8, 30, 33, 32, 3, 3, 1, 0, 1, 1, 1, 1.0, "random"),      # one group of all 32 channels
+    (1, 16, 21, 22, 64, 3, 3, 1, 1, 1, 1, 4, 1.0, "random"),     # 64 channels, 16 per group
+    (1, 16, 21, 22, 64, 3, 3, 1, 1, 1, 1, 1, 1.0, "random"),     # 64 channels in one group
+    (1, 16, 19, 140, 64, 3, 3, 1, 1, 1, 1, 32, 1.0, "random"),   # 64 channels, 2 per group
 ]
 
 
