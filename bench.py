@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload depthwise|tiny_grouped|fused_chain|dense_5x9]
-                    [--shapes] [--sweep]
+                    [--no-shapes] [--sweep] [--force-kernel NAME]
 
 One step = one call of the library's entry point on one batch of the
 workload (default: the depthwise conv of a MobileNetV2 inverted-residual
@@ -88,6 +88,41 @@ def stored_traffic(workload: str):
         return float(e["dram_bytes_per_launch"])
     except Exception:
         return None
+
+
+TF32_OVER_BF16 = 1.1 / 2.25      # nominal dense tf32 / bf16 tensor throughput on B200
+
+
+def fp32_peak_tflops():
+    """CUDA-core FP32 peak: 148 SMs x 128 FMA lanes x 2 FLOP x 1965 MHz."""
+    return wl.fp32_fma_peak_tflops()
+
+
+def tensor_3xtf32_peak_tflops(meas):
+    """Useful FP32 FLOP/s ceiling of 3xTF32 on the tensor cores: the measured
+    bf16 GEMM peak x the nominal tf32/bf16 ratio, divided by 3 products."""
+    bf16 = float(meas.get("bf16_tflops", 1590.0)) if meas else 1590.0
+    return bf16 * TF32_OVER_BF16 / 3.0
+
+
+def roofline_for(wk, sec, plan, hbm_peak, meas):
+    """Binding roofline term of one call: HBM bytes, FP32 CUDA-core FLOPs or
+    3xTF32 tensor FLOPs (for the implicit-GEMM plan)."""
+    t_hbm = wk.bytes / (hbm_peak * 1e9)
+    if plan.startswith("igemm"):
+        peak_c = tensor_3xtf32_peak_tflops(meas)
+        bound_c = "tensor"
+    else:
+        peak_c = fp32_peak_tflops()
+        bound_c = "alu"
+    t_cmp = wk.flops / (peak_c * 1e12)
+    if t_hbm >= t_cmp:
+        ach = wk.bytes / sec / 1e9
+        return {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(ach / hbm_peak, 4)}
+    ach = wk.flops / sec / 1e12
+    return {"bound": bound_c, "achieved": round(ach, 2), "peak": round(peak_c, 1), "unit": "TFLOP/s",
+            "frac": round(ach / peak_c, 4)}
 
 
 class ClockSampler:
@@ -390,7 +425,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="depthwise")
-    ap.add_argument("--shapes", action="store_true", help="also time the other page workloads")
+    ap.add_argument("--no-shapes", action="store_true",
+                    help="skip timing the other page workloads (tiny grouped, depthwise, chain, dense)")
     ap.add_argument("--sweep", action="store_true", help="also time the 80-shape sweep")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -427,7 +463,7 @@ def main():
 
     props = torch.cuda.get_device_properties(device)
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
-    hbm_peak, peak_kind, _ = peaks()
+    hbm_peak, peak_kind, meas = peaks()
 
     wk = Workload(args.workload)
     runner = DeviceRunner(wk, device, l2)
@@ -449,16 +485,13 @@ def main():
     e2e_value = wk.bytes * world * args.steps / (e2e_ms / 1e3) / 1e9
     gflops = wk.flops * world * args.steps / (ms / 1e3) / 1e9
 
-    # dominant kernel: the conv kernel (the only one for a plain conv)
-    launch_s = per_step_s if not wk.chain else None
-    achieved = wk.bytes / launch_s / 1e9 if launch_s else None
-    roof = None
-    if achieved is not None:
-        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                "frac": round(achieved / hbm_peak, 4), "traffic": stored_traffic(wk.name),
-                "peak_kind": peak_kind, "kernel": gc.plan_name(
-                    wk.shape.N, wk.shape.C, wk.shape.H, wk.shape.W, wk.shape.K, wk.shape.R,
-                    wk.shape.S, wk.shape.stride, wk.shape.pad, wk.shape.dil, wk.shape.groups)}
+    # dominant kernel: the convolution (the only kernel of a direct plain conv)
+    shp = wk.shape
+    plan = gc.plan_name(shp.N, shp.C, shp.H, shp.W, shp.K, shp.R, shp.S, shp.stride, shp.pad, shp.dil,
+                        shp.groups, wk.chain)
+    roof = roofline_for(wk, per_step_s, plan, hbm_peak, meas)
+    roof.update({"traffic": stored_traffic(wk.name), "peak_kind": peak_kind, "kernel": plan})
+    launches = wk.kernels_per_step + (2 if plan.startswith("igemm") else 0)
 
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
@@ -476,14 +509,14 @@ def main():
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "roofline": roof,
-        "gpu_launches": wk.kernels_per_step * args.steps,
+        "gpu_launches": launches * args.steps,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         "clock_samples": {"n": clocks.get("samples"), "window": clocks.get("window")},
     }
 
-    if args.shapes or args.sweep:
+    if not args.no_shapes or args.sweep:
         extra = {}
-        names = ["tiny_grouped", "depthwise", "fused_chain", "dense_5x9"] if args.shapes else []
+        names = [] if args.no_shapes else ["tiny_grouped", "depthwise", "fused_chain", "dense_5x9"]
         if args.sweep:
             names += [f"sweep{i}" for i in range(80)]
         for nm in names:
@@ -491,14 +524,16 @@ def main():
                 continue
             w2 = Workload(nm)
             r2 = DeviceRunner(w2, device, l2)
-            k2 = max(3, min(args.steps, 50))
+            k2 = max(3, min(args.steps, 20))
             ms2, _, _ = time_graph(r2, k2, 3, barrier)
             sec = ms2 / 1e3 / k2
+            s2 = w2.shape
+            plan2 = gc.plan_name(s2.N, s2.C, s2.H, s2.W, s2.K, s2.R, s2.S, s2.stride, s2.pad, s2.dil,
+                                 s2.groups, w2.chain)
             extra[nm] = {"us": round(sec * 1e6, 3), "GB/s": round(w2.bytes / sec / 1e9, 1),
-                         "GFLOP/s": round(w2.flops / sec / 1e9, 1),
-                         "hbm_frac": round(w2.bytes / sec / 1e9 / hbm_peak, 4),
-                         "fp32_frac": round(w2.flops / sec / 1e12 / wl.fp32_fma_peak_tflops(), 4),
-                         "label": w2.shape.label()}
+                         "GFLOP/s": round(w2.flops / sec / 1e9, 1), "kernel": plan2,
+                         "roofline": roofline_for(w2, sec, plan2, hbm_peak, meas),
+                         "label": s2.label()}
             del r2
             torch.cuda.empty_cache()
         result["shapes"] = extra

@@ -120,9 +120,10 @@ GCONV_API gconv_status_t gconv2d_bias_scale_sigmoid_groupnorm_fwd(
  * stream is being captured), engines that must not stall on an implicit
  * device synchronisation or must keep a fixed memory budget after start-up,
  * and hosts whose allocator is owned by another framework.
- * - Shapes whose partial statistics need more than the capacity
- *   (gconv2d_chain_workspace_size() > capacity) return GCONV_ERR_WORKSPACE
- *   and launch nothing; use the regular entry point for them.
+ * - It always runs the direct (CUDA-core) convolution kernels, whose only
+ *   scratch is the partial statistics; shapes whose partials need more than
+ *   the capacity return GCONV_ERR_WORKSPACE and launch nothing; use the
+ *   regular entry point for them.
  * - The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
  *   before any stream capture.
