@@ -90,6 +90,23 @@ def stored_traffic(workload: str):
         return None
 
 
+def max_over_ranks(values, device, world):
+    """Element-wise maximum of per-rank timings (the job takes as long as its
+    slowest rank); identity on one rank."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def weak_scaling_rate(units_per_step, world, steps, ms):
+    """Whole-job rate: every rank processes `units_per_step` per step."""
+    return units_per_step * world * steps / (ms / 1e3)
+
+
 TF32_OVER_BF16 = 1.1 / 2.25      # nominal dense tf32 / bf16 tensor throughput on B200
 
 
@@ -266,12 +283,15 @@ class DeviceRunner:
         per_set = (h["x"].numel() + s.n_out) * 4
         # one set already larger than L2, or enough sets to cover 4 x L2
         self.n_sets = 1 if per_set >= l2_bytes else math.ceil(4 * l2_bytes / per_set)
-        self.xs = []
-        self.ys = []
-        x0 = h["x"].to(device)
-        for i in range(self.n_sets):
-            self.xs.append(x0 if i == 0 else x0.clone())
-            self.ys.append(torch.empty((s.N, s.K, s.P, s.Q), device=device))
+        # two pooled allocations sliced into per-set views (16-byte aligned slices)
+        xn = (h["x"].numel() + 3) // 4 * 4
+        yn = (s.n_out + 3) // 4 * 4
+        xpool = torch.empty(self.n_sets * xn, device=device)
+        ypool = torch.empty(self.n_sets * yn, device=device)
+        x0 = h["x"].to(device).reshape(-1)
+        xpool.view(self.n_sets, xn)[:, :x0.numel()].copy_(x0.expand(self.n_sets, -1))
+        self.xs = [xpool[i * xn:i * xn + x0.numel()].view(h["x"].shape) for i in range(self.n_sets)]
+        self.ys = [ypool[i * yn:i * yn + s.n_out].view(s.N, s.K, s.P, s.Q) for i in range(self.n_sets)]
         self.pool_bytes = self.n_sets * per_set
         if wk.chain:
             self.bias = (h["b_conv"] + h["b_extra"]).to(device)
@@ -416,6 +436,84 @@ def cpu_oracle_rate(wk: Workload, budget_s: float):
     return gbs, desc, oracle.num_threads()
 
 
+def bootstrap_ci(samples, reps=2000, seed=0):
+    """95% bootstrap interval of the mean of `samples`."""
+    a = np.asarray(samples, dtype=np.float64)
+    rng = np.random.default_rng(seed)
+    means = a[rng.integers(0, len(a), (reps, len(a)))].mean(axis=1)
+    return float(np.percentile(means, 2.5)), float(np.percentile(means, 97.5))
+
+
+def write_records(args, gc, device, l2, hbm_peak, meas, batches=10, per_batch=30):
+    """One record per shape: kernel chosen, status, graph-device and synchronized-API
+    latency (mean over 10 batches of 30 calls, 95% bootstrap interval), GB/s,
+    GFLOP/s and the binding roofline term."""
+    import torch
+    names = ["tiny_grouped", "depthwise", "fused_chain", "dense_5x9"] + [f"sweep{i}" for i in range(80)]
+    out = []
+    for nm in names:
+        wk = Workload(nm)
+        s = wk.shape
+        plan = gc.plan_name(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil, s.groups, wk.chain)
+        rec = {"workload": nm, "shape": s.label(), "kernel": plan, "bytes": wk.bytes, "flops": wk.flops}
+        if plan in ("unsupported", "invalid"):
+            rec["status"] = plan
+            out.append(rec)
+            continue
+        r = DeviceRunner(wk, device, l2)
+        for i in range(3):
+            r.step(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        st = torch.cuda.Stream()
+        st.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(st):
+            with torch.cuda.graph(g, stream=st):
+                for i in range(per_batch):
+                    r.step(i)
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        graph_us = []
+        for b in range(batches):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(st):
+                e0.record(st)
+                g.replay()
+                e1.record(st)
+            torch.cuda.synchronize()
+            graph_us.append(e0.elapsed_time(e1) * 1e3 / per_batch)
+        del g
+        sync_us = []
+        for b in range(batches):
+            lat = []
+            for i in range(per_batch):
+                t0 = time.perf_counter()
+                r.step(i)
+                torch.cuda.current_stream().synchronize()
+                lat.append(time.perf_counter() - t0)
+            sync_us.append(statistics.mean(lat) * 1e6)
+        gm = statistics.mean(graph_us)
+        sm = statistics.mean(sync_us)
+        rec.update({
+            "status": "measured",
+            "graph_us": round(gm, 3), "graph_ci95": [round(v, 3) for v in bootstrap_ci(graph_us)],
+            "sync_us": round(sm, 3), "sync_ci95": [round(v, 3) for v in bootstrap_ci(sync_us)],
+            "GB/s": round(wk.bytes / gm / 1e3, 1), "GFLOP/s": round(wk.flops / gm / 1e3, 1),
+            "roofline": roofline_for(wk, gm * 1e-6, plan, hbm_peak, meas),
+            "pool_sets": r.n_sets,
+        })
+        out.append(rec)
+        del r
+        torch.cuda.empty_cache()
+    with open(args.records, "w") as f:
+        json.dump({"device": torch.cuda.get_device_name(device), "hbm_peak_gbs": hbm_peak,
+                   "kernel_family": args.force_kernel, "batches": batches, "per_batch": per_batch,
+                   "records": out}, f, indent=1)
+    print(json.dumps({"records": len(out), "file": args.records}))
+
+
 # ------------------------------------------------------------------ main
 
 def main():
@@ -429,6 +527,9 @@ def main():
                     help="skip timing the other page workloads (tiny grouped, depthwise, chain, dense)")
     ap.add_argument("--sweep", action="store_true", help="also time the 80-shape sweep")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--records", default=None,
+                    help="write per-shape records (page workloads + 80-shape sweep) to this JSON file "
+                         "and exit: 10 batches x 30 calls per boundary, 95%% bootstrap intervals")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--force-kernel", default="auto",
                     help="kernel family for A/B runs: auto, direct, direct_cpasync, generic, igemm")
@@ -465,6 +566,9 @@ def main():
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
     hbm_peak, peak_kind, meas = peaks()
 
+    if args.records:
+        return write_records(args, gc, device, l2, hbm_peak, meas)
+
     wk = Workload(args.workload)
     runner = DeviceRunner(wk, device, l2)
     sampler = ClockSampler(local_rank)
@@ -474,16 +578,11 @@ def main():
         sync_us = time_sync_api(runner, min(args.steps, 200))
     clocks = sampler.summary(t0, t1)
 
-    # max over ranks
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
-
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], device, world)
     per_step_s = ms / 1e3 / args.steps
-    value = wk.bytes * world * args.steps / (ms / 1e3) / 1e9
-    e2e_value = wk.bytes * world * args.steps / (e2e_ms / 1e3) / 1e9
-    gflops = wk.flops * world * args.steps / (ms / 1e3) / 1e9
+    value = weak_scaling_rate(wk.bytes, world, args.steps, ms) / 1e9
+    e2e_value = weak_scaling_rate(wk.bytes, world, args.steps, e2e_ms) / 1e9
+    gflops = weak_scaling_rate(wk.flops, world, args.steps, ms) / 1e9
 
     # dominant kernel: the convolution (the only kernel of a direct plain conv)
     shp = wk.shape
