@@ -98,6 +98,19 @@ struct DirectPlan {
     size_t smem;
 };
 
+int sm_count() {
+    static const int n = [] {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+            cudaGetLastError();
+            return 148;
+        }
+        return v;
+    }();
+    return n;
+}
+
 // Choose the CTA tile for a direct-kernel launch.  Returns false when no tile
 // fits the shared-memory limit (the shape is then unsupported by this family).
 bool plan_direct(const Shape &s, bool chain, int gn_groups, int geom, bool x_vec, DirectPlan &pl) {
@@ -125,27 +138,56 @@ bool plan_direct(const Shape &s, bool chain, int gn_groups, int geom, bool x_vec
     int KZ = 1;
     for (int z = 1; z <= m; ++z)
         if (m % z == 0 && KT * z <= 32 && CX * z <= kMaxThreads && (!chain || compat(kgn, KT * z))) KZ = z;
-    const int KB = KT * KZ;
-    const int n_kb = s.kpg / KB;
 
     const int strips = ceil_div(s.P, RPT);
-    int ry_max = kMaxThreads / (CX * KZ);
-    if (ry_max < 1) ry_max = 1;
-    int n_pt = ceil_div(strips, ry_max);
-    int RY = ceil_div(strips, n_pt);
-    const int TP = RY * RPT;
+    auto pick_ry = [&](int ry_cap, int &n_pt_out) {
+        int ry_max = std::max(1, std::min(ry_cap, kMaxThreads / (CX * KZ)));
+        n_pt_out = ceil_div(strips, ry_max);
+        return ceil_div(strips, n_pt_out);
+    };
+    int n_pt = 1;
+    int RY = pick_ry(strips, n_pt);
 
     // conv groups per CTA (only when a CTA already holds all channels of a group)
-    int GB = 1;
-    if (n_kb == 1) {
-        const int per = CX * RY * KZ;
-        for (int gcand = 1; gcand <= s.groups; ++gcand) {
-            if (s.groups % gcand) continue;
-            if (per * gcand > kMaxThreads) break;
-            if (chain && !compat(kgn, gcand * s.kpg)) continue;
-            GB = gcand;
+    auto pick_gb = [&](int gb_cap) {
+        int gb = 1;
+        if (s.kpg / (KT * KZ) == 1) {
+            const int per = CX * RY * KZ;
+            for (int gcand = 1; gcand <= std::min(s.groups, gb_cap); ++gcand) {
+                if (s.groups % gcand) continue;
+                if (per * gcand > kMaxThreads) break;
+                if (chain && !compat(kgn, gcand * s.kpg)) continue;
+                gb = gcand;
+            }
+        }
+        return gb;
+    };
+    int GB = pick_gb(s.groups);
+
+    // Small problems: split the work until the grid covers about two CTAs per
+    // SM (fewer groups per CTA, then fewer rows, then fewer channel slices).
+    const long long target = 2LL * sm_count();
+    auto ctas = [&]() {
+        return (long long)s.N * (s.kpg / (KT * KZ)) * (s.groups / GB) * n_qt * n_pt;
+    };
+    for (int guard = 0; guard < 64 && ctas() < target; ++guard) {
+        if (GB > 1) {
+            GB = pick_gb(GB - 1);
+        } else if (RY > 1) {
+            RY = pick_ry((RY + 1) / 2, n_pt);
+        } else if (KZ > 1) {
+            int z = KZ - 1;
+            while (z > 1 && (m % z != 0 || (chain && !compat(kgn, KT * z)))) --z;
+            KZ = z;
+            RY = pick_ry(strips, n_pt);
+            GB = 1;
+        } else {
+            break;
         }
     }
+    const int TP = RY * RPT;
+    const int KB = KT * KZ;
+    const int n_kb = s.kpg / KB;
     const int KBtot = GB * KB;
     if (chain && !compat(kgn, KBtot)) return false;
 
@@ -313,19 +355,6 @@ struct IgemmPlan {
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
-int sm_count() {
-    static const int n = [] {
-        int dev = 0, v = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
-            cudaGetLastError();
-            return 148;
-        }
-        return v;
-    }();
-    return n;
-}
-
 int env_int(const char *name) {
     const char *e = std::getenv(name);
     return e ? std::atoi(e) : 0;
@@ -343,22 +372,30 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     COLS = (COLS + 7) / 8 * 8;   // 128-byte aligned row segments
     if (COLS > 256) return false;
     static const int force_th = env_int("GCONV_IGEMM_TH");
-    static const int force_st = env_int("GCONV_IGEMM_STAGES");
+    static const int force_sa = env_int("GCONV_IGEMM_SA");
+    static const int force_sb = env_int("GCONV_IGEMM_SB");
     // output rows per tile: two accumulator buffers of TH*NT columns fit TMEM
     int TH = std::max(1, std::min(8, 256 / NT));
     if (force_th > 0) TH = force_th;
     TH = std::min(TH, s.P);
+    const size_t limit = 227 * 1024 - igemm_header_bytes(NT, chain);
+    const int b_bytes = 32 * s.S * NT;              // one w operand slice: S taps x 8 channels x NT
+    int AR = 0, a_bytes = 0, sa = 0, sb = 0;
+    for (; TH >= 1; --TH) {
+        AR = TH + (s.R - 1) * s.dil;               // staged rows serving every tap row
+        if (AR > 256) continue;
+        a_bytes = 32 * COLS * AR;                   // one x operand tile: 2 quads x AR x COLS x 16 B
+        sa = force_sa > 0 ? std::min(force_sa, 4) : 2;
+        sb = force_sb > 0 ? std::min(force_sb, 4) : 4;
+        while (sb > 2 && (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes > limit) --sb;
+        while (sa > 1 && (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes > limit) --sa;
+        while (sb > 1 && (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes > limit) --sb;
+        if ((size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes <= limit) break;
+    }
+    if (TH < 1) return false;
     int tmem_cols = 32;
     while (tmem_cols < 2 * TH * NT) tmem_cols *= 2;
     if (tmem_cols > 512) return false;
-    const int a_bytes = 32 * COLS * TH;
-    const int b_bytes = 32 * s.S * NT;
-    const size_t stage = 2 * (size_t)a_bytes + 2 * (size_t)b_bytes;
-    int stages = 4;
-    if (force_st > 0) stages = std::min(force_st, 8);
-    const size_t limit = 227 * 1024 - igemm_header_bytes(NT, chain);
-    while (stages > 1 && stages * stage > limit) --stages;
-    if (stages * stage > limit) return false;
 
     IgemmParams &p = pl.prm;
     std::memset(&p, 0, sizeof(p));
@@ -372,7 +409,9 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     const long long n_tiles = (long long)s.N * s.groups * p.n_qt * p.n_pt;
     if (n_tiles > 0x7fffffffLL) return false;
     p.n_tiles = (int)n_tiles;
-    p.stages = stages;
+    p.AR = AR;
+    p.sa = sa;
+    p.sb = sb;
     p.a_bytes = a_bytes;
     p.b_bytes = b_bytes;
     p.tmem_cols = tmem_cols;
@@ -380,7 +419,7 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     p.kgn = kgn;
     p.slots = p.n_qt * p.n_pt;
     pl.grid = dim3((unsigned)std::min<long long>(n_tiles, sm_count()));
-    pl.smem = igemm_header_bytes(NT, chain) + stages * stage;
+    pl.smem = igemm_header_bytes(NT, chain) + (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes;
 
     const size_t xbytes = (size_t)s.N * s.C * s.H * s.W * sizeof(float);
     const size_t wbytes = (size_t)s.K * s.cpg * s.R * s.S * sizeof(float);
@@ -416,8 +455,12 @@ gconv_status_t run_igemm(const Shape &s, IgemmPlan &pl, const float *x, const fl
     float *wl = reinterpret_cast<float *>(base + pl.off_wl);
     IgemmParams &p = pl.prm;
     const long long quads = (long long)s.N * (s.C / 4);
-    TensorMap tmh, tml;
-    if (!make_nc4hw4_tensor_map(&tmh, xh, quads, s.H, s.W) || !make_nc4hw4_tensor_map(&tml, xl, quads, s.H, s.W))
+    TensorMap tm[4];
+    const int tail = p.COLS % 64;
+    if (!make_nc4hw4_tensor_map(&tm[0], xh, quads, s.H, s.W, 64) ||
+        !make_nc4hw4_tensor_map(&tm[1], xl, quads, s.H, s.W, 64) ||
+        !make_nc4hw4_tensor_map(&tm[2], xh, quads, s.H, s.W, tail > 0 ? tail : 64) ||
+        !make_nc4hw4_tensor_map(&tm[3], xl, quads, s.H, s.W, tail > 0 ? tail : 64))
         return GCONV_ERR_UNSUPPORTED;
     p.wh = reinterpret_cast<const float4 *>(wh);
     p.wl = reinterpret_cast<const float4 *>(wl);
@@ -428,7 +471,7 @@ gconv_status_t run_igemm(const Shape &s, IgemmPlan &pl, const float *x, const fl
     p.gn_part = chain ? reinterpret_cast<float4 *>(base + pl.off_part) : nullptr;
     if (launch_split_x(x, xh, xl, s.N, s.C, s.H, s.W, stream) != cudaSuccess) return GCONV_ERR_CUDA;
     if (launch_split_w(w, wh, wl, s.K, s.cpg, s.R, s.S, s.groups, stream) != cudaSuccess) return GCONV_ERR_CUDA;
-    if (launch_igemm(p, tmh, tml, chain ? 1 : 0, pl.grid, pl.smem, stream) != cudaSuccess) return GCONV_ERR_CUDA;
+    if (launch_igemm(p, tm, chain ? 1 : 0, pl.grid, pl.smem, stream) != cudaSuccess) return GCONV_ERR_CUDA;
     if (!chain) return GCONV_OK;
     GnParams g;
     g.y = y;

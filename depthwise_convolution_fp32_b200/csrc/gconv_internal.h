@@ -98,12 +98,13 @@ struct IgemmParams {
     float4 *gn_part;           // chain only
     int N, C, H, W, K, R, S, pad, dil, groups, cpg, kpg, P, Q;
     int CC8;                   // cpg / 8 (K-steps of 8 channels)
-    int TH;                    // output rows per CTA (one 128-pixel M tile each)
+    int TH;                    // output rows per tile (one 128-pixel M tile each)
+    int AR;                    // staged x rows per channel step: TH + (R-1)*dil
     int COLS;                  // staged columns per row (>= 128 + (S-1)*dil, multiple of 8)
     int n_qt, n_pt;
     int n_tiles;               // N * groups * n_pt * n_qt
-    int stages;                // shared-memory pipeline depth
-    int a_bytes, b_bytes;      // one x operand (hi or lo) / one w operand per stage
+    int sa, sb;                // slots of the x-tile ring and of the weight-slice ring
+    int a_bytes, b_bytes;      // one x operand (hi or lo) tile / one w operand slice
     int tmem_cols;
     int gn_groups, kgn, slots;
 };
@@ -112,13 +113,14 @@ int igemm_supported_nt(int kpg);
 size_t igemm_header_bytes(int nt, bool chain);
 int igemm_threads();
 // 3-D tensor map over an NC4HW4 tensor viewed as [quads][H][W*4] floats with
-// a box of 256 floats (64 pixels of one row of one channel quad).
-bool make_nc4hw4_tensor_map(TensorMap *tm, const float *base, long long quads, int H, int W);
+// a box of box_px (<= 64) pixels of one row of one channel quad.
+bool make_nc4hw4_tensor_map(TensorMap *tm, const float *base, long long quads, int H, int W, int box_px);
 cudaError_t launch_split_x(const float *x, float *xh, float *xl, int N, int C, int H, int W, cudaStream_t st);
 cudaError_t launch_split_w(const float *w, float *wh, float *wl, int K, int cpg, int R, int S, int groups,
                            cudaStream_t st);
-cudaError_t launch_igemm(const IgemmParams &p, const TensorMap &tmh, const TensorMap &tml, int chain, dim3 grid,
-                         size_t smem, cudaStream_t st);
+// tm: x_hi 64-pixel map, x_lo 64-pixel map, x_hi tail map, x_lo tail map
+cudaError_t launch_igemm(const IgemmParams &p, const TensorMap *tm, int chain, dim3 grid, size_t smem,
+                         cudaStream_t st);
 int read_and_clear_igemm_error();
 
 cudaError_t launch_gn_finalize(const GnParams &p, cudaStream_t stream);

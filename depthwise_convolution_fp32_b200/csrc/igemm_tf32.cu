@@ -145,14 +145,17 @@ __device__ __forceinline__ IgTile ig_tile(const IgemmParams &p, int t) {
 template <int NT, int KGN>
 __global__ void __launch_bounds__(kIgThreads, 1)
     igemm_tf32x3_kernel(const __grid_constant__ TensorMap tmh, const __grid_constant__ TensorMap tml,
+                        const __grid_constant__ TensorMap tmh_tail, const __grid_constant__ TensorMap tml_tail,
                         const IgemmParams p) {
     extern __shared__ __align__(1024) unsigned char smem[];
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem);   // [stages]
-    uint64_t *empty = full + 8;                             // [stages]
-    uint64_t *accf = full + 16;                             // [2] accumulator ready
-    uint64_t *acce = full + 18;                             // [2] accumulator drained
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(full + 20);
-    int *abort_flag = reinterpret_cast<int *>(full + 21);
+    uint64_t *fullA = reinterpret_cast<uint64_t *>(smem);  // [4] x tiles (hi and lo) landed
+    uint64_t *emptyA = fullA + 4;                           // [4] x tile slot free
+    uint64_t *fullB = fullA + 8;                            // [4] weight slices landed
+    uint64_t *emptyB = fullA + 12;                          // [4] weight slice slot free
+    uint64_t *accf = fullA + 16;                            // [2] accumulator ready
+    uint64_t *acce = fullA + 18;                            // [2] accumulator drained
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(fullA + 20);
+    int *abort_flag = reinterpret_cast<int *>(fullA + 21);
     constexpr bool CHAIN = KGN > 0;
     double *st_n = reinterpret_cast<double *>(smem + 256);   // [fragment][4] chain statistics
     double *st_1 = st_n + NT * 4;
@@ -161,15 +164,19 @@ __global__ void __launch_bounds__(kIgThreads, 1)
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int num_k = p.CC8 * p.R;
     const int num_tiles = p.n_tiles;
-    const uint32_t stage_bytes = 2u * p.a_bytes + 2u * p.b_bytes;
+    const uint32_t a_slot = 2u * p.a_bytes;   // x_hi + x_lo tile of one channel step
+    const uint32_t b_slot = 2u * p.b_bytes;   // w_hi + w_lo slice of one (channel step, tap row)
+    unsigned char *ringA = stages;
+    unsigned char *ringB = stages + (size_t)p.sa * a_slot;
     const uint32_t acc_cols = (uint32_t)(p.TH * NT);
 
     if (tid == 0) {
-        for (int s = 0; s < p.stages; ++s) {
-            dev::mbar_init(&full[s], 1);
-            dev::mbar_init(&empty[s], 1);
+        for (int s = 0; s < 4; ++s) {
+            dev::mbar_init(&fullA[s], 1);
+            dev::mbar_init(&emptyA[s], 1);
+            dev::mbar_init(&fullB[s], 1);
+            dev::mbar_init(&emptyB[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             dev::mbar_init(&accf[b], 1);
@@ -192,45 +199,56 @@ __global__ void __launch_bounds__(kIgThreads, 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
-        // Each staged row segment of one channel quad is contiguous in the
-        // NC4HW4 tensor; it is fetched as boxes of 64 pixels (1 KB), the last
-        // one aligned to the row end (overlapping the previous box), so the
-        // whole warp issues a few dozen 1 KB TMA loads per stage.
-        const int nseg = (p.COLS + 63) / 64;
-        const int per_op = 2 * p.TH * nseg;                 // boxes per x operand
-        const uint32_t tx = (uint32_t)(2 * per_op * 1024 + 2 * p.b_bytes);
-        int it = 0;
+        // Per tile and 8-channel step: one x tile of AR = TH + (R-1)*dil rows
+        // (hi and lo, exact-width boxes: 64-pixel boxes plus one tail box per
+        // row) serving every tap row, then R weight slices (one per tap row).
+        const int nmain = p.COLS / 64;
+        const int tail = p.COLS - nmain * 64;               // pixels, multiple of 8
+        const int per_row = nmain + (tail > 0 ? 1 : 0);
+        const int boxes = 2 * 2 * p.AR * per_row;           // (hi, lo) x quads x rows x segments
+        int ia = 0, ib = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
             const IgTile tl = ig_tile(p, t);
             const int z0 = tl.n * (p.C / 4) + tl.g * (p.cpg / 4);
-            for (int kt = 0; kt < num_k; ++kt, ++it) {
-                const int slot = it % p.stages;
-                const int use = it / p.stages;
+            for (int cc8 = 0; cc8 < p.CC8 && ok; ++cc8, ++ia) {
+                const int sa = ia % p.sa, ua = ia / p.sa;
                 if (lane == 0) {
-                    if (use > 0 && !dev::mbar_wait_bounded(&empty[slot], (use - 1) & 1)) ok = false;
+                    if (ua > 0 && !dev::mbar_wait_bounded(&emptyA[sa], (ua - 1) & 1)) ok = false;
                     if (*(volatile int *)abort_flag) ok = false;
-                    if (ok) dev::mbar_arrive_expect_tx(&full[slot], tx);
+                    if (ok) dev::mbar_arrive_expect_tx(&fullA[sa], a_slot);
                 }
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 if (!ok) break;
-                const int cc8 = kt / p.R, r = kt - cc8 * p.R;
-                unsigned char *st = stages + (size_t)slot * stage_bytes;
-                const int x0 = tl.q0 - p.pad, y0 = tl.p0 - p.pad + r * p.dil, cz = z0 + cc8 * 2;
-                for (int b = lane; b < 2 * per_op; b += 32) {
-                    const int lo = b >= per_op;
-                    const int bb = b - lo * per_op;
-                    const int seg = bb % nseg;
-                    const int row = (bb / nseg) % p.TH;
-                    const int quad = bb / (nseg * p.TH);
-                    const int px = seg < nseg - 1 ? seg * 64 : p.COLS - 64;
-                    unsigned char *dst = st + lo * p.a_bytes + ((size_t)(quad * p.TH + row) * p.COLS + px) * 16;
-                    dev::tma_load_3d(dst, lo ? &tml : &tmh, &full[slot], (x0 + px) * 4, y0 + row, cz + quad);
+                unsigned char *st = ringA + (size_t)sa * a_slot;
+                const int x0 = tl.q0 - p.pad, y0 = tl.p0 - p.pad, cz = z0 + cc8 * 2;
+                for (int b = lane; b < boxes; b += 32) {
+                    const int seg = b % per_row;
+                    int rest = b / per_row;
+                    const int row = rest % p.AR; rest /= p.AR;
+                    const int quad = rest & 1;
+                    const int lo = rest >> 1;
+                    const int px = seg * 64;
+                    unsigned char *dst = st + lo * p.a_bytes + ((size_t)(quad * p.AR + row) * p.COLS + px) * 16;
+                    const void *map = seg < nmain ? (lo ? (const void *)&tml : (const void *)&tmh)
+                                                  : (lo ? (const void *)&tml_tail : (const void *)&tmh_tail);
+                    dev::tma_load_3d(dst, map, &fullA[sa], (x0 + px) * 4, y0 + row, cz + quad);
                 }
-                if (lane == 0) {
-                    const long long woff = (((long long)tl.g * p.CC8 + cc8) * p.R + r) * (p.b_bytes / 16);
-                    dev::bulk_load(st + 2 * p.a_bytes, p.wh + woff, p.b_bytes, &full[slot]);
-                    dev::bulk_load(st + 2 * p.a_bytes + p.b_bytes, p.wl + woff, p.b_bytes, &full[slot]);
+                for (int r = 0; r < p.R; ++r, ++ib) {
+                    const int sb = ib % p.sb, ub = ib / p.sb;
+                    if (lane == 0) {
+                        if (ub > 0 && !dev::mbar_wait_bounded(&emptyB[sb], (ub - 1) & 1)) ok = false;
+                        if (*(volatile int *)abort_flag) ok = false;
+                        if (ok) {
+                            dev::mbar_arrive_expect_tx(&fullB[sb], b_slot);
+                            unsigned char *wb = ringB + (size_t)sb * b_slot;
+                            const long long woff = (((long long)tl.g * p.CC8 + cc8) * p.R + r) * (p.b_bytes / 16);
+                            dev::bulk_load(wb, p.wh + woff, p.b_bytes, &fullB[sb]);
+                            dev::bulk_load(wb + p.b_bytes, p.wl + woff, p.b_bytes, &fullB[sb]);
+                        }
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                    if (!ok) break;
                 }
             }
         }
@@ -243,42 +261,53 @@ __global__ void __launch_bounds__(kIgThreads, 1)
         if (lane == 0) {
             // ------------------------------------------------------ MMA issuer
             constexpr uint32_t idesc = dev::idesc_tf32(128, NT);
-            const uint32_t a_lbo = (uint32_t)p.TH * p.COLS * 16;
+            const uint32_t a_lbo = (uint32_t)p.AR * p.COLS * 16;   // one channel quad apart
             const uint32_t b_lbo = NT * 16;
-            int it = 0, j = 0;
+            int ia = 0, ib = 0, j = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++j) {
-                const int buf = j & 1, ub = j >> 1;
-                if (ub > 0 && !dev::mbar_wait_bounded(&acce[buf], (ub - 1) & 1)) {
+                const int buf = j & 1, ubuf = j >> 1;
+                if (ubuf > 0 && !dev::mbar_wait_bounded(&acce[buf], (ubuf - 1) & 1)) {
                     ok = false;
                     break;
                 }
                 dev::tc_fence_after();
                 const uint32_t dbase = tmem + (uint32_t)buf * acc_cols;
-                for (int kt = 0; kt < num_k; ++kt, ++it) {
-                    const int slot = it % p.stages;
-                    if (!dev::mbar_wait_bounded(&full[slot], (it / p.stages) & 1)) {
+                for (int cc8 = 0; cc8 < p.CC8 && ok; ++cc8, ++ia) {
+                    const int sa = ia % p.sa;
+                    if (!dev::mbar_wait_bounded(&fullA[sa], (ia / p.sa) & 1)) {
                         ok = false;
                         break;
                     }
                     dev::tc_fence_after();
-                    const unsigned char *st = stages + (size_t)slot * stage_bytes;
-                    const uint64_t dah = dev::smem_desc(st, a_lbo, 128);
-                    const uint64_t dal = dev::smem_desc(st + p.a_bytes, a_lbo, 128);
-                    const uint64_t dbh = dev::smem_desc(st + 2 * p.a_bytes, b_lbo, 128);
-                    const uint64_t dbl = dev::smem_desc(st + 2 * p.a_bytes + p.b_bytes, b_lbo, 128);
-                    for (int i = 0; i < p.TH; ++i) {
-                        const uint32_t d = dbase + (uint32_t)(i * NT);
-                        for (int s = 0; s < p.S; ++s) {
-                            const uint64_t ao = (uint64_t)((i * p.COLS + s * p.dil));   // 16-byte units
-                            const uint64_t bo = (uint64_t)(s * 2 * NT);
-                            const uint32_t acc = (kt > 0 || s > 0) ? 1u : 0u;
-                            dev::mma_tf32(d, dal + ao, dbh + bo, idesc, acc);
-                            dev::mma_tf32(d, dah + ao, dbl + bo, idesc, 1u);
-                            dev::mma_tf32(d, dah + ao, dbh + bo, idesc, 1u);
+                    const unsigned char *xa = ringA + (size_t)sa * a_slot;
+                    const uint64_t dah = dev::smem_desc(xa, a_lbo, 128);
+                    const uint64_t dal = dev::smem_desc(xa + p.a_bytes, a_lbo, 128);
+                    for (int r = 0; r < p.R; ++r, ++ib) {
+                        const int sb = ib % p.sb;
+                        if (!dev::mbar_wait_bounded(&fullB[sb], (ib / p.sb) & 1)) {
+                            ok = false;
+                            break;
                         }
+                        dev::tc_fence_after();
+                        const unsigned char *wb = ringB + (size_t)sb * b_slot;
+                        const uint64_t dbh = dev::smem_desc(wb, b_lbo, 128);
+                        const uint64_t dbl = dev::smem_desc(wb + p.b_bytes, b_lbo, 128);
+                        for (int i = 0; i < p.TH; ++i) {
+                            const uint32_t d = dbase + (uint32_t)(i * NT);
+                            for (int s = 0; s < p.S; ++s) {
+                                // 16-byte units: staged row i + r*dil, column s*dil
+                                const uint64_t ao = (uint64_t)((i + r * p.dil) * p.COLS + s * p.dil);
+                                const uint64_t bo = (uint64_t)(s * 2 * NT);
+                                const uint32_t acc = (cc8 > 0 || r > 0 || s > 0) ? 1u : 0u;
+                                dev::mma_tf32(d, dal + ao, dbh + bo, idesc, acc);
+                                dev::mma_tf32(d, dah + ao, dbl + bo, idesc, 1u);
+                                dev::mma_tf32(d, dah + ao, dbh + bo, idesc, 1u);
+                            }
+                        }
+                        dev::mma_commit(&emptyB[sb]);
                     }
-                    dev::mma_commit(&empty[slot]);
+                    dev::mma_commit(&emptyA[sa]);
                 }
                 dev::mma_commit(&accf[buf]);   // fires once this tile's MMAs have completed
             }
@@ -323,10 +352,12 @@ __global__ void __launch_bounds__(kIgThreads, 1)
                     mul[jj] = CHAIN ? __ldg(p.scale + k) : 1.f;
                     add[jj] = CHAIN ? b * mul[jj] : b;
                 }
-                float shift[16], s1[16], s2[16];
+                // shifted sums per GroupNorm group of this chunk (shift = the
+                // group's first value seen by this thread)
+                float shift[GPC], s1[GPC], s2[GPC];
                 float cnt = 0.f;
 #pragma unroll
-                for (int jj = 0; jj < 16; ++jj) { shift[jj] = 0.f; s1[jj] = 0.f; s2[jj] = 0.f; }
+                for (int gg = 0; gg < GPC; ++gg) { shift[gg] = 0.f; s1[gg] = 0.f; s2[gg] = 0.f; }
                 // rows are processed two at a time so one TMEM load latency covers both
 #pragma unroll 1
                 for (int i = 0; i < p.TH; i += 2) {
@@ -354,14 +385,14 @@ __global__ void __launch_bounds__(kIgThreads, 1)
                             if constexpr (CHAIN) {
                                 if (cnt == 0.f) {
 #pragma unroll
-                                    for (int jj = 0; jj < 16; ++jj) shift[jj] = v[jj];
+                                    for (int gg = 0; gg < GPC; ++gg) shift[gg] = v[gg * GW];
                                 }
                                 cnt += 1.f;
 #pragma unroll
                                 for (int jj = 0; jj < 16; ++jj) {
-                                    const float d = v[jj] - shift[jj];
-                                    s1[jj] += d;
-                                    s2[jj] = fmaf(d, d, s2[jj]);
+                                    const float d = v[jj] - shift[jj / GW];
+                                    s1[jj / GW] += d;
+                                    s2[jj / GW] = fmaf(d, d, s2[jj / GW]);
                                 }
                             }
                         }
@@ -381,14 +412,12 @@ __global__ void __launch_bounds__(kIgThreads, 1)
                     for (int gg = 0; gg < GPC; ++gg) {
                         double S1 = 0.0, S2 = 0.0;
                         if (cnt > 0.f) {
-#pragma unroll
-                            for (int jj = gg * GW; jj < (gg + 1) * GW; ++jj) {
-                                const double a1 = (double)s1[jj];
-                                const double mu = (double)shift[jj] + a1 / cnt;
-                                const double m2 = fmax((double)s2[jj] - a1 * a1 / cnt, 0.0);
-                                S1 += cnt * mu;
-                                S2 += m2 + cnt * mu * mu;
-                            }
+                            const double n = (double)cnt * GW;
+                            const double a1 = (double)s1[gg];
+                            const double mu = (double)shift[gg] + a1 / n;
+                            const double m2 = fmax((double)s2[gg] - a1 * a1 / n, 0.0);
+                            S1 = n * mu;
+                            S2 = m2 + n * mu * mu;
                         }
                         double Nn = (double)cnt * GW;
 #pragma unroll
@@ -454,25 +483,24 @@ cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_
 }
 
 template <int NT, int KGN>
-cudaError_t launch_nt(const IgemmParams &p, const TensorMap &tmh, const TensorMap &tml, dim3 grid, size_t smem,
-                      cudaStream_t st) {
+cudaError_t launch_nt(const IgemmParams &p, const TensorMap *tm, dim3 grid, size_t smem, cudaStream_t st) {
     auto kern = igemm_tf32x3_kernel<NT, KGN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_ex(kern, grid, dim3(kIgThreads), smem, st, tmh, tml, p);
+    return launch_ex(kern, grid, dim3(kIgThreads), smem, st, tm[0], tm[1], tm[2], tm[3], p);
 }
 
 template <int NT>
-cudaError_t launch_chain_nt(const IgemmParams &p, const TensorMap &tmh, const TensorMap &tml, dim3 grid,
-                            size_t smem, cudaStream_t st) {
+cudaError_t launch_chain_nt(const IgemmParams &p, const TensorMap *tm, dim3 grid, size_t smem,
+                            cudaStream_t st) {
     switch (p.kgn) {
-        case 1: return launch_nt<NT, 1>(p, tmh, tml, grid, smem, st);
-        case 2: return launch_nt<NT, 2>(p, tmh, tml, grid, smem, st);
-        case 4: return launch_nt<NT, 4>(p, tmh, tml, grid, smem, st);
-        case 8: return launch_nt<NT, 8>(p, tmh, tml, grid, smem, st);
-        case 16: return launch_nt<NT, 16>(p, tmh, tml, grid, smem, st);
+        case 1: return launch_nt<NT, 1>(p, tm, grid, smem, st);
+        case 2: return launch_nt<NT, 2>(p, tm, grid, smem, st);
+        case 4: return launch_nt<NT, 4>(p, tm, grid, smem, st);
+        case 8: return launch_nt<NT, 8>(p, tm, grid, smem, st);
+        case 16: return launch_nt<NT, 16>(p, tm, grid, smem, st);
         default:
-            if (p.kgn % 16 == 0) return launch_nt<NT, 32>(p, tmh, tml, grid, smem, st);
+            if (p.kgn % 16 == 0) return launch_nt<NT, 32>(p, tm, grid, smem, st);
             return cudaErrorInvalidValue;
     }
 }
@@ -499,13 +527,13 @@ size_t igemm_header_bytes(int nt, bool chain) { return ig_header(nt, chain); }
 
 int igemm_threads() { return kIgThreads; }
 
-bool make_nc4hw4_tensor_map(TensorMap *tm, const float *base, long long quads, int H, int W) {
+bool make_nc4hw4_tensor_map(TensorMap *tm, const float *base, long long quads, int H, int W, int box_px) {
     auto fn = encode_fn();
-    if (!fn) return false;
-    // [quads][H][W*4] floats; box = 64 pixels x 4 channels of one row of one quad
+    if (!fn || box_px <= 0 || box_px > 64) return false;
+    // [quads][H][W*4] floats; box = box_px pixels x 4 channels of one row of one quad
     cuuint64_t dims[3] = {(cuuint64_t)W * 4, (cuuint64_t)H, (cuuint64_t)quads};
     cuuint64_t strides[2] = {(cuuint64_t)W * 16, (cuuint64_t)W * H * 16};
-    cuuint32_t box[3] = {256, 1, 1};
+    cuuint32_t box[3] = {(cuuint32_t)box_px * 4, 1, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(reinterpret_cast<CUtensorMap *>(tm), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
                     const_cast<float *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -529,20 +557,20 @@ cudaError_t launch_split_w(const float *w, float *wh, float *wl, int K, int cpg,
                      reinterpret_cast<float4 *>(wl), kpg, cpg, R, S, cells);
 }
 
-cudaError_t launch_igemm(const IgemmParams &p, const TensorMap &tmh, const TensorMap &tml, int chain, dim3 grid,
-                         size_t smem, cudaStream_t st) {
+cudaError_t launch_igemm(const IgemmParams &p, const TensorMap *tm, int chain, dim3 grid, size_t smem,
+                         cudaStream_t st) {
     if (chain) {
         switch (p.kpg) {
-            case 32: return launch_chain_nt<32>(p, tmh, tml, grid, smem, st);
-            case 64: return launch_chain_nt<64>(p, tmh, tml, grid, smem, st);
+            case 32: return launch_chain_nt<32>(p, tm, grid, smem, st);
+            case 64: return launch_chain_nt<64>(p, tm, grid, smem, st);
             default: return cudaErrorInvalidValue;
         }
     }
     switch (p.kpg) {
-        case 32: return launch_nt<32, 0>(p, tmh, tml, grid, smem, st);
-        case 64: return launch_nt<64, 0>(p, tmh, tml, grid, smem, st);
-        case 128: return launch_nt<128, 0>(p, tmh, tml, grid, smem, st);
-        case 256: return launch_nt<256, 0>(p, tmh, tml, grid, smem, st);
+        case 32: return launch_nt<32, 0>(p, tm, grid, smem, st);
+        case 64: return launch_nt<64, 0>(p, tm, grid, smem, st);
+        case 128: return launch_nt<128, 0>(p, tm, grid, smem, st);
+        case 256: return launch_nt<256, 0>(p, tm, grid, smem, st);
         default: return cudaErrorInvalidValue;
     }
 }
