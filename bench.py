@@ -115,19 +115,21 @@ def fp32_peak_tflops():
     return wl.fp32_fma_peak_tflops()
 
 
-def tensor_3xtf32_peak_tflops(meas):
-    """Useful FP32 FLOP/s ceiling of 3xTF32 on the tensor cores: the measured
-    bf16 GEMM peak x the nominal tf32/bf16 ratio, divided by 3 products."""
+def tensor_fp32_peak_tflops(meas):
+    """Useful FP32 FLOP/s ceiling of the tensor-core path: each multiply-add
+    costs one tf32 MAC (main term) plus two bf16 MACs (the two cross terms,
+    one K=16 bf16 MMA per 8 channels).  With the measured bf16 GEMM peak and
+    the nominal tf32/bf16 ratio r, the ceiling is bf16 / (1/r + 2)."""
     bf16 = float(meas.get("bf16_tflops", 1590.0)) if meas else 1590.0
-    return bf16 * TF32_OVER_BF16 / 3.0
+    return bf16 / (1.0 / TF32_OVER_BF16 + 2.0)
 
 
 def roofline_for(wk, sec, plan, hbm_peak, meas):
     """Binding roofline term of one call: HBM bytes, FP32 CUDA-core FLOPs or
-    3xTF32 tensor FLOPs (for the implicit-GEMM plan)."""
+    the tensor-core FP32-accurate ceiling (for the implicit-GEMM plan)."""
     t_hbm = wk.bytes / (hbm_peak * 1e9)
     if plan.startswith("igemm"):
-        peak_c = tensor_3xtf32_peak_tflops(meas)
+        peak_c = tensor_fp32_peak_tflops(meas)
         bound_c = "tensor"
     else:
         peak_c = fp32_peak_tflops()

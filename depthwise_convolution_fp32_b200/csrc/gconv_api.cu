@@ -551,7 +551,7 @@ const char *gconv2d_plan_name(int N, int C, int H, int W, int K, int R, int S, i
     if (st == GCONV_ERR_INVALID_ARG) return "invalid";
     if (st != GCONV_OK) return "unsupported";
     IgemmPlan ig;
-    if (use_igemm(s, chain != 0, chain ? s.K : 1, ig)) return "igemm_tf32x3";
+    if (use_igemm(s, chain != 0, chain ? s.K : 1, ig)) return "igemm_tf32_bf16x";
     DirectPlan pl;
     int gn = 1;
     if (!choose_direct(s, chain != 0, gn, s.W % 4 == 0, pl)) return "unsupported";

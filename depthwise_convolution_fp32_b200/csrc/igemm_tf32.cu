@@ -6,14 +6,21 @@
 // channels of a group, K = C/groups * R * S):
 //   y[n,k,p,q] = bias[k] + sum_{c,r,s} w[k,c,r,s] * x[n, gi*cpg + c, p - pad + r*dil, q - pad + s*dil]
 // in FP32 accuracy: every operand v is split into v_hi = tf32(v) and
-// v_lo = v - v_hi (exact in FP32), and each product is accumulated as
-// a_lo*b_hi + a_hi*b_lo + a_hi*b_hi in FP32 (the dropped a_lo*b_lo term is
-// below 2^-22 of |a*b|).  TF32 on its own (2^-11 relative) would miss the
-// 1e-5 * sum|w*x| bound; the pages flag TF32 as "not exactly fp32".
+// v_lo = v - v_hi (exact in FP32).  Each product is accumulated in FP32 as
+// a_hi*b_hi (a tf32 MMA) plus the two cross terms a_hi*b_lo + a_lo*b_hi,
+// which are 2^-11 smaller and need only a few bits: they run as ONE bf16 MMA
+// over K = 16 (the 8 channels' [bf16(a_hi), bf16(a_lo)] against
+// [bf16(b_lo), bf16(b_hi)]), at twice the tf32 rate and half the operand
+// bytes.  Error per product: bf16 rounding of the cross-term operands
+// (<= 2^-20 |a*b| each) plus the dropped a_lo*b_lo (<= 2^-22 |a*b|), about
+// 2e-6 |a*b| at most, against the 1e-5 * sum|w*x| bound.  TF32 on its own
+// (2^-11 relative) would miss that bound; the pages flag TF32 as "not
+// exactly fp32".
 //
-// Data layout.  A prep pass writes x_hi and x_lo as NC4HW4 ([n][c/4][h][w][4]:
-// four consecutive channels in one 16-byte cell) and the weights, split the
-// same way, as [g][c/8][r][s][2][kpg][4].  In the NC4HW4 tile a CTA stages
+// Data layout.  A prep pass writes x_hi as NC4HW4 ([n][c/4][h][w][4]: four
+// consecutive channels in one 16-byte cell) and the bf16 cross-term operand
+// as [n][c/8][2][h][w][8] (same cell geometry), and the weights split the
+// same way as [g][c/8][r][s][2][kpg][4 tf32 | 8 bf16].  In the NC4HW4 tile a CTA stages
 // ([2 channel quads][rows][cols][4]), consecutive output pixels of one row
 // are 16 bytes apart, which is exactly a K-major, no-swizzle UMMA operand
 // with 8-row core matrices (SBO = 128 B) whose two K halves are one channel
@@ -38,6 +45,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cuda_bf16.h>
+
 #include "device_utils.cuh"
 #include "gconv_internal.h"
 
@@ -48,8 +57,19 @@ namespace {
 __device__ int g_igemm_error = 0;
 
 // ------------------------------------------------------------------ prep
+// Two bf16 values packed in 32 bits, first in the low half (memory order).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo_half, float hi_half) {
+    const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(lo_half));
+    const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(hi_half));
+    return a | (b << 16);
+}
+
+// x[N][C][H][W] -> per 8 input channels (octet c8) and pixel:
+//   xh: tf32 parts in NC4HW4 cells, [n][2*c8 + q][h][w][4]  (q = channel quad)
+//   xc: bf16 parts, [n][c8][2][h][w][8]: chunk 0 = bf16(x_hi), chunk 1 = bf16(x - x_hi)
+// Both tensors have the same geometry when read as 32-bit words.
 __global__ void __launch_bounds__(256) split_x_kernel(const float *__restrict__ x, float4 *__restrict__ xh,
-                                                      float4 *__restrict__ xl, int C4, int H, int W,
+                                                      uint4 *__restrict__ xc, int C8, int H, int W,
                                                       long long cells) {
     dev::griddep_wait();
     dev::griddep_launch_dependents();
@@ -57,23 +77,31 @@ __global__ void __launch_bounds__(256) split_x_kernel(const float *__restrict__ 
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < cells;
          i += (long long)gridDim.x * blockDim.x) {
         const long long pix = i % HW;          // h*W + w
-        const long long nc4 = i / HW;          // n*C4 + c4
-        const float *src = x + nc4 * 4 * HW + pix;
-        float v[4], hi[4], lo[4];
+        const long long nc8 = i / HW;          // n*C8 + c8
+        const float *src = x + nc8 * 8 * HW + pix;
+        float hi[8], lo[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            v[j] = __ldg(src + j * HW);
-            hi[j] = dev::to_tf32(v[j]);
-            lo[j] = v[j] - hi[j];
+        for (int j = 0; j < 8; ++j) {
+            const float v = __ldg(src + j * HW);
+            hi[j] = dev::to_tf32(v);
+            lo[j] = v - hi[j];
         }
-        xh[i] = make_float4(hi[0], hi[1], hi[2], hi[3]);
-        xl[i] = make_float4(lo[0], lo[1], lo[2], lo[3]);
+        const long long q0 = (nc8 * 2) * HW + pix;   // cell index of quad 0 (and of chunk 0)
+        xh[q0] = make_float4(hi[0], hi[1], hi[2], hi[3]);
+        xh[q0 + HW] = make_float4(hi[4], hi[5], hi[6], hi[7]);
+        xc[q0] = make_uint4(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]), pack_bf16x2(hi[4], hi[5]),
+                            pack_bf16x2(hi[6], hi[7]));
+        xc[q0 + HW] = make_uint4(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]), pack_bf16x2(lo[4], lo[5]),
+                                 pack_bf16x2(lo[6], lo[7]));
     }
 }
 
-// w[K][cpg][R][S] -> [g][cpg/8][r][s][2][kpg][4] (hi and lo)
+// w[K][cpg][R][S] -> per (g, c8, r, s, output channel kk), 8 input channels:
+//   wh: [g][c8][r][s][2][kpg][4]   tf32 parts (two channel quads)
+//   wc: [g][c8][r][s][2][kpg][8]   bf16 parts: chunk 0 = bf16(w - w_hi), chunk 1 = bf16(w_hi)
+// so that the bf16 MMA over K = 16 computes x_hi*w_lo + x_lo*w_hi.
 __global__ void __launch_bounds__(256) split_w_kernel(const float *__restrict__ w, float4 *__restrict__ wh,
-                                                      float4 *__restrict__ wl, int kpg, int cpg, int R, int S,
+                                                      uint4 *__restrict__ wc, int kpg, int cpg, int R, int S,
                                                       long long cells) {
     dev::griddep_wait();
     dev::griddep_launch_dependents();
@@ -81,22 +109,26 @@ __global__ void __launch_bounds__(256) split_w_kernel(const float *__restrict__ 
          i += (long long)gridDim.x * blockDim.x) {
         long long t = i;
         const int kk = (int)(t % kpg); t /= kpg;
-        const int h2 = (int)(t % 2); t /= 2;
         const int s = (int)(t % S); t /= S;
         const int r = (int)(t % R); t /= R;
-        const int cc8 = (int)(t % (cpg / 8));
+        const int c8 = (int)(t % (cpg / 8));
         const long long g = t / (cpg / 8);
         const long long k = g * kpg + kk;
-        float hi[4], lo[4];
+        float hi[8], lo[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int c = cc8 * 8 + h2 * 4 + j;
-            const float v = __ldg(w + ((k * cpg + c) * R + r) * S + s);
+        for (int j = 0; j < 8; ++j) {
+            const float v = __ldg(w + ((k * cpg + c8 * 8 + j) * R + r) * S + s);
             hi[j] = dev::to_tf32(v);
             lo[j] = v - hi[j];
         }
-        wh[i] = make_float4(hi[0], hi[1], hi[2], hi[3]);
-        wl[i] = make_float4(lo[0], lo[1], lo[2], lo[3]);
+        // slot of (g, c8, r, s): [2][kpg] cells
+        const long long base = ((((g * (cpg / 8) + c8) * R + r) * S + s) * 2) * kpg + kk;
+        wh[base] = make_float4(hi[0], hi[1], hi[2], hi[3]);
+        wh[base + kpg] = make_float4(hi[4], hi[5], hi[6], hi[7]);
+        wc[base] = make_uint4(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]), pack_bf16x2(lo[4], lo[5]),
+                              pack_bf16x2(lo[6], lo[7]));
+        wc[base + kpg] = make_uint4(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]), pack_bf16x2(hi[4], hi[5]),
+                                    pack_bf16x2(hi[6], hi[7]));
     }
 }
 
@@ -261,7 +293,8 @@ __global__ void __launch_bounds__(kIgThreads, 1)
         if (lane == 0) {
             // ------------------------------------------------------ MMA issuer
             constexpr uint32_t idesc = dev::idesc_tf32(128, NT);
-            const uint32_t a_lbo = (uint32_t)p.AR * p.COLS * 16;   // one channel quad apart
+            constexpr uint32_t idesc_c = dev::idesc_bf16(128, NT);
+            const uint32_t a_lbo = (uint32_t)p.AR * p.COLS * 16;   // one channel quad / bf16 chunk apart
             const uint32_t b_lbo = NT * 16;
             int ia = 0, ib = 0, j = 0;
             bool ok = true;
@@ -300,8 +333,9 @@ __global__ void __launch_bounds__(kIgThreads, 1)
                                 const uint64_t ao = (uint64_t)((i + r * p.dil) * p.COLS + s * p.dil);
                                 const uint64_t bo = (uint64_t)(s * 2 * NT);
                                 const uint32_t acc = (cc8 > 0 || r > 0 || s > 0) ? 1u : 0u;
-                                dev::mma_tf32(d, dal + ao, dbh + bo, idesc, acc);
-                                dev::mma_tf32(d, dah + ao, dbl + bo, idesc, 1u);
+                                // cross terms x_hi*w_lo + x_lo*w_hi: one bf16 MMA over K = 16
+                                dev::mma_bf16(d, dal + ao, dbl + bo, idesc_c, acc);
+                                // main term x_hi*w_hi: tf32 MMA over K = 8
                                 dev::mma_tf32(d, dah + ao, dbh + bo, idesc, 1u);
                             }
                         }
@@ -542,19 +576,19 @@ bool make_nc4hw4_tensor_map(TensorMap *tm, const float *base, long long quads, i
 }
 
 cudaError_t launch_split_x(const float *x, float *xh, float *xl, int N, int C, int H, int W, cudaStream_t st) {
-    const long long cells = (long long)N * (C / 4) * H * W;
+    const long long cells = (long long)N * (C / 8) * H * W;
     const long long blocks = std::min<long long>((cells + 255) / 256, 148LL * 64);
     return launch_ex(split_x_kernel, dim3((unsigned)blocks), dim3(256), 0, st, x, reinterpret_cast<float4 *>(xh),
-                     reinterpret_cast<float4 *>(xl), C / 4, H, W, cells);
+                     reinterpret_cast<uint4 *>(xl), C / 8, H, W, cells);
 }
 
 cudaError_t launch_split_w(const float *w, float *wh, float *wl, int K, int cpg, int R, int S, int groups,
                            cudaStream_t st) {
     const int kpg = K / groups;
-    const long long cells = (long long)groups * (cpg / 8) * R * S * 2 * kpg;
+    const long long cells = (long long)groups * (cpg / 8) * R * S * kpg;
     const long long blocks = std::min<long long>((cells + 255) / 256, 148LL * 8);
     return launch_ex(split_w_kernel, dim3((unsigned)blocks), dim3(256), 0, st, w, reinterpret_cast<float4 *>(wh),
-                     reinterpret_cast<float4 *>(wl), kpg, cpg, R, S, cells);
+                     reinterpret_cast<uint4 *>(wl), kpg, cpg, R, S, cells);
 }
 
 cudaError_t launch_igemm(const IgemmParams &p, const TensorMap *tm, int chain, dim3 grid, size_t smem,

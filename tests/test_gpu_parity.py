@@ -374,7 +374,7 @@ def test_igemm_matches_oracle(oracle_mod, geo):
                            x_dist="normal", bias=bias)
     gc.force_kernel("igemm")
     try:
-        assert gc.plan_name(N, C, H, W, K, R, S, st, pad, dil, g) == "igemm_tf32x3"
+        assert gc.plan_name(N, C, H, W, K, R, S, st, pad, dil, g) == "igemm_tf32_bf16x"
         full_check(oracle_mod, d, st, pad, dil, g, "igemm " + str(geo))
     finally:
         gc.force_kernel("auto")
