@@ -193,6 +193,30 @@ __device__ __forceinline__ void tmem_ld16_pair(uint32_t ta, uint32_t tb, float (
     }
 }
 
+// Two 8-column TMEM loads in flight, one wait.
+__device__ __forceinline__ void tmem_ld8_pair(uint32_t ta, uint32_t tb, float (&va)[8], float (&vb)[8]) {
+    uint32_t r[8], q[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(ta));
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+                 : "=r"(q[0]), "=r"(q[1]), "=r"(q[2]), "=r"(q[3]), "=r"(q[4]), "=r"(q[5]), "=r"(q[6]), "=r"(q[7])
+                 : "r"(tb));
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        va[i] = __uint_as_float(r[i]);
+        vb[i] = __uint_as_float(q[i]);
+    }
+}
+
+template <int CW>
+__device__ __forceinline__ void tmem_ld_pair(uint32_t ta, uint32_t tb, float (&va)[CW], float (&vb)[CW]) {
+    static_assert(CW == 8 || CW == 16, "chunk width");
+    if constexpr (CW == 16) tmem_ld16_pair(ta, tb, va, vb);
+    else tmem_ld8_pair(ta, tb, va, vb);
+}
+
 // Shared-memory matrix descriptor, K-major, no swizzle: core matrices of
 // 8 rows x 16 bytes; `lbo` = bytes between the two 16-byte K halves of one
 // K=8 (tf32) step, `sbo` = bytes between consecutive 8-row groups.

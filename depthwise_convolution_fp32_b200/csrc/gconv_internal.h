@@ -111,7 +111,7 @@ struct IgemmParams {
 
 int igemm_supported_nt(int kpg);
 size_t igemm_header_bytes(int nt, bool chain);
-int igemm_threads();
+int igemm_threads(int nt);
 // 3-D tensor map over an NC4HW4 tensor viewed as [quads][H][W*4] floats with
 // a box of box_px (<= 64) pixels of one row of one channel quad.
 bool make_nc4hw4_tensor_map(TensorMap *tm, const float *base, long long quads, int H, int W, int box_px);

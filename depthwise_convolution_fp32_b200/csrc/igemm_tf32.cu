@@ -132,8 +132,11 @@ __global__ void __launch_bounds__(256) split_w_kernel(const float *__restrict__ 
     }
 }
 
-constexpr int kIgEpiWarps = 8;                      // epilogue warps (2 per TMEM lane quarter)
-constexpr int kIgThreads = 64 + 32 * kIgEpiWarps;    // + producer warp + MMA warp
+// Epilogue warps: 16 (4 per TMEM lane quarter, 8-column chunks) for 32
+// output channels, 8 (2 per lane quarter, 16-column chunks) for wider tiles,
+// so the epilogue keeps enough warps in flight without spilling registers.
+__host__ __device__ constexpr int ig_epi_warps(int NT) { return NT <= 32 ? 16 : 8; }
+__host__ __device__ constexpr int ig_threads(int NT) { return 64 + 32 * ig_epi_warps(NT); }
 // shared memory ahead of the stage ring: barriers, TMEM slot and, for the
 // chain, per-fragment statistics [NT fragments at most][4 lane quarters][3 doubles]
 __host__ __device__ constexpr int ig_header(int NT, bool chain) {
@@ -145,8 +148,9 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
 }
 
 // Named barrier over the epilogue warps only.
+template <int EPW>
 __device__ __forceinline__ void epi_sync() {
-    asm volatile("bar.sync 1, %0;\n" ::"r"(32 * kIgEpiWarps) : "memory");
+    asm volatile("bar.sync 1, %0;\n" ::"r"(32 * EPW) : "memory");
 }
 
 // Output tile t -> (n, g, row tile, column tile); column tiles vary fastest so
@@ -175,7 +179,7 @@ __device__ __forceinline__ IgTile ig_tile(const IgemmParams &p, int t) {
 // KGN: 0 = plain convolution; otherwise the GroupNorm group width of the
 // chain (1, 2, 4, 8, 16, or 32 standing for any multiple of 16).
 template <int NT, int KGN>
-__global__ void __launch_bounds__(kIgThreads, 1)
+__global__ void __launch_bounds__(ig_threads(NT), 1)
     igemm_tf32x3_kernel(const __grid_constant__ TensorMap tmh, const __grid_constant__ TensorMap tml,
                         const __grid_constant__ TensorMap tmh_tail, const __grid_constant__ TensorMap tml_tail,
                         const IgemmParams p) {
@@ -212,7 +216,7 @@ __global__ void __launch_bounds__(kIgThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             dev::mbar_init(&accf[b], 1);
-            dev::mbar_init(&acce[b], kIgEpiWarps);
+            dev::mbar_init(&acce[b], ig_epi_warps(NT));
         }
         *abort_flag = 0;
         dev::fence_mbar_init();
@@ -353,13 +357,17 @@ __global__ void __launch_bounds__(kIgThreads, 1)
         __syncwarp();
     } else {
         // ---------------------------------------------------------- epilogue
-        // chain: GroupNorm groups per 16-channel chunk and their width in it
-        constexpr int GPC = CHAIN ? (KGN >= 16 ? 1 : 16 / KGN) : 1;
-        constexpr int GW = CHAIN ? (KGN >= 16 ? 16 : KGN) : 16;
-        const int ew = warp - 2;                 // 0..7
+        // columns: each warp owns NT/4 accumulator columns of its lane quarter,
+        // processed in chunks of CW; chain: GroupNorm groups per chunk (GPC)
+        // and their width inside it (GW)
+        constexpr int EPW = ig_epi_warps(NT);
+        constexpr int PART = NT / (EPW / 4);
+        constexpr int CW = PART < 16 ? PART : 16;
+        constexpr int GPC = CHAIN ? (KGN >= CW ? 1 : CW / KGN) : 1;
+        constexpr int GW = CHAIN ? (KGN >= CW ? CW : KGN) : CW;
+        const int ew = warp - 2;                 // 0..EPW-1
         const int lq = warp & 3;                 // TMEM lane quarter this warp may access
-        const int chalf = ew >> 2;               // column half
-        constexpr int HALF = NT / 2;
+        const int cpart = ew >> 2;               // column block of this warp
         const int m = lq * 32 + lane;
         const long long plane = (long long)p.P * p.Q;
         int j = 0;
@@ -376,11 +384,11 @@ __global__ void __launch_bounds__(kIgThreads, 1)
             float *ybase = p.y + ((long long)tl.n * p.K + (long long)tl.g * p.kpg) * plane + q;
             const uint32_t tbase = tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)buf * acc_cols;
 #pragma unroll 1
-            for (int c0 = chalf * HALF; c0 < (chalf + 1) * HALF; c0 += 16) {
+            for (int c0 = cpart * PART; c0 < (cpart + 1) * PART; c0 += CW) {
                 // z = acc * mul + add: plain (mul 1, add bias) or chain (scale, bias*scale)
-                float mul[16], add[16];
+                float mul[CW], add[CW];
 #pragma unroll
-                for (int jj = 0; jj < 16; ++jj) {
+                for (int jj = 0; jj < CW; ++jj) {
                     const int k = tl.g * p.kpg + c0 + jj;
                     const float b = p.bias ? __ldg(p.bias + k) : 0.f;
                     mul[jj] = CHAIN ? __ldg(p.scale + k) : 1.f;
@@ -395,10 +403,10 @@ __global__ void __launch_bounds__(kIgThreads, 1)
                 // rows are processed two at a time so one TMEM load latency covers both
 #pragma unroll 1
                 for (int i = 0; i < p.TH; i += 2) {
-                    float vv[2][16];
+                    float vv[2][CW];
                     const bool two = i + 1 < p.TH;
-                    dev::tmem_ld16_pair(tbase + (uint32_t)(i * NT + c0), tbase + (uint32_t)((i + (two ? 1 : 0)) * NT + c0),
-                                        vv[0], vv[1]);
+                    dev::tmem_ld_pair<CW>(tbase + (uint32_t)(i * NT + c0),
+                                          tbase + (uint32_t)((i + (two ? 1 : 0)) * NT + c0), vv[0], vv[1]);
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         if (h == 1 && !two) break;
@@ -406,7 +414,7 @@ __global__ void __launch_bounds__(kIgThreads, 1)
                         const int pp = tl.p0 + i + h;
                         const bool valid = ok && qvalid && pp < p.P;
 #pragma unroll
-                        for (int jj = 0; jj < 16; ++jj) {
+                        for (int jj = 0; jj < CW; ++jj) {
                             float z = fmaf(v[jj], mul[jj], add[jj]);
                             // logistic; the clamp keeps 1 + e finite (e^80 < 2^126)
                             if constexpr (CHAIN) z = __fdividef(1.f, 1.f + __expf(fminf(-z, 80.f)));
@@ -415,7 +423,7 @@ __global__ void __launch_bounds__(kIgThreads, 1)
                         if (valid) {
                             float *yr = ybase + (long long)c0 * plane + (long long)pp * p.Q;
 #pragma unroll
-                            for (int jj = 0; jj < 16; ++jj) yr[(long long)jj * plane] = v[jj];
+                            for (int jj = 0; jj < CW; ++jj) yr[(long long)jj * plane] = v[jj];
                             if constexpr (CHAIN) {
                                 if (cnt == 0.f) {
 #pragma unroll
@@ -423,7 +431,7 @@ __global__ void __launch_bounds__(kIgThreads, 1)
                                 }
                                 cnt += 1.f;
 #pragma unroll
-                                for (int jj = 0; jj < 16; ++jj) {
+                                for (int jj = 0; jj < CW; ++jj) {
                                     const float d = v[jj] - shift[jj / GW];
                                     s1[jj / GW] += d;
                                     s2[jj / GW] = fmaf(d, d, s2[jj / GW]);
@@ -432,7 +440,7 @@ __global__ void __launch_bounds__(kIgThreads, 1)
                         }
                     }
                 }
-                if (c0 + 16 >= (chalf + 1) * HALF) {
+                if (c0 + CW >= (cpart + 1) * PART) {
                     // last TMEM read of this tile by this warp: hand the buffer back
                     dev::tc_fence_before();
                     __syncwarp();
@@ -462,7 +470,7 @@ __global__ void __launch_bounds__(kIgThreads, 1)
                             if (lane < off) { S1 += o1; S2 += o2; Nn += on; }
                         }
                         if (lane == 0) {
-                            const int fr = (c0 >> 4) * GPC + gg;
+                            const int fr = (c0 / CW) * GPC + gg;
                             st_n[fr * 4 + lq] = Nn;
                             st_1[fr * 4 + lq] = S1;
                             st_2[fr * 4 + lq] = S2;
@@ -471,13 +479,13 @@ __global__ void __launch_bounds__(kIgThreads, 1)
                 }
             }
             if constexpr (CHAIN) {
-                epi_sync();
+                epi_sync<EPW>();
                 const int et = tid - 64;
                 const int ngroups = NT / p.kgn;
                 if (et < ngroups) {
-                    // fragments of group et: one per group (width <= 16) or kgn/16 chunks
-                    const int f0 = KGN >= 16 ? et * (p.kgn / 16) : et;
-                    const int f1 = KGN >= 16 ? (et + 1) * (p.kgn / 16) : et + 1;
+                    // fragments of group et: one per group (width <= CW) or kgn/CW chunks
+                    const int f0 = p.kgn > CW ? et * (p.kgn / CW) : et;
+                    const int f1 = p.kgn > CW ? (et + 1) * (p.kgn / CW) : et + 1;
                     double Nn = 0.0, S1 = 0.0, S2 = 0.0;
                     for (int fr = f0; fr < f1; ++fr)
                         for (int l = 0; l < 4; ++l) {
@@ -491,7 +499,7 @@ __global__ void __launch_bounds__(kIgThreads, 1)
                     p.gn_part[((long long)tl.n * p.gn_groups + G) * p.slots + tl.sp] =
                         make_float4((float)Nn, (float)mean, (float)m2, 0.f);
                 }
-                epi_sync();   // statistics scratch free for the next tile
+                epi_sync<EPW>();   // statistics scratch free for the next tile
             }
         }
     }
@@ -521,7 +529,7 @@ cudaError_t launch_nt(const IgemmParams &p, const TensorMap *tm, dim3 grid, size
     auto kern = igemm_tf32x3_kernel<NT, KGN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_ex(kern, grid, dim3(kIgThreads), smem, st, tm[0], tm[1], tm[2], tm[3], p);
+    return launch_ex(kern, grid, dim3(ig_threads(NT)), smem, st, tm[0], tm[1], tm[2], tm[3], p);
 }
 
 template <int NT>
@@ -559,7 +567,7 @@ int igemm_supported_nt(int kpg) { return kpg == 32 || kpg == 64 || kpg == 128 ||
 
 size_t igemm_header_bytes(int nt, bool chain) { return ig_header(nt, chain); }
 
-int igemm_threads() { return kIgThreads; }
+int igemm_threads(int nt) { return ig_threads(nt); }
 
 bool make_nc4hw4_tensor_map(TensorMap *tm, const float *base, long long quads, int H, int W, int box_px) {
     auto fn = encode_fn();
