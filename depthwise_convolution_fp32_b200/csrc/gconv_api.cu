@@ -369,8 +369,13 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     if (chain && (s.kpg > 64 || s.kpg % kgn != 0 || (kgn > 16 && kgn % 16 != 0))) return false;
     const int NT = s.kpg;
     int COLS = 128 + (s.S - 1) * s.dil;
-    COLS = (COLS + 7) / 8 * 8;   // 128-byte aligned row segments
+    COLS = (COLS + 15) / 16 * 16;   // whole 16-pixel groups of the tile box
     if (COLS > 256) return false;
+    // padded split operands: every tile box starts at a 16-pixel group and a
+    // non-negative row, the zero border supplies the padding
+    const long long Hp = (long long)s.H + s.pad;
+    const long long Wp = ((long long)s.W + s.pad + 15) / 16 * 16;
+    if (Hp > 0x7fffffffLL || Wp / 16 > 0x7fffffffLL) return false;
     static const int force_th = env_int("GCONV_IGEMM_TH");
     static const int force_sa = env_int("GCONV_IGEMM_SA");
     static const int force_sb = env_int("GCONV_IGEMM_SB");
@@ -404,6 +409,8 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     p.CC8 = s.cpg / 8;
     p.TH = TH;
     p.COLS = COLS;
+    p.Hp = (int)Hp;
+    p.Wp = (int)Wp;
     p.n_qt = (s.Q + 127) / 128;
     p.n_pt = (s.P + TH - 1) / TH;
     const long long n_tiles = (long long)s.N * s.groups * p.n_qt * p.n_pt;
@@ -412,16 +419,17 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     p.AR = AR;
     p.sa = sa;
     p.sb = sb;
+    p.b_resident = p.CC8 * s.R <= sb ? 1 : 0;
     p.a_bytes = a_bytes;
     p.b_bytes = b_bytes;
     p.tmem_cols = tmem_cols;
     p.gn_groups = chain ? gn_groups : 0;
     p.kgn = kgn;
-    p.slots = p.n_qt * p.n_pt;
+    p.slots = p.n_qt * p.n_pt * (chain ? igemm_partials_per_tile(NT, kgn) : 1);
     pl.grid = dim3((unsigned)std::min<long long>(n_tiles, sm_count()));
     pl.smem = igemm_header_bytes(NT, chain) + (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes;
 
-    const size_t xbytes = (size_t)s.N * s.C * s.H * s.W * sizeof(float);
+    const size_t xbytes = (size_t)s.N * s.C * (size_t)Hp * (size_t)Wp * sizeof(float);
     const size_t wbytes = (size_t)s.K * s.cpg * s.R * s.S * sizeof(float);
     pl.off_xl = align256(xbytes);
     pl.off_wh = pl.off_xl + align256(xbytes);
@@ -455,12 +463,9 @@ gconv_status_t run_igemm(const Shape &s, IgemmPlan &pl, const float *x, const fl
     float *wl = reinterpret_cast<float *>(base + pl.off_wl);
     IgemmParams &p = pl.prm;
     const long long quads = (long long)s.N * (s.C / 4);
-    TensorMap tm[4];
-    const int tail = p.COLS % 64;
-    if (!make_nc4hw4_tensor_map(&tm[0], xh, quads, s.H, s.W, 64) ||
-        !make_nc4hw4_tensor_map(&tm[1], xl, quads, s.H, s.W, 64) ||
-        !make_nc4hw4_tensor_map(&tm[2], xh, quads, s.H, s.W, tail > 0 ? tail : 64) ||
-        !make_nc4hw4_tensor_map(&tm[3], xl, quads, s.H, s.W, tail > 0 ? tail : 64))
+    TensorMap tm[2];
+    if (!make_nc4hw4_tile_map(&tm[0], xh, quads, p.Hp, p.Wp, p.COLS, p.AR) ||
+        !make_nc4hw4_tile_map(&tm[1], xl, quads, p.Hp, p.Wp, p.COLS, p.AR))
         return GCONV_ERR_UNSUPPORTED;
     p.wh = reinterpret_cast<const float4 *>(wh);
     p.wl = reinterpret_cast<const float4 *>(wl);
@@ -469,7 +474,8 @@ gconv_status_t run_igemm(const Shape &s, IgemmPlan &pl, const float *x, const fl
     p.y = y;
     const bool chain = scale != nullptr;
     p.gn_part = chain ? reinterpret_cast<float4 *>(base + pl.off_part) : nullptr;
-    if (launch_split_x(x, xh, xl, s.N, s.C, s.H, s.W, stream) != cudaSuccess) return GCONV_ERR_CUDA;
+    if (launch_split_x(x, xh, xl, s.N, s.C, s.H, s.W, s.pad, p.Hp, p.Wp, stream) != cudaSuccess)
+        return GCONV_ERR_CUDA;
     if (launch_split_w(w, wh, wl, s.K, s.cpg, s.R, s.S, s.groups, stream) != cudaSuccess) return GCONV_ERR_CUDA;
     if (launch_igemm(p, tm, chain ? 1 : 0, pl.grid, pl.smem, stream) != cudaSuccess) return GCONV_ERR_CUDA;
     if (!chain) return GCONV_OK;

@@ -100,25 +100,34 @@ struct IgemmParams {
     int CC8;                   // cpg / 8 (K-steps of 8 channels)
     int TH;                    // output rows per tile (one 128-pixel M tile each)
     int AR;                    // staged x rows per channel step: TH + (R-1)*dil
-    int COLS;                  // staged columns per row (>= 128 + (S-1)*dil, multiple of 8)
+    int COLS;                  // staged columns per row (>= 128 + (S-1)*dil, multiple of 16)
+    int Hp, Wp;                // padded x planes of the split operands: pad rows on top, pad
+                               // columns on the left, zero columns up to Wp (multiple of 16)
     int n_qt, n_pt;
     int n_tiles;               // N * groups * n_pt * n_qt
     int sa, sb;                // slots of the x-tile ring and of the weight-slice ring
+    int b_resident;            // 1: all CC8*R weight slices fit the ring and are loaded once per CTA
     int a_bytes, b_bytes;      // one x operand (hi or lo) tile / one w operand slice
     int tmem_cols;
-    int gn_groups, kgn, slots;
+    int gn_groups, kgn, slots;  // chain: partials per (image, group) = tiles per image x per-tile partials
 };
 
 int igemm_supported_nt(int kpg);
 size_t igemm_header_bytes(int nt, bool chain);
+// GroupNorm partials the chain epilogue writes per tile and group (one per
+// TMEM lane quarter and per channel chunk the group spans)
+int igemm_partials_per_tile(int nt, int kgn);
 int igemm_threads(int nt);
-// 3-D tensor map over an NC4HW4 tensor viewed as [quads][H][W*4] floats with
-// a box of box_px (<= 64) pixels of one row of one channel quad.
-bool make_nc4hw4_tensor_map(TensorMap *tm, const float *base, long long quads, int H, int W, int box_px);
-cudaError_t launch_split_x(const float *x, float *xh, float *xl, int N, int C, int H, int W, cudaStream_t st);
+// 4-D tensor map over a padded NC4HW4 tensor [quads][Hp][Wp][4] viewed as
+// [quads][Hp][Wp/16][64 floats]; one box is a whole x tile of one channel
+// step: 2 quads x box_rows rows x box_cols (multiple of 16) pixels.
+bool make_nc4hw4_tile_map(TensorMap *tm, const float *base, long long quads, int Hp, int Wp, int box_cols,
+                          int box_rows);
+cudaError_t launch_split_x(const float *x, float *xh, float *xl, int N, int C, int H, int W, int pad, int Hp,
+                           int Wp, cudaStream_t st);
 cudaError_t launch_split_w(const float *w, float *wh, float *wl, int K, int cpg, int R, int S, int groups,
                            cudaStream_t st);
-// tm: x_hi 64-pixel map, x_lo 64-pixel map, x_hi tail map, x_lo tail map
+// tm: x_hi tile map, cross-term tile map
 cudaError_t launch_igemm(const IgemmParams &p, const TensorMap *tm, int chain, dim3 grid, size_t smem,
                          cudaStream_t st);
 int read_and_clear_igemm_error();

@@ -1,5 +1,5 @@
-// Implicit-GEMM convolution on the 5th-generation tensor cores (tcgen05) with
-// 3xTF32 splitting, for stride-1 dense and wide-group convolutions.
+// Implicit-GEMM convolution on the 5th-generation tensor cores (tcgen05) at
+// FP32 accuracy, for stride-1 dense and wide-group convolutions.
 //
 // What it computes (POPCORNBENCH "Kimi-K2.6__l1_p62" and "Kimi-K2.6__l2_p21":
 // the convolution viewed as a GEMM with M = output pixels, N = output
@@ -17,31 +17,32 @@
 // (2^-11 relative) would miss that bound; the pages flag TF32 as "not
 // exactly fp32".
 //
-// Data layout.  A prep pass writes x_hi as NC4HW4 ([n][c/4][h][w][4]: four
-// consecutive channels in one 16-byte cell) and the bf16 cross-term operand
-// as [n][c/8][2][h][w][8] (same cell geometry), and the weights split the
-// same way as [g][c/8][r][s][2][kpg][4 tf32 | 8 bf16].  In the NC4HW4 tile a CTA stages
-// ([2 channel quads][rows][cols][4]), consecutive output pixels of one row
-// are 16 bytes apart, which is exactly a K-major, no-swizzle UMMA operand
-// with 8-row core matrices (SBO = 128 B) whose two K halves are one channel
-// quad apart (LBO).  The operand for filter tap (r, s) is therefore the same
-// staged tile with its start address moved by (row r*dil, column s*dil): the
-// im2col matrix is never materialised, and every staged element feeds S
-// taps of MMAs.
+// Data layout.  A prep pass writes x_hi as padded NC4HW4 ([n][c/4][hp][wp][4]:
+// four consecutive channels in one 16-byte cell; pad zero rows on top, pad
+// zero columns on the left, zero columns up to a multiple of 16 pixels) and
+// the bf16 cross-term operand as [n][c/8][2][hp][wp][8] (same cell geometry),
+// and the weights split the same way as [g][c/8][r][s][2][kpg][4 tf32 | 8 bf16].
+// In the tile a CTA stages ([2 channel quads][rows][cols][4], one TMA box),
+// consecutive output pixels of one row are 16 bytes apart, which is exactly
+// a K-major, no-swizzle UMMA operand with 8-row core matrices (SBO = 128 B)
+// whose two K halves are one channel quad apart (LBO).  The operand for filter
+// tap (r, s) is therefore the same staged tile with its start address moved by
+// (row r*dil, column s*dil): the im2col matrix is never materialised, and
+// every staged element feeds up to R*S taps of MMAs.
 //
-// Pipeline (one CTA = one image n, TH output rows x 128 output columns, all
-// kpg output channels of group g):
-//   warp 0 lane 0 : producer - per K-stage (8 input channels, one tap row r)
-//                   two 4-D TMA loads (x_hi, x_lo tiles, zero fill supplies
-//                   the padding) and two bulk copies (w_hi, w_lo slices) into
-//                   a ring of shared-memory stages, signalled on mbarriers;
-//   warp 1 lane 0 : MMA issuer - for every output row i and tap s, three
-//                   tcgen05.mma (M=128, N=kpg, K=8) into the row's TMEM
-//                   accumulator; tcgen05.commit frees the stage;
-//   all 8 warps   : epilogue - tcgen05.ld of the accumulators (warp w reads
-//                   TMEM lanes 32*(w%4).. and half of the columns), +bias, or
-//                   the chain's +bias, *scale, logistic and GroupNorm partial
-//                   statistics, coalesced stores along q.
+// Pipeline (persistent; a tile = one image n, TH output rows x 128 output
+// columns, all kpg output channels of group g):
+//   warp 0 lane 0 : producer - per 8-channel step one TMA box of x_hi and one
+//                   of the cross-term operand (all staged rows and columns),
+//                   then the weight slices of the R tap rows (bulk copies;
+//                   loaded once per CTA when they all fit the ring);
+//   warp 1 lane 0 : MMA issuer - for every output row i and tap (r, s) one
+//                   bf16 and one tf32 tcgen05.mma (M=128, N=kpg) into the
+//                   row's TMEM accumulator; tcgen05.commit frees the stages;
+//   other warps   : epilogue - tcgen05.ld of the accumulators, +bias, or the
+//                   chain's +bias, *scale, logistic and GroupNorm partial
+//                   statistics, coalesced stores along q; two TMEM
+//                   accumulator buffers let it overlap the next tile's MMAs.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -64,35 +65,39 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo_half, float hi_half) {
     return a | (b << 16);
 }
 
-// x[N][C][H][W] -> per 8 input channels (octet c8) and pixel:
-//   xh: tf32 parts in NC4HW4 cells, [n][2*c8 + q][h][w][4]  (q = channel quad)
-//   xc: bf16 parts, [n][c8][2][h][w][8]: chunk 0 = bf16(x_hi), chunk 1 = bf16(x - x_hi)
+// x[N][C][H][W] -> per 8 input channels (octet c8) and padded pixel (hp, wp)
+// of a [Hp][Wp] plane holding x[h][w] at (h + pad, w + pad) and zeros
+// elsewhere:
+//   xh: tf32 parts in NC4HW4 cells, [n][2*c8 + q][hp][wp][4]  (q = channel quad)
+//   xc: bf16 parts, [n][c8][2][hp][wp][8]: chunk 0 = bf16(x_hi), chunk 1 = bf16(x - x_hi)
 // Both tensors have the same geometry when read as 32-bit words.
 __global__ void __launch_bounds__(256) split_x_kernel(const float *__restrict__ x, float4 *__restrict__ xh,
-                                                      uint4 *__restrict__ xc, int C8, int H, int W,
-                                                      long long cells) {
+                                                      uint4 *__restrict__ xc, int C8, int H, int W, int pad,
+                                                      int Hp, int Wp, long long cells) {
     dev::griddep_wait();
     dev::griddep_launch_dependents();
-    const long long HW = (long long)H * W;
+    const long long HW = (long long)H * W, HWp = (long long)Hp * Wp;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < cells;
          i += (long long)gridDim.x * blockDim.x) {
-        const long long pix = i % HW;          // h*W + w
-        const long long nc8 = i / HW;          // n*C8 + c8
-        const float *src = x + nc8 * 8 * HW + pix;
+        const long long pix = i % HWp;         // hp*Wp + wp
+        const long long nc8 = i / HWp;         // n*C8 + c8
+        const int h = (int)(pix / Wp) - pad, w = (int)(pix % Wp) - pad;
+        const bool in = h >= 0 && h < H && w >= 0 && w < W;
+        const float *src = x + nc8 * 8 * HW + (in ? (long long)h * W + w : 0);
         float hi[8], lo[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const float v = __ldg(src + j * HW);
+            const float v = in ? __ldg(src + j * HW) : 0.f;
             hi[j] = dev::to_tf32(v);
             lo[j] = v - hi[j];
         }
-        const long long q0 = (nc8 * 2) * HW + pix;   // cell index of quad 0 (and of chunk 0)
+        const long long q0 = (nc8 * 2) * HWp + pix;   // cell index of quad 0 (and of chunk 0)
         xh[q0] = make_float4(hi[0], hi[1], hi[2], hi[3]);
-        xh[q0 + HW] = make_float4(hi[4], hi[5], hi[6], hi[7]);
+        xh[q0 + HWp] = make_float4(hi[4], hi[5], hi[6], hi[7]);
         xc[q0] = make_uint4(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]), pack_bf16x2(hi[4], hi[5]),
                             pack_bf16x2(hi[6], hi[7]));
-        xc[q0 + HW] = make_uint4(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]), pack_bf16x2(lo[4], lo[5]),
-                                 pack_bf16x2(lo[6], lo[7]));
+        xc[q0 + HWp] = make_uint4(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]), pack_bf16x2(lo[4], lo[5]),
+                                  pack_bf16x2(lo[6], lo[7]));
     }
 }
 
@@ -137,20 +142,29 @@ __global__ void __launch_bounds__(256) split_w_kernel(const float *__restrict__ 
 // so the epilogue keeps enough warps in flight without spilling registers.
 __host__ __device__ constexpr int ig_epi_warps(int NT) { return NT <= 32 ? 16 : 8; }
 __host__ __device__ constexpr int ig_threads(int NT) { return 64 + 32 * ig_epi_warps(NT); }
-// shared memory ahead of the stage ring: barriers, TMEM slot and, for the
-// chain, per-fragment statistics [NT fragments at most][4 lane quarters][3 doubles]
-__host__ __device__ constexpr int ig_header(int NT, bool chain) {
-    return chain ? (256 + 96 * NT + 1023) / 1024 * 1024 : 1024;
+// shared memory ahead of the stage ring: barriers, TMEM slot, abort flag
+__host__ __device__ constexpr int ig_header(int NT, bool chain) { return 1024; }
+
+// Number of GroupNorm partials one tile leaves per group: one per TMEM lane
+// quarter and per chunk of CW channels the group spans.
+__host__ __device__ constexpr int ig_chunk_width(int NT) {
+    return NT / (ig_epi_warps(NT) / 4) < 16 ? NT / (ig_epi_warps(NT) / 4) : 16;
+}
+
+// logistic helpers: 2^x and 1/x on the special-function unit (flush to zero)
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_ftz(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(dev::smem_addr(bar)) : "memory");
-}
-
-// Named barrier over the epilogue warps only.
-template <int EPW>
-__device__ __forceinline__ void epi_sync() {
-    asm volatile("bar.sync 1, %0;\n" ::"r"(32 * EPW) : "memory");
 }
 
 // Output tile t -> (n, g, row tile, column tile); column tiles vary fastest so
@@ -171,6 +185,80 @@ __device__ __forceinline__ IgTile ig_tile(const IgemmParams &p, int t) {
     return r;
 }
 
+// Rows per tile the planner picks when shared memory allows: two TMEM
+// accumulator buffers of TH x NT columns.
+__host__ __device__ constexpr int ig_default_th(int NT) { return NT >= 256 ? 1 : (256 / NT < 8 ? 256 / NT : 8); }
+
+// MMA issuer (one thread).  For every tile and 8-channel step: wait for the
+// x tile, then per tap row r wait for its weight slice and issue, for every
+// output row i and tap s, the bf16 cross-term MMA and the tf32 main-term MMA
+// into row i's accumulator.  TH_, R_, S_ > 0 fix the loop bounds (dilation 1,
+// COLS = 128 + S_ - 1 rounded up to 16); 0 reads them from p.  Returns false
+// when a bounded wait gave up.
+template <int NT, int TH_, int R_, int S_>
+__device__ __forceinline__ bool ig_mma_loop(const IgemmParams &p, uint32_t tmem, const unsigned char *ringA,
+                                            const unsigned char *ringB, uint32_t a_slot, uint32_t b_slot,
+                                            uint64_t *fullA, uint64_t *emptyA, uint64_t *fullB, uint64_t *emptyB,
+                                            uint64_t *accf, uint64_t *acce) {
+    constexpr uint32_t idesc = dev::idesc_tf32(128, NT);
+    constexpr uint32_t idesc_c = dev::idesc_bf16(128, NT);
+    constexpr bool FIX = TH_ > 0;
+    const int TH = FIX ? TH_ : p.TH, R = FIX ? R_ : p.R, S = FIX ? S_ : p.S;
+    const int dil = FIX ? 1 : p.dil;
+    const int COLS = FIX ? (128 + S_ - 1 + 15) / 16 * 16 : p.COLS;
+    const uint32_t a_bytes = 32u * (uint32_t)COLS * (uint32_t)(TH + (R - 1) * dil);
+    const uint32_t a_lbo = a_bytes / 2;          // one channel quad / bf16 chunk apart
+    constexpr uint32_t b_lbo = NT * 16;
+    const uint32_t acc_cols = (uint32_t)(TH * NT);
+    int ia = 0, ib = 0, j = 0;
+    for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++j) {
+        const int buf = j & 1, ubuf = j >> 1;
+        if (ubuf > 0 && !dev::mbar_wait_bounded(&acce[buf], (ubuf - 1) & 1)) return false;
+        dev::tc_fence_after();
+        const uint32_t dbase = tmem + (uint32_t)buf * acc_cols;
+        for (int cc8 = 0; cc8 < p.CC8; ++cc8, ++ia) {
+            const int sa = ia % p.sa;
+            if (!dev::mbar_wait_bounded(&fullA[sa], (ia / p.sa) & 1)) return false;
+            dev::tc_fence_after();
+            const unsigned char *xa = ringA + (size_t)sa * a_slot;
+            const uint64_t dah = dev::smem_desc(xa, a_lbo, 128);
+            const uint64_t dal = dev::smem_desc(xa + a_bytes, a_lbo, 128);
+#pragma unroll 1
+            for (int r = 0; r < R; ++r, ++ib) {
+                const int sb = p.b_resident ? cc8 * R + r : ib % p.sb;
+                // resident slices: loaded once, waited for on the first tile only
+                if (!p.b_resident || j == 0) {
+                    if (!dev::mbar_wait_bounded(&fullB[sb], p.b_resident ? 0u : (uint32_t)((ib / p.sb) & 1)))
+                        return false;
+                    dev::tc_fence_after();
+                }
+                const unsigned char *wb = ringB + (size_t)sb * b_slot;
+                const uint64_t dbh = dev::smem_desc(wb, b_lbo, 128);
+                const uint64_t dbl = dev::smem_desc(wb + b_slot / 2, b_lbo, 128);
+#pragma unroll
+                for (int i = 0; i < TH; ++i) {
+                    const uint32_t d = dbase + (uint32_t)(i * NT);
+#pragma unroll
+                    for (int s = 0; s < S; ++s) {
+                        // 16-byte units: staged row i + r*dil, column s*dil
+                        const uint64_t ao = (uint64_t)((i + r * dil) * COLS + s * dil);
+                        const uint64_t bo = (uint64_t)(s * 2 * NT);
+                        const uint32_t acc = (cc8 > 0 || r > 0 || s > 0) ? 1u : 0u;
+                        // cross terms x_hi*w_lo + x_lo*w_hi: one bf16 MMA over K = 16
+                        dev::mma_bf16(d, dal + ao, dbl + bo, idesc_c, acc);
+                        // main term x_hi*w_hi: tf32 MMA over K = 8
+                        dev::mma_tf32(d, dah + ao, dbh + bo, idesc, 1u);
+                    }
+                }
+                if (!p.b_resident) dev::mma_commit(&emptyB[sb]);
+            }
+            dev::mma_commit(&emptyA[sa]);
+        }
+        dev::mma_commit(&accf[buf]);   // fires once this tile's MMAs have completed
+    }
+    return true;
+}
+
 // ------------------------------------------------------------------ main kernel
 // Persistent: CTA b processes tiles b, b + gridDim.x, ...  The producer and
 // the MMA issuer run ahead through a ring of shared-memory stages; the MMA
@@ -180,8 +268,7 @@ __device__ __forceinline__ IgTile ig_tile(const IgemmParams &p, int t) {
 // chain (1, 2, 4, 8, 16, or 32 standing for any multiple of 16).
 template <int NT, int KGN>
 __global__ void __launch_bounds__(ig_threads(NT), 1)
-    igemm_tf32x3_kernel(const __grid_constant__ TensorMap tmh, const __grid_constant__ TensorMap tml,
-                        const __grid_constant__ TensorMap tmh_tail, const __grid_constant__ TensorMap tml_tail,
+    igemm_tf32x3_kernel(const __grid_constant__ TensorMap tmh, const __grid_constant__ TensorMap tmc,
                         const IgemmParams p) {
     extern __shared__ __align__(1024) unsigned char smem[];
     uint64_t *fullA = reinterpret_cast<uint64_t *>(smem);  // [4] x tiles (hi and lo) landed
@@ -193,9 +280,6 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
     uint32_t *tslot = reinterpret_cast<uint32_t *>(fullA + 20);
     int *abort_flag = reinterpret_cast<int *>(fullA + 21);
     constexpr bool CHAIN = KGN > 0;
-    double *st_n = reinterpret_cast<double *>(smem + 256);   // [fragment][4] chain statistics
-    double *st_1 = st_n + NT * 4;
-    double *st_2 = st_1 + NT * 4;
     unsigned char *stages = smem + ig_header(NT, CHAIN);
 
     const int tid = threadIdx.x;
@@ -235,13 +319,11 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
-        // Per tile and 8-channel step: one x tile of AR = TH + (R-1)*dil rows
-        // (hi and lo, exact-width boxes: 64-pixel boxes plus one tail box per
-        // row) serving every tap row, then R weight slices (one per tap row).
-        const int nmain = p.COLS / 64;
-        const int tail = p.COLS - nmain * 64;               // pixels, multiple of 8
-        const int per_row = nmain + (tail > 0 ? 1 : 0);
-        const int boxes = 2 * 2 * p.AR * per_row;           // (hi, lo) x quads x rows x segments
+        // Per tile and 8-channel step: one x tile of AR = TH + (R-1)*dil
+        // rows x COLS columns x 2 channel quads, x_hi and cross-term operand
+        // one TMA box each, serving every tap row; then R weight slices (one
+        // per tap row).  Tile coordinates are padded ones: output (p, q) reads
+        // padded rows p.. and columns q.. of the split operands.
         int ia = 0, ib = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
@@ -252,26 +334,20 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
                 if (lane == 0) {
                     if (ua > 0 && !dev::mbar_wait_bounded(&emptyA[sa], (ua - 1) & 1)) ok = false;
                     if (*(volatile int *)abort_flag) ok = false;
-                    if (ok) dev::mbar_arrive_expect_tx(&fullA[sa], a_slot);
+                    if (ok) {
+                        dev::mbar_arrive_expect_tx(&fullA[sa], a_slot);
+                        unsigned char *st = ringA + (size_t)sa * a_slot;
+                        const int cz = z0 + cc8 * 2;
+                        dev::tma_load_4d(st, &tmh, &fullA[sa], 0, tl.q0 / 16, tl.p0, cz);
+                        dev::tma_load_4d(st + p.a_bytes, &tmc, &fullA[sa], 0, tl.q0 / 16, tl.p0, cz);
+                    }
                 }
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 if (!ok) break;
-                unsigned char *st = ringA + (size_t)sa * a_slot;
-                const int x0 = tl.q0 - p.pad, y0 = tl.p0 - p.pad, cz = z0 + cc8 * 2;
-                for (int b = lane; b < boxes; b += 32) {
-                    const int seg = b % per_row;
-                    int rest = b / per_row;
-                    const int row = rest % p.AR; rest /= p.AR;
-                    const int quad = rest & 1;
-                    const int lo = rest >> 1;
-                    const int px = seg * 64;
-                    unsigned char *dst = st + lo * p.a_bytes + ((size_t)(quad * p.AR + row) * p.COLS + px) * 16;
-                    const void *map = seg < nmain ? (lo ? (const void *)&tml : (const void *)&tmh)
-                                                  : (lo ? (const void *)&tml_tail : (const void *)&tmh_tail);
-                    dev::tma_load_3d(dst, map, &fullA[sa], (x0 + px) * 4, y0 + row, cz + quad);
-                }
+                if (p.b_resident && t != (int)blockIdx.x) continue;   // slices already resident
                 for (int r = 0; r < p.R; ++r, ++ib) {
-                    const int sb = ib % p.sb, ub = ib / p.sb;
+                    const int sb = p.b_resident ? cc8 * p.R + r : ib % p.sb;
+                    const int ub = p.b_resident ? 0 : ib / p.sb;
                     if (lane == 0) {
                         if (ub > 0 && !dev::mbar_wait_bounded(&emptyB[sb], (ub - 1) & 1)) ok = false;
                         if (*(volatile int *)abort_flag) ok = false;
@@ -296,59 +372,16 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------------ MMA issuer
-            constexpr uint32_t idesc = dev::idesc_tf32(128, NT);
-            constexpr uint32_t idesc_c = dev::idesc_bf16(128, NT);
-            const uint32_t a_lbo = (uint32_t)p.AR * p.COLS * 16;   // one channel quad / bf16 chunk apart
-            const uint32_t b_lbo = NT * 16;
-            int ia = 0, ib = 0, j = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++j) {
-                const int buf = j & 1, ubuf = j >> 1;
-                if (ubuf > 0 && !dev::mbar_wait_bounded(&acce[buf], (ubuf - 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                dev::tc_fence_after();
-                const uint32_t dbase = tmem + (uint32_t)buf * acc_cols;
-                for (int cc8 = 0; cc8 < p.CC8 && ok; ++cc8, ++ia) {
-                    const int sa = ia % p.sa;
-                    if (!dev::mbar_wait_bounded(&fullA[sa], (ia / p.sa) & 1)) {
-                        ok = false;
-                        break;
-                    }
-                    dev::tc_fence_after();
-                    const unsigned char *xa = ringA + (size_t)sa * a_slot;
-                    const uint64_t dah = dev::smem_desc(xa, a_lbo, 128);
-                    const uint64_t dal = dev::smem_desc(xa + p.a_bytes, a_lbo, 128);
-                    for (int r = 0; r < p.R; ++r, ++ib) {
-                        const int sb = ib % p.sb;
-                        if (!dev::mbar_wait_bounded(&fullB[sb], (ib / p.sb) & 1)) {
-                            ok = false;
-                            break;
-                        }
-                        dev::tc_fence_after();
-                        const unsigned char *wb = ringB + (size_t)sb * b_slot;
-                        const uint64_t dbh = dev::smem_desc(wb, b_lbo, 128);
-                        const uint64_t dbl = dev::smem_desc(wb + p.b_bytes, b_lbo, 128);
-                        for (int i = 0; i < p.TH; ++i) {
-                            const uint32_t d = dbase + (uint32_t)(i * NT);
-                            for (int s = 0; s < p.S; ++s) {
-                                // 16-byte units: staged row i + r*dil, column s*dil
-                                const uint64_t ao = (uint64_t)((i + r * p.dil) * p.COLS + s * p.dil);
-                                const uint64_t bo = (uint64_t)(s * 2 * NT);
-                                const uint32_t acc = (cc8 > 0 || r > 0 || s > 0) ? 1u : 0u;
-                                // cross terms x_hi*w_lo + x_lo*w_hi: one bf16 MMA over K = 16
-                                dev::mma_bf16(d, dal + ao, dbl + bo, idesc_c, acc);
-                                // main term x_hi*w_hi: tf32 MMA over K = 8
-                                dev::mma_tf32(d, dah + ao, dbh + bo, idesc, 1u);
-                            }
-                        }
-                        dev::mma_commit(&emptyB[sb]);
-                    }
-                    dev::mma_commit(&emptyA[sa]);
-                }
-                dev::mma_commit(&accf[buf]);   // fires once this tile's MMAs have completed
-            }
+            // loop bounds fixed at compile time for the common geometries
+            // (dilation 1, default rows per tile): the issue loop then runs
+            // back to back on constant operand offsets
+            constexpr int THD = ig_default_th(NT);
+            const bool d1 = p.dil == 1 && p.TH == THD;
+            bool ok;
+            if (d1 && p.R == 3 && p.S == 3) ok = ig_mma_loop<NT, THD, 3, 3>(p, tmem, ringA, ringB, a_slot, b_slot, fullA, emptyA, fullB, emptyB, accf, acce);
+            else if (d1 && p.R == 5 && p.S == 9) ok = ig_mma_loop<NT, THD, 5, 9>(p, tmem, ringA, ringB, a_slot, b_slot, fullA, emptyA, fullB, emptyB, accf, acce);
+            else if (d1 && p.R == 1 && p.S == 1) ok = ig_mma_loop<NT, THD, 1, 1>(p, tmem, ringA, ringB, a_slot, b_slot, fullA, emptyA, fullB, emptyB, accf, acce);
+            else ok = ig_mma_loop<NT, 0, 0, 0>(p, tmem, ringA, ringB, a_slot, b_slot, fullA, emptyA, fullB, emptyB, accf, acce);
             if (!ok) {
                 *abort_flag = 1;
                 atomicExch(&g_igemm_error, 1);
@@ -357,19 +390,26 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
         __syncwarp();
     } else {
         // ---------------------------------------------------------- epilogue
-        // columns: each warp owns NT/4 accumulator columns of its lane quarter,
-        // processed in chunks of CW; chain: GroupNorm groups per chunk (GPC)
-        // and their width inside it (GW)
+        // Warp w reads TMEM lane quarter w % 4 (32 output pixels) and a block
+        // of PART accumulator columns (output channels), in chunks of CW, for
+        // all TH rows of the tile.  Chain: per GroupNorm group of a chunk the
+        // warp sums (a - shift) and (a - shift)^2 per thread in FP32 with one
+        // shift for the whole warp (lane 0's first value), adds the 32 lanes
+        // in FP64 and writes one (count, mean, M2) partial to global memory;
+        // no barrier between epilogue warps.
         constexpr int EPW = ig_epi_warps(NT);
         constexpr int PART = NT / (EPW / 4);
-        constexpr int CW = PART < 16 ? PART : 16;
+        constexpr int CW = ig_chunk_width(NT);
         constexpr int GPC = CHAIN ? (KGN >= CW ? 1 : CW / KGN) : 1;
         constexpr int GW = CHAIN ? (KGN >= CW ? CW : KGN) : CW;
+        constexpr float kLog2e = 1.4426950408889634f;
         const int ew = warp - 2;                 // 0..EPW-1
         const int lq = warp & 3;                 // TMEM lane quarter this warp may access
         const int cpart = ew >> 2;               // column block of this warp
         const int m = lq * 32 + lane;
         const long long plane = (long long)p.P * p.Q;
+        // GroupNorm fragments per group (chunks of CW channels it spans)
+        const int fpg = CHAIN ? (p.kgn > CW ? p.kgn / CW : 1) : 1;
         int j = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++j) {
             const IgTile tl = ig_tile(p, t);
@@ -381,23 +421,28 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
             const bool ok = have && !*(volatile int *)abort_flag;
             const int q = tl.q0 + m;
             const bool qvalid = q < p.Q;
+            const int rows = ok ? min(p.TH, p.P - tl.p0) : 0;   // valid output rows of the tile
             float *ybase = p.y + ((long long)tl.n * p.K + (long long)tl.g * p.kpg) * plane + q;
             const uint32_t tbase = tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)buf * acc_cols;
 #pragma unroll 1
             for (int c0 = cpart * PART; c0 < (cpart + 1) * PART; c0 += CW) {
-                // z = acc * mul + add: plain (mul 1, add bias) or chain (scale, bias*scale)
+                // plain: a = acc + bias.  chain: t = -(acc*scale + bias*scale)*log2(e)
+                // (so that the logistic is 1 / (1 + 2^t)) as acc*mul + add
                 float mul[CW], add[CW];
 #pragma unroll
                 for (int jj = 0; jj < CW; ++jj) {
                     const int k = tl.g * p.kpg + c0 + jj;
                     const float b = p.bias ? __ldg(p.bias + k) : 0.f;
-                    mul[jj] = CHAIN ? __ldg(p.scale + k) : 1.f;
-                    add[jj] = CHAIN ? b * mul[jj] : b;
+                    if constexpr (CHAIN) {
+                        const float sc = __ldg(p.scale + k);
+                        mul[jj] = -sc * kLog2e;
+                        add[jj] = -(b * sc) * kLog2e;
+                    } else {
+                        mul[jj] = 1.f;
+                        add[jj] = b;
+                    }
                 }
-                // shifted sums per GroupNorm group of this chunk (shift = the
-                // group's first value seen by this thread)
                 float shift[GPC], s1[GPC], s2[GPC];
-                float cnt = 0.f;
 #pragma unroll
                 for (int gg = 0; gg < GPC; ++gg) { shift[gg] = 0.f; s1[gg] = 0.f; s2[gg] = 0.f; }
                 // rows are processed two at a time so one TMEM load latency covers both
@@ -411,25 +456,27 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
                     for (int h = 0; h < 2; ++h) {
                         if (h == 1 && !two) break;
                         float *v = vv[h];
-                        const int pp = tl.p0 + i + h;
-                        const bool valid = ok && qvalid && pp < p.P;
+                        const bool rvalid = i + h < rows;            // warp-uniform
+                        if constexpr (CHAIN) {
 #pragma unroll
-                        for (int jj = 0; jj < CW; ++jj) {
-                            float z = fmaf(v[jj], mul[jj], add[jj]);
-                            // logistic; the clamp keeps 1 + e finite (e^80 < 2^126)
-                            if constexpr (CHAIN) z = __fdividef(1.f, 1.f + __expf(fminf(-z, 80.f)));
-                            v[jj] = z;
+                            for (int jj = 0; jj < CW; ++jj) {
+                                // 2^t overflows past 128: clamp keeps 1 + 2^t finite
+                                const float e = ex2_ftz(fminf(fmaf(v[jj], mul[jj], add[jj]), 126.f));
+                                v[jj] = rcp_ftz(1.f + e);
+                            }
+                            if (rvalid && i + h == 0) {
+#pragma unroll
+                                for (int gg = 0; gg < GPC; ++gg) shift[gg] = __shfl_sync(0xffffffffu, v[gg * GW], 0);
+                            }
+                        } else {
+#pragma unroll
+                            for (int jj = 0; jj < CW; ++jj) v[jj] = fmaf(v[jj], mul[jj], add[jj]);
                         }
-                        if (valid) {
-                            float *yr = ybase + (long long)c0 * plane + (long long)pp * p.Q;
+                        if (rvalid && qvalid) {
+                            float *yr = ybase + (long long)c0 * plane + (long long)(tl.p0 + i + h) * p.Q;
 #pragma unroll
                             for (int jj = 0; jj < CW; ++jj) yr[(long long)jj * plane] = v[jj];
                             if constexpr (CHAIN) {
-                                if (cnt == 0.f) {
-#pragma unroll
-                                    for (int gg = 0; gg < GPC; ++gg) shift[gg] = v[gg * GW];
-                                }
-                                cnt += 1.f;
 #pragma unroll
                                 for (int jj = 0; jj < CW; ++jj) {
                                     const float d = v[jj] - shift[jj / GW];
@@ -447,59 +494,27 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
                     if (lane == 0) mbar_arrive(&acce[buf]);
                 }
                 if constexpr (CHAIN) {
-                    // per GroupNorm group in this chunk: raw sums (n, sum a, sum a^2) in
-                    // double, combined over the thread's channels, then a fixed
-                    // shuffle tree over the warp's 32 pixels
+                    const unsigned vmask = __ballot_sync(0xffffffffu, qvalid);
+                    const double cnt = (double)(__popc(vmask) * rows * GW);
 #pragma unroll
                     for (int gg = 0; gg < GPC; ++gg) {
-                        double S1 = 0.0, S2 = 0.0;
-                        if (cnt > 0.f) {
-                            const double n = (double)cnt * GW;
-                            const double a1 = (double)s1[gg];
-                            const double mu = (double)shift[gg] + a1 / n;
-                            const double m2 = fmax((double)s2[gg] - a1 * a1 / n, 0.0);
-                            S1 = n * mu;
-                            S2 = m2 + n * mu * mu;
-                        }
-                        double Nn = (double)cnt * GW;
+                        double S1 = (double)s1[gg], S2 = (double)s2[gg];
 #pragma unroll
                         for (int off = 16; off > 0; off >>= 1) {
-                            const double o1 = __shfl_down_sync(0xffffffffu, S1, off);
-                            const double o2 = __shfl_down_sync(0xffffffffu, S2, off);
-                            const double on = __shfl_down_sync(0xffffffffu, Nn, off);
-                            if (lane < off) { S1 += o1; S2 += o2; Nn += on; }
+                            S1 += __shfl_xor_sync(0xffffffffu, S1, off);
+                            S2 += __shfl_xor_sync(0xffffffffu, S2, off);
                         }
                         if (lane == 0) {
-                            const int fr = (c0 / CW) * GPC + gg;
-                            st_n[fr * 4 + lq] = Nn;
-                            st_1[fr * 4 + lq] = S1;
-                            st_2[fr * 4 + lq] = S2;
+                            const int k0 = tl.g * p.kpg + c0 + gg * GW;   // first channel of the fragment
+                            const int G = k0 / p.kgn;
+                            const int fr = fpg > 1 ? (k0 % p.kgn) / CW : 0;
+                            const double mean = cnt > 0.0 ? (double)shift[gg] + S1 / cnt : 0.0;
+                            const double m2 = cnt > 0.0 ? fmax(S2 - S1 * S1 / cnt, 0.0) : 0.0;
+                            p.gn_part[((long long)tl.n * p.gn_groups + G) * p.slots + (tl.sp * 4 + lq) * fpg + fr] =
+                                make_float4((float)cnt, (float)mean, (float)m2, 0.f);
                         }
                     }
                 }
-            }
-            if constexpr (CHAIN) {
-                epi_sync<EPW>();
-                const int et = tid - 64;
-                const int ngroups = NT / p.kgn;
-                if (et < ngroups) {
-                    // fragments of group et: one per group (width <= CW) or kgn/CW chunks
-                    const int f0 = p.kgn > CW ? et * (p.kgn / CW) : et;
-                    const int f1 = p.kgn > CW ? (et + 1) * (p.kgn / CW) : et + 1;
-                    double Nn = 0.0, S1 = 0.0, S2 = 0.0;
-                    for (int fr = f0; fr < f1; ++fr)
-                        for (int l = 0; l < 4; ++l) {
-                            Nn += st_n[fr * 4 + l];
-                            S1 += st_1[fr * 4 + l];
-                            S2 += st_2[fr * 4 + l];
-                        }
-                    const double mean = Nn > 0.0 ? S1 / Nn : 0.0;
-                    const double m2 = Nn > 0.0 ? fmax(S2 - S1 * mean, 0.0) : 0.0;
-                    const int G = (tl.g * p.kpg) / p.kgn + et;
-                    p.gn_part[((long long)tl.n * p.gn_groups + G) * p.slots + tl.sp] =
-                        make_float4((float)Nn, (float)mean, (float)m2, 0.f);
-                }
-                epi_sync<EPW>();   // statistics scratch free for the next tile
             }
         }
     }
@@ -529,7 +544,7 @@ cudaError_t launch_nt(const IgemmParams &p, const TensorMap *tm, dim3 grid, size
     auto kern = igemm_tf32x3_kernel<NT, KGN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_ex(kern, grid, dim3(ig_threads(NT)), smem, st, tm[0], tm[1], tm[2], tm[3], p);
+    return launch_ex(kern, grid, dim3(ig_threads(NT)), smem, st, tm[0], tm[1], p);
 }
 
 template <int NT>
@@ -567,27 +582,35 @@ int igemm_supported_nt(int kpg) { return kpg == 32 || kpg == 64 || kpg == 128 ||
 
 size_t igemm_header_bytes(int nt, bool chain) { return ig_header(nt, chain); }
 
+int igemm_partials_per_tile(int nt, int kgn) {
+    const int cw = ig_chunk_width(nt);
+    return 4 * (kgn > cw ? kgn / cw : 1);
+}
+
 int igemm_threads(int nt) { return ig_threads(nt); }
 
-bool make_nc4hw4_tensor_map(TensorMap *tm, const float *base, long long quads, int H, int W, int box_px) {
+bool make_nc4hw4_tile_map(TensorMap *tm, const float *base, long long quads, int Hp, int Wp, int box_cols,
+                          int box_rows) {
     auto fn = encode_fn();
-    if (!fn || box_px <= 0 || box_px > 64) return false;
-    // [quads][H][W*4] floats; box = box_px pixels x 4 channels of one row of one quad
-    cuuint64_t dims[3] = {(cuuint64_t)W * 4, (cuuint64_t)H, (cuuint64_t)quads};
-    cuuint64_t strides[2] = {(cuuint64_t)W * 16, (cuuint64_t)W * H * 16};
-    cuuint32_t box[3] = {(cuuint32_t)box_px * 4, 1, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(reinterpret_cast<CUtensorMap *>(tm), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+    if (!fn || Wp % 16 != 0 || box_cols % 16 != 0 || box_cols / 16 > 256 || box_rows < 1 || box_rows > 256)
+        return false;
+    // [quads][Hp][Wp/16][64 floats]: 16 pixels x 4 channels per innermost row
+    cuuint64_t dims[4] = {64, (cuuint64_t)Wp / 16, (cuuint64_t)Hp, (cuuint64_t)quads};
+    cuuint64_t strides[3] = {256, (cuuint64_t)Wp * 16, (cuuint64_t)Wp * Hp * 16};
+    cuuint32_t box[4] = {64, (cuuint32_t)box_cols / 16, (cuuint32_t)box_rows, 2};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(reinterpret_cast<CUtensorMap *>(tm), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
                     const_cast<float *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
-cudaError_t launch_split_x(const float *x, float *xh, float *xl, int N, int C, int H, int W, cudaStream_t st) {
-    const long long cells = (long long)N * (C / 8) * H * W;
+cudaError_t launch_split_x(const float *x, float *xh, float *xl, int N, int C, int H, int W, int pad, int Hp,
+                           int Wp, cudaStream_t st) {
+    const long long cells = (long long)N * (C / 8) * Hp * Wp;
     const long long blocks = std::min<long long>((cells + 255) / 256, 148LL * 64);
     return launch_ex(split_x_kernel, dim3((unsigned)blocks), dim3(256), 0, st, x, reinterpret_cast<float4 *>(xh),
-                     reinterpret_cast<uint4 *>(xl), C / 8, H, W, cells);
+                     reinterpret_cast<uint4 *>(xl), C / 8, H, W, pad, Hp, Wp, cells);
 }
 
 cudaError_t launch_split_w(const float *w, float *wh, float *wl, int K, int cpg, int R, int S, int groups,
