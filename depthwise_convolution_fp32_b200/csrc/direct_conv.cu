@@ -182,13 +182,14 @@ __global__ void __launch_bounds__(256, 2)
         } else {
             __syncthreads();   // the previous pass is done with shared memory
         }
-        // weight slice, transposed to [c][r][s][channel] so KT channels are contiguous
+        // weight slice, transposed to [c][r][s][channel] so KT channels are
+        // contiguous; asynchronous 4-byte copies keep every load in flight at once
         const int nw = cc * RS * p.KBtot;
         for (int e = tid; e < nw; e += blockDim.x) {
             int kl = e % p.KBtot;
             int rest = e / p.KBtot;
             int c = rest / RS, rs = rest - c * RS;
-            sw[e] = __ldg(p.w + ((long long)(kc0 + kl) * p.cpg + c0 + c) * RS + rs);
+            dev::cp_async4(sw + e, p.w + ((long long)(kc0 + kl) * p.cpg + c0 + c) * RS + rs, true);
         }
         if constexpr (FAST && !TMA) {
             const int planes = p.GB * cc;
@@ -222,8 +223,8 @@ __global__ void __launch_bounds__(256, 2)
                     dev::cp_async4(sx + (long long)pl * p.pstride + row * p.pitch + j, src, ok);
                 }
             }
-            dev::cp_async_wait_all();
         }
+        dev::cp_async_wait_all();
         __syncthreads();
         if (!active) continue;
 

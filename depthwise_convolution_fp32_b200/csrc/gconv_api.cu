@@ -83,6 +83,8 @@ const char *geom_name_tma(int geom) {
     }
 }
 
+int env_int(const char *name);   // positive integer from the environment, else 0
+
 bool compat(int a, int b) { return a % b == 0 || b % a == 0; }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -119,12 +121,22 @@ bool plan_direct(const Shape &s, bool chain, int gn_groups, int geom, bool x_vec
     DirectParams &p = pl.prm;
     std::memset(&p, 0, sizeof(p));
 
-    // channels per thread: largest of 8,4,2,1 dividing kpg (and, for the chain,
-    // nesting with the GroupNorm group width)
+    // channels per thread: the largest of 8, 4, 2, 1 dividing kpg (and, for
+    // the chain, nesting with the GroupNorm group width) that still gives the
+    // GPU about 128 threads per SM (the best geometric mean over the 80-shape
+    // sweep among 128, 192, 320 and 512).  A thread's KT channels share every
+    // input value it loads, but on small problems parallelism wins.
     int KT = 1;
     if (fast) {
-        for (int c : {8, 4, 2, 1})
-            if (s.kpg % c == 0 && (!chain || compat(kgn, c))) { KT = c; break; }
+        static const int force_tgt = env_int("GCONV_DIRECT_THREADS_PER_SM");
+        const long long want = (long long)sm_count() * (force_tgt > 0 ? force_tgt : kMaxThreads / 2);
+        for (int c : {8, 4, 2, 1}) {
+            if (s.kpg % c != 0 || (chain && !compat(kgn, c))) continue;
+            KT = c;
+            const long long threads =
+                (long long)s.N * (s.K / c) * ceil_div(s.P, direct_rpt(c)) * ceil_div(s.Q, 4);
+            if (threads >= want) break;
+        }
     }
     const int RPT = fast ? direct_rpt(KT) : direct_rpt(1);
     if (!fast) KT = 1;

@@ -414,9 +414,14 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++j) {
             const IgTile tl = ig_tile(p, t);
             const int buf = j & 1;
-            // after an abort nothing more will be committed: do not wait for it
-            const bool have = !*(volatile int *)abort_flag && dev::mbar_wait_bounded(&accf[buf], (j >> 1) & 1);
-            if (!have) atomicExch(&g_igemm_error, 1);
+            // after an abort nothing more will be committed: do not wait for it.
+            // One lane per warp polls the barrier; the others wait at the shuffle.
+            int have_l = 0;
+            if (lane == 0) {
+                have_l = !*(volatile int *)abort_flag && dev::mbar_wait_bounded(&accf[buf], (j >> 1) & 1);
+                if (!have_l) atomicExch(&g_igemm_error, 1);
+            }
+            const bool have = __shfl_sync(0xffffffffu, have_l, 0) != 0;
             dev::tc_fence_after();
             const bool ok = have && !*(volatile int *)abort_flag;
             const int q = tl.q0 + m;

@@ -80,3 +80,24 @@ def chain_inputs(N, C, H, W, K, R, S, groups, gn_groups, seed, bias_scale_std=0.
         beta = normal((K,), 0.5, g)
     return {"x": x, "w": w, "b_conv": b_conv, "b_extra": b_extra, "scale": scale,
             "gamma": gamma, "beta": beta, "gn_groups": gn_groups}
+
+
+def mobilenet_block_inputs(seed, N=4, cin=24, cexp=144, H=56, W=56):
+    """Random-init parameters and input of one MobileNetV2 inverted-residual
+    block (expansion 6: 1x1 conv cin->cexp, BN, ReLU6, depthwise 3x3, BN,
+    ReLU6, 1x1 conv cexp->cin, residual add), the block the "Fix the
+    experiment" page substitutes one convolution in.
+
+    x ~ N(0,1); conv weights ~ U(+-1/sqrt(fan_in)); each BatchNorm (inference
+    form) has gamma ~ U[0.5,1.5), beta ~ N(0,0.1), running mean ~ N(0,0.1),
+    running var ~ U[0.5,1.5)."""
+    g = generator(seed)
+    x = normal((N, cin, H, W), 1.0, g)
+    w1 = uniform((cexp, cin, 1, 1), -1.0 / math.sqrt(cin), 1.0 / math.sqrt(cin), g)
+    wd = uniform((cexp, 1, 3, 3), -1.0 / 3.0, 1.0 / 3.0, g)
+    w3 = uniform((cin, cexp, 1, 1), -1.0 / math.sqrt(cexp), 1.0 / math.sqrt(cexp), g)
+
+    def bn(c):
+        return {"gamma": uniform((c,), 0.5, 1.5, g), "beta": normal((c,), 0.1, g),
+                "mean": normal((c,), 0.1, g), "var": uniform((c,), 0.5, 1.5, g)}
+    return {"x": x, "w1": w1, "bn1": bn(cexp), "wd": wd, "bn2": bn(cexp), "w3": w3}
