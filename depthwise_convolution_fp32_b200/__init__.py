@@ -46,6 +46,8 @@ def library_path() -> str:
 def library():
     """Load libgconv.so (once).  Raises if it has not been built."""
     global _lib
+    if _lib is not None:
+        return _lib
     with _lock:
         if _lib is not None:
             return _lib
@@ -118,22 +120,38 @@ def chain_workspace_size(N, C, H, W, K, R, S, stride, pad, dilation, groups, gn_
                                                       groups, gn_groups))
 
 
+_torch_mod = None
+_SIZES: dict = {}
+
+
+def _torch():
+    global _torch_mod
+    if _torch_mod is None:
+        import torch
+        _torch_mod = torch
+    return _torch_mod
+
+
 def _dev(t, name, allow_none=False):
     if t is None:
         if allow_none:
             return None
         raise ValueError(f"{name} is required")
-    import torch
+    torch = _torch()
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+    if not (t.is_cuda and t.dtype is torch.float32 and t.is_contiguous()):
         raise ValueError(f"{name} must be a contiguous float32 CUDA tensor "
                          f"(got device={t.device}, dtype={t.dtype}, contiguous={t.is_contiguous()})")
     return t.data_ptr()
 
 
 def _stream(t):
-    import torch
+    """The raw handle of the current stream on t's device."""
+    torch = _torch()
+    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+    if raw is not None:
+        return ctypes.c_void_p(raw(t.get_device()))
     return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
 
 
@@ -145,24 +163,42 @@ def _scalar(v, name):
     return int(v)
 
 
+def _out_size(H, W, R, S, stride, padding, dilation):
+    key = (H, W, R, S, stride, padding, dilation)
+    pq = _SIZES.get(key)
+    if pq is None:
+        pq = output_size(H, W, R, S, stride, padding, dilation)
+        if len(_SIZES) > 4096:
+            _SIZES.clear()
+        _SIZES[key] = pq
+    return pq
+
+
+def _output(x, out, shape):
+    if out is None:
+        if x.dtype is not _torch().float32:
+            raise ValueError("x must be a contiguous float32 CUDA tensor")
+        return x.new_empty(shape)
+    if tuple(out.shape) != shape:
+        raise ValueError(f"out must have shape {shape}")
+    return out
+
+
 def conv2d(x, w, bias=None, stride=1, padding=0, dilation=1, groups=1, out=None):
     """y = conv2d(x, w) (+ bias) on the GPU; x[N,C,H,W], w[K,C/groups,R,S]."""
-    import torch
     N, C, H, W = x.shape
     K, cpg, R, S = w.shape
     stride, padding, dilation = (_scalar(stride, "stride"), _scalar(padding, "padding"),
                                  _scalar(dilation, "dilation"))
     if cpg * groups != C:
         raise ValueError("w.shape[1] * groups must equal C")
-    P, Q = output_size(H, W, R, S, stride, padding, dilation)
-    if out is None:
-        out = torch.empty((N, K, P, Q), device=x.device, dtype=torch.float32)
-    elif tuple(out.shape) != (N, K, P, Q):
-        raise ValueError(f"out must have shape {(N, K, P, Q)}")
+    P, Q = _out_size(H, W, R, S, stride, padding, dilation)
+    out = _output(x, out, (N, K, P, Q))
     st = library().gconv2d_fwd(_dev(x, "x"), _dev(w, "w"), _dev(bias, "bias", True),
                                N, C, H, W, K, R, S, stride, padding, dilation, groups,
                                _dev(out, "out"), _stream(x))
-    _check(st, "gconv2d_fwd")
+    if st:
+        _check(st, "gconv2d_fwd")
     return out
 
 
@@ -172,21 +208,17 @@ def conv2d_bias_scale_sigmoid_groupnorm(x, w, bias, scale, gn_groups, gamma, bet
 
     bias ([K] or None) is the folded conv bias + extra bias; scale, gamma and
     beta are [K] (a [K,1,1] view is accepted)."""
-    import torch
     N, C, H, W = x.shape
     K, cpg, R, S = w.shape
     stride, padding, dilation = (_scalar(stride, "stride"), _scalar(padding, "padding"),
                                  _scalar(dilation, "dilation"))
     if cpg * groups != C:
         raise ValueError("w.shape[1] * groups must equal C")
-    P, Q = output_size(H, W, R, S, stride, padding, dilation)
+    P, Q = _out_size(H, W, R, S, stride, padding, dilation)
     for name, t in (("bias", bias), ("scale", scale), ("gamma", gamma), ("beta", beta)):
         if t is not None and t.numel() != K:
             raise ValueError(f"{name} must hold K={K} values")
-    if out is None:
-        out = torch.empty((N, K, P, Q), device=x.device, dtype=torch.float32)
-    elif tuple(out.shape) != (N, K, P, Q):
-        raise ValueError(f"out must have shape {(N, K, P, Q)}")
+    out = _output(x, out, (N, K, P, Q))
     st = library().gconv2d_bias_scale_sigmoid_groupnorm_fwd(
         _dev(x, "x"), _dev(w, "w"), _dev(bias, "bias", True),
         N, C, H, W, K, R, S, stride, padding, dilation, groups,

@@ -294,6 +294,64 @@ bool choose_direct(const Shape &s, bool chain, int gn_groups, bool x_vec, Direct
     return false;
 }
 
+// Per-thread caches for repeated calls of the plain convolution: the last
+// few direct plans by shape (planning walks several tile candidates), and the
+// last TMA descriptor by input pointer and box (encoding goes through the
+// driver).  Keys hold everything the cached value depends on.
+struct DirectKey {
+    int v[11];
+    int x_vec, force, dev, sms;
+    bool operator==(const DirectKey &o) const { return std::memcmp(this, &o, sizeof(*this)) == 0; }
+};
+
+bool cached_direct_plan(const Shape &s, bool x_vec, DirectPlan &pl) {
+    struct Entry {
+        DirectKey key;
+        DirectPlan plan;
+        bool valid;
+    };
+    thread_local Entry cache[4] = {};
+    thread_local int next = 0;
+    DirectKey k;
+    std::memset(&k, 0, sizeof(k));
+    const int vals[11] = {s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil, s.groups};
+    std::memcpy(k.v, vals, sizeof(vals));
+    k.x_vec = x_vec ? 1 : 0;
+    k.force = g_force.load(std::memory_order_relaxed);
+    if (cudaGetDevice(&k.dev) != cudaSuccess) return false;
+    k.sms = sm_count();
+    for (const Entry &e : cache)
+        if (e.valid && e.key == k) {
+            pl = e.plan;
+            return true;
+        }
+    if (!choose_direct(s, false, 1, x_vec, pl)) return false;
+    cache[next] = Entry{k, pl, true};
+    next = (next + 1) % 4;
+    return true;
+}
+
+bool cached_x_tensor_map(TensorMap *tm, const float *x, long long planes, int H, int W, int box_w, int box_h) {
+    struct Entry {
+        const float *x;
+        long long planes;
+        int H, W, box_w, box_h, dev;
+        TensorMap tm;
+        bool valid;
+    };
+    thread_local Entry last = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    if (last.valid && last.x == x && last.planes == planes && last.H == H && last.W == W && last.box_w == box_w &&
+        last.box_h == box_h && last.dev == dev) {
+        *tm = last.tm;
+        return true;
+    }
+    if (!make_x_tensor_map(tm, x, planes, H, W, box_w, box_h)) return false;
+    last = Entry{x, planes, H, W, box_w, box_h, dev, *tm, true};
+    return true;
+}
+
 // Fill the pointer-dependent fields and the TMA descriptor of a plan; a map
 // the driver rejects falls back to cp.async staging.
 bool finish_plan(const Shape &s, bool chain, int gn_groups, const float *x, float *y, DirectPlan &pl,
@@ -302,7 +360,7 @@ bool finish_plan(const Shape &s, bool chain, int gn_groups, const float *x, floa
     p.vec_in = (s.W % 4 == 0) && aligned16(x);
     p.vec_out = (s.Q % 4 == 0) && aligned16(y);
     std::memset(&tm, 0, sizeof(tm));
-    if (p.tma && !make_x_tensor_map(&tm, x, (long long)s.N * s.C, s.H, s.W, 4 * p.PC, p.bh)) {
+    if (p.tma && !cached_x_tensor_map(&tm, x, (long long)s.N * s.C, s.H, s.W, 4 * p.PC, p.bh)) {
         DirectPlan again;
         if (!plan_direct(s, chain, gn_groups, pl.geom, false, again)) return false;
         again.prm.vec_in = p.vec_in;
@@ -593,7 +651,7 @@ gconv_status_t gconv2d_fwd(const float *x, const float *w, const float *bias, in
     if (g_force.load(std::memory_order_relaxed) == kForceIgemm) return GCONV_ERR_UNSUPPORTED;
     DirectPlan pl;
     const bool x_vec = (s.W % 4 == 0) && aligned16(x);
-    if (!choose_direct(s, false, 1, x_vec, pl)) return GCONV_ERR_UNSUPPORTED;
+    if (!cached_direct_plan(s, x_vec, pl)) return GCONV_ERR_UNSUPPORTED;
     TensorMap tm;
     if (!finish_plan(s, false, 1, x, y, pl, tm)) return GCONV_ERR_UNSUPPORTED;
     DirectParams &p = pl.prm;

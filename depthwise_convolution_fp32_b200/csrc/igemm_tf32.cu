@@ -43,6 +43,8 @@
 //                   chain's +bias, *scale, logistic and GroupNorm partial
 //                   statistics, coalesced stores along q; two TMEM
 //                   accumulator buffers let it overlap the next tile's MMAs.
+#include <atomic>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -547,8 +549,18 @@ cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_
 template <int NT, int KGN>
 cudaError_t launch_nt(const IgemmParams &p, const TensorMap *tm, dim3 grid, size_t smem, cudaStream_t st) {
     auto kern = igemm_tf32x3_kernel<NT, KGN>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    // the shared-memory opt-in is per function and device: raise it to the
+    // planner's ceiling once per device instead of on every launch
+    static std::atomic<unsigned long long> opted{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    const unsigned long long bit = dev < 64 ? 1ull << dev : 0;
+    if (!bit || !(opted.load(std::memory_order_acquire) & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return e;
+        if (bit) opted.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    if (smem > 227 * 1024) return cudaErrorInvalidValue;
     return launch_ex(kern, grid, dim3(ig_threads(NT)), smem, st, tm[0], tm[1], p);
 }
 
