@@ -64,15 +64,19 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback", {}
 
 
-def kernel_source_hash() -> str:
-    """Hash of the CUDA sources; a stored ncu traffic figure is only valid for
-    the sources it was captured from."""
+KERNEL_TU = {"depthwise": "direct_conv.cu", "tiny_grouped": "direct_conv.cu",
+             "dense_5x9": "igemm_tf32.cu", "fused_chain": "igemm_tf32.cu"}
+
+
+def kernel_source_hash(tu: str) -> str:
+    """Hash of one kernel translation unit and the headers every kernel
+    includes; a stored ncu traffic figure is only valid for the sources it
+    was captured from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "depthwise_convolution_fp32_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".h", ".cuh")):
-            h.update(f.encode())
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in (tu, "device_utils.cuh", "gconv_internal.h"):
+        h.update(f.encode())
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -83,7 +87,7 @@ def stored_traffic(workload: str):
     try:
         d = json.load(open(path))
         e = d[workload]
-        if e.get("source_hash") != kernel_source_hash():
+        if e.get("source_hash") != kernel_source_hash(KERNEL_TU[workload]):
             return None
         return float(e["dram_bytes_per_launch"])
     except Exception:
