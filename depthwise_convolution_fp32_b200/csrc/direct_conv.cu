@@ -184,43 +184,56 @@ __global__ void __launch_bounds__(256, 2)
         }
         // weight slice, transposed to [c][r][s][channel] so KT channels are
         // contiguous; asynchronous 4-byte copies keep every load in flight at once
-        const int nw = cc * RS * p.KBtot;
-        for (int e = tid; e < nw; e += blockDim.x) {
-            int kl = e % p.KBtot;
-            int rest = e / p.KBtot;
-            int c = rest / RS, rs = rest - c * RS;
-            dev::cp_async4(sw + e, p.w + ((long long)(kc0 + kl) * p.cpg + c0 + c) * RS + rs, true);
+        {
+            // element e = (c * RS + rs) * KBtot + kl, walked incrementally like the x tile
+            const int nw = cc * RS * p.KBtot;
+            const int step = blockDim.x;
+            const int dq = step / p.KBtot, dr = step - dq * p.KBtot;
+            int kl = tid % p.KBtot, rs = tid / p.KBtot, c = 0;
+            while (rs >= RS) { rs -= RS; ++c; }
+            for (int e = tid; e < nw; e += step) {
+                dev::cp_async4(sw + e, p.w + ((long long)(kc0 + kl) * p.cpg + c0 + c) * RS + rs, true);
+                kl += dr;
+                rs += dq;
+                if (kl >= p.KBtot) { kl -= p.KBtot; ++rs; }
+                while (rs >= RS) { rs -= RS; ++c; }
+            }
         }
         if constexpr (FAST && !TMA) {
+            // element e = ((plane * IHt) + row) * cols + col, strided by the
+            // block size; the coordinates advance incrementally (no division
+            // per element: with 4-byte copies the divisions dominated the
+            // kernel's instruction count)
             const int planes = p.GB * cc;
-            if (p.vec_in) {
-                const int total = planes * p.IHt * p.PC;
-                for (int e = tid; e < total; e += blockDim.x) {
-                    int ch = e % p.PC;
-                    int rest = e / p.PC;
-                    int row = rest % p.IHt;
-                    int pl = rest / p.IHt;
-                    int gbb = pl / cc, c = pl - gbb * cc;
-                    int ci = (g0 + gbb) * p.cpg + c0 + c;
-                    int ih = ih0 + row, iw = iw0 + 4 * ch;
-                    bool ok = ih >= 0 && ih < p.H && iw >= 0 && iw < p.W;
+            const int cols = p.vec_in ? p.PC : 4 * p.PC;      // 16-byte chunks or floats per row
+            const int total = planes * p.IHt * cols;
+            const int step = blockDim.x;
+            const int dq = step / cols, dr = step - dq * cols;  // step = dq rows + dr columns
+            int col = tid % cols, row = tid / cols, pl = 0;
+            while (row >= p.IHt) { row -= p.IHt; ++pl; }
+            int c = pl % cc, gbb = pl / cc;
+            for (int e = tid; e < total; e += step) {
+                const int ci = (g0 + gbb) * p.cpg + c0 + c;
+                const int ih = ih0 + row;
+                float *dst = sx + (long long)pl * p.pstride + row * p.pitch;
+                if (p.vec_in) {
+                    const int iw = iw0 + 4 * col;
+                    const bool ok = ih >= 0 && ih < p.H && iw >= 0 && iw < p.W;
                     const float *src = ok ? p.x + (((long long)n * p.C + ci) * p.H + ih) * p.W + iw : p.x;
-                    dev::cp_async16(sx + (long long)pl * p.pstride + row * p.pitch + 4 * ch, src, ok);
+                    dev::cp_async16(dst + 4 * col, src, ok);
+                } else {
+                    const int iw = iw0 + col;
+                    const bool ok = ih >= 0 && ih < p.H && iw >= 0 && iw < p.W;
+                    const float *src = ok ? p.x + (((long long)n * p.C + ci) * p.H + ih) * p.W + iw : p.x;
+                    dev::cp_async4(dst + col, src, ok);
                 }
-            } else {
-                const int cols = 4 * p.PC;
-                const int total = planes * p.IHt * cols;
-                for (int e = tid; e < total; e += blockDim.x) {
-                    int j = e % cols;
-                    int rest = e / cols;
-                    int row = rest % p.IHt;
-                    int pl = rest / p.IHt;
-                    int gbb = pl / cc, c = pl - gbb * cc;
-                    int ci = (g0 + gbb) * p.cpg + c0 + c;
-                    int ih = ih0 + row, iw = iw0 + j;
-                    bool ok = ih >= 0 && ih < p.H && iw >= 0 && iw < p.W;
-                    const float *src = ok ? p.x + (((long long)n * p.C + ci) * p.H + ih) * p.W + iw : p.x;
-                    dev::cp_async4(sx + (long long)pl * p.pstride + row * p.pitch + j, src, ok);
+                col += dr;
+                row += dq;
+                if (col >= cols) { col -= cols; ++row; }
+                while (row >= p.IHt) {
+                    row -= p.IHt;
+                    ++pl;
+                    if (++c == cc) { c = 0; ++gbb; }
                 }
             }
         }
