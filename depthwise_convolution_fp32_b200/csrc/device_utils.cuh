@@ -32,6 +32,13 @@ __device__ __forceinline__ void cp_async16(float *sdst, const float *gsrc, bool 
                  : "memory");
 }
 
+__device__ __forceinline__ void cp_async8(float *sdst, const float *gsrc, bool valid) {
+    int nbytes = valid ? 8 : 0;
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(smem_addr(sdst)), "l"(gsrc),
+                 "r"(nbytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ void cp_async4(float *sdst, const float *gsrc, bool valid) {
     int nbytes = valid ? 4 : 0;
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(smem_addr(sdst)), "l"(gsrc),

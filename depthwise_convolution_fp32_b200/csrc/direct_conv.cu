@@ -205,7 +205,8 @@ __global__ void __launch_bounds__(256, 2)
             // per element: with 4-byte copies the divisions dominated the
             // kernel's instruction count)
             const int planes = p.GB * cc;
-            const int cols = p.vec_in ? p.PC : 4 * p.PC;      // 16-byte chunks or floats per row
+            // 16-byte chunks, 8-byte pairs or floats per row
+            const int cols = p.vec_in ? p.PC : (p.vec2_in ? 2 * p.PC : 4 * p.PC);
             const int total = planes * p.IHt * cols;
             const int step = blockDim.x;
             const int dq = step / cols, dr = step - dq * cols;  // step = dq rows + dr columns
@@ -221,6 +222,12 @@ __global__ void __launch_bounds__(256, 2)
                     const bool ok = ih >= 0 && ih < p.H && iw >= 0 && iw < p.W;
                     const float *src = ok ? p.x + (((long long)n * p.C + ci) * p.H + ih) * p.W + iw : p.x;
                     dev::cp_async16(dst + 4 * col, src, ok);
+                } else if (p.vec2_in) {
+                    // W even and iw0 a multiple of 4: a pair never straddles the image edge
+                    const int iw = iw0 + 2 * col;
+                    const bool ok = ih >= 0 && ih < p.H && iw >= 0 && iw < p.W;
+                    const float *src = ok ? p.x + (((long long)n * p.C + ci) * p.H + ih) * p.W + iw : p.x;
+                    dev::cp_async8(dst + 2 * col, src, ok);
                 } else {
                     const int iw = iw0 + col;
                     const bool ok = ih >= 0 && ih < p.H && iw >= 0 && iw < p.W;

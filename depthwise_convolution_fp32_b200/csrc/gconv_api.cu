@@ -358,12 +358,14 @@ bool finish_plan(const Shape &s, bool chain, int gn_groups, const float *x, floa
                  TensorMap &tm) {
     DirectParams &p = pl.prm;
     p.vec_in = (s.W % 4 == 0) && aligned16(x);
+    p.vec2_in = !p.vec_in && (s.W % 2 == 0) && (reinterpret_cast<uintptr_t>(x) & 7u) == 0;
     p.vec_out = (s.Q % 4 == 0) && aligned16(y);
     std::memset(&tm, 0, sizeof(tm));
     if (p.tma && !cached_x_tensor_map(&tm, x, (long long)s.N * s.C, s.H, s.W, 4 * p.PC, p.bh)) {
         DirectPlan again;
         if (!plan_direct(s, chain, gn_groups, pl.geom, false, again)) return false;
         again.prm.vec_in = p.vec_in;
+        again.prm.vec2_in = p.vec2_in;
         again.prm.vec_out = p.vec_out;
         pl = again;
     }

@@ -43,6 +43,7 @@ struct DirectParams {
     int cchunk;       // input channels staged per pass
     int w_floats;     // floats reserved for the weight slice (multiple of 4)
     int vec_in;       // x rows are 16-byte aligned (16-byte cp.async staging)
+    int vec2_in;      // else: W even and x 8-byte aligned (8-byte cp.async staging)
     int vec_out;      // y rows are 16-byte aligned (float4 stores)
 
     // TMA staging (tma != 0): the tile's rows are fetched as nb bands of bh
