@@ -662,7 +662,8 @@ def main():
 def measure_block(device, steps, warmup):
     """One MobileNetV2 inverted-residual block x[4,24,56,56] (1x1 24->144, BN,
     ReLU6, depthwise 3x3, BN, ReLU6, 1x1 144->24, residual add), forward with
-    PyTorch's depthwise convolution and with this library's, timed both ways
+    PyTorch's depthwise convolution, with this library's, and with this
+    library's depthwise convolution + BatchNorm + ReLU6 in one call, timed both ways
     the pages distinguish: `steps` forwards replayed from one CUDA graph
     (device events), and eager forwards each followed by a synchronize
     (host clock).  Activations stay L2-resident for both variants alike."""
@@ -672,18 +673,22 @@ def measure_block(device, steps, warmup):
     x = prm.pop("x").to(device)
     prm = block.to_device(prm, device)
     out = {}
-    for name, dw in (("library", block.library_depthwise), ("torch", block.torch_depthwise)):
+    folded = block.fold_bn(prm["bn2"])
+    variants = (("library", lambda: block.forward(x, prm, block.library_depthwise)),
+                ("library_fused_bn_relu6", lambda: block.forward_fused(x, prm, folded)),
+                ("torch", lambda: block.forward(x, prm, block.torch_depthwise)))
+    for name, fwd in variants:
         for _ in range(max(3, warmup)):
-            block.forward(x, prm, dw)
+            fwd()
         torch.cuda.synchronize()
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
-            block.forward(x, prm, dw)
+            fwd()
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=s):
                 for _ in range(steps):
-                    block.forward(x, prm, dw)
+                    fwd()
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
         g.replay()
@@ -698,17 +703,21 @@ def measure_block(device, steps, warmup):
         n_sync = max(20, steps // 2)
         t0 = time.perf_counter()
         for _ in range(n_sync):
-            block.forward(x, prm, dw)
+            fwd()
             torch.cuda.synchronize()
         sync_us = (time.perf_counter() - t0) * 1e6 / n_sync
         out[name] = (graph_us, sync_us)
     y_lib = block.forward(x, prm, block.library_depthwise)
+    y_fused = block.forward_fused(x, prm, folded)
     y_ref = block.forward(x, prm, block.torch_depthwise)
     return {"x": list(x.shape), "graph_us": {k: round(v[0], 3) for k, v in out.items()},
             "sync_us": {k: round(v[1], 3) for k, v in out.items()},
             "speedup_graph": round(out["torch"][0] / out["library"][0], 3),
             "speedup_sync": round(out["torch"][1] / out["library"][1], 3),
+            "speedup_graph_fused": round(out["torch"][0] / out["library_fused_bn_relu6"][0], 3),
+            "speedup_sync_fused": round(out["torch"][1] / out["library_fused_bn_relu6"][1], 3),
             "max_abs_diff_vs_torch": float((y_lib - y_ref).abs().max()),
+            "max_abs_diff_fused_vs_torch": float((y_fused - y_ref).abs().max()),
             "pages_reported": {"speedup_graph": 1.14, "speedup_sync": 0.68, "gpu": "RTX 4090"}}
 
 

@@ -16,7 +16,7 @@ import os
 import threading
 
 __all__ = [
-    "GconvError", "conv2d", "conv2d_bias_scale_sigmoid_groupnorm", "output_size",
+    "GconvError", "conv2d", "conv2d_affine_clamp", "conv2d_bias_scale_sigmoid_groupnorm", "output_size",
     "plan_name", "force_kernel", "reserve_workspace", "chain_workspace_size",
     "library", "library_path", "status_string", "version",
     "OK", "ERR_INVALID_ARG", "ERR_UNSUPPORTED", "ERR_CUDA", "ERR_WORKSPACE", "ERR_TIMEOUT",
@@ -66,6 +66,8 @@ def library():
         lib.gconv2d_output_size.argtypes = [i] * 7 + [ctypes.POINTER(i), ctypes.POINTER(i)]
         lib.gconv2d_fwd.restype = i
         lib.gconv2d_fwd.argtypes = [p, p, p] + geo + [p, p]
+        lib.gconv2d_affine_clamp_fwd.restype = i
+        lib.gconv2d_affine_clamp_fwd.argtypes = [p, p] + geo + [p, p, f, f, p, p]
         lib.gconv2d_bias_scale_sigmoid_groupnorm_fwd.restype = i
         lib.gconv2d_bias_scale_sigmoid_groupnorm_fwd.argtypes = [p, p, p] + geo + [p, i, p, p, f, p, p]
         lib.gconv2d_chain_workspace_size.restype = sz
@@ -199,6 +201,31 @@ def conv2d(x, w, bias=None, stride=1, padding=0, dilation=1, groups=1, out=None)
                                _dev(out, "out"), _stream(x))
     if st:
         _check(st, "gconv2d_fwd")
+    return out
+
+
+def conv2d_affine_clamp(x, w, scale=None, shift=None, lo=float("-inf"), hi=float("inf"), stride=1,
+                        padding=0, dilation=1, groups=1, out=None):
+    """y = clamp(conv2d(x, w) * scale[k] + shift[k], lo, hi) on the GPU (scale /
+    shift [K] or None for 1 / 0).  With BatchNorm folded into scale and shift
+    and lo=0, hi=6 this is a convolution + BatchNorm + ReLU6 in one kernel."""
+    N, C, H, W = x.shape
+    K, cpg, R, S = w.shape
+    stride, padding, dilation = (_scalar(stride, "stride"), _scalar(padding, "padding"),
+                                 _scalar(dilation, "dilation"))
+    if cpg * groups != C:
+        raise ValueError("w.shape[1] * groups must equal C")
+    for name, t in (("scale", scale), ("shift", shift)):
+        if t is not None and t.numel() != K:
+            raise ValueError(f"{name} must hold K={K} values")
+    P, Q = _out_size(H, W, R, S, stride, padding, dilation)
+    out = _output(x, out, (N, K, P, Q))
+    st = library().gconv2d_affine_clamp_fwd(_dev(x, "x"), _dev(w, "w"),
+                                            N, C, H, W, K, R, S, stride, padding, dilation, groups,
+                                            _dev(scale, "scale", True), _dev(shift, "shift", True),
+                                            float(lo), float(hi), _dev(out, "out"), _stream(x))
+    if st:
+        _check(st, "gconv2d_affine_clamp_fwd")
     return out
 
 

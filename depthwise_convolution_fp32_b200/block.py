@@ -48,3 +48,19 @@ def library_depthwise(h, wd):
 
 def forward(x, p, dw) -> torch.Tensor:
     return project(x, dw(expand(x, p), p["wd"]), p)
+
+
+def fold_bn(p, eps=1e-5):
+    """BatchNorm (inference form) as a per-channel scale and shift."""
+    scale = p["gamma"] / torch.sqrt(p["var"] + eps)
+    return scale.contiguous(), (p["beta"] - p["mean"] * scale).contiguous()
+
+
+def forward_fused(x, p, folded=None) -> torch.Tensor:
+    """The block with this library's depthwise convolution, BN and ReLU6 in one
+    call (conv2d_affine_clamp); `folded` = fold_bn(p["bn2"]) may be passed in."""
+    import depthwise_convolution_fp32_b200 as gc
+    sc, sh = folded if folded is not None else fold_bn(p["bn2"])
+    h = expand(x, p)
+    d = gc.conv2d_affine_clamp(h, p["wd"], sc, sh, 0.0, 6.0, 1, 1, 1, p["wd"].shape[0])
+    return x + F.conv2d(d, p["w3"])

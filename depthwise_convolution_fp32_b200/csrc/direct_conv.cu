@@ -329,12 +329,20 @@ __global__ void __launch_bounds__(256, 2)
             const float b = p.bias ? __ldg(p.bias + kk) : 0.f;
             float sc = 1.f;
             if constexpr (CHAIN) sc = __ldg(p.scale + kk);
+            else if (p.aff_scale) sc = __ldg(p.aff_scale + kk);
 #pragma unroll
             for (int rp = 0; rp < RPT; ++rp)
 #pragma unroll
                 for (int v = 0; v < kV; ++v) {
-                    float z = acc[rp][v][k] + b;
-                    if constexpr (CHAIN) z = __frcp_rn(1.f + __expf(-(z * sc)));
+                    float z;
+                    if constexpr (CHAIN) {
+                        z = acc[rp][v][k] + b;
+                        z = __frcp_rn(1.f + __expf(-(z * sc)));
+                    } else {
+                        // plain: acc + bias; affine epilogue: one rounding of acc * scale + shift
+                        z = p.aff_scale ? fmaf(acc[rp][v][k], sc, b) : acc[rp][v][k] + b;
+                        if (p.clamp) z = fminf(fmaxf(z, p.lo), p.hi);
+                    }
                     acc[rp][v][k] = z;
                 }
         }

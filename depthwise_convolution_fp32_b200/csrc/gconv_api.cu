@@ -3,6 +3,7 @@
 // entry points of the FP32 NCHW conv2d forward and the fused
 // conv -> bias -> scale -> sigmoid -> GroupNorm chain.
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -544,7 +545,7 @@ gconv_status_t run_igemm(const Shape &s, IgemmPlan &pl, const float *x, const fl
     p.bias = bias;
     p.scale = scale;
     p.y = y;
-    const bool chain = scale != nullptr;
+    const bool chain = gn_groups > 0;
     p.gn_part = chain ? reinterpret_cast<float4 *>(base + pl.off_part) : nullptr;
     if (launch_split_x(x, xh, xl, s.N, s.C, s.H, s.W, s.pad, p.Hp, p.Wp, stream) != cudaSuccess)
         return GCONV_ERR_CUDA;
@@ -571,6 +572,43 @@ gconv_status_t validate_ptrs(const float *x, const float *w, const float *y) {
     if (!x || !w || !y) return GCONV_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(y)) & 3u)
         return GCONV_ERR_INVALID_ARG;
+    return GCONV_OK;
+}
+
+// Plain convolution, optionally with the affine + clamp epilogue.
+gconv_status_t conv_fwd(const float *x, const float *w, const float *bias, const float *aff_scale, int clamp,
+                        float lo, float hi, int N, int C, int H, int W, int K, int R, int S, int stride, int pad,
+                        int dilation, int groups, float *y, cudaStream_t stream) {
+    Shape s;
+    gconv_status_t st = make_shape(s, N, C, H, W, K, R, S, stride, pad, dilation, groups);
+    if (st != GCONV_OK) return st;
+    if ((st = validate_ptrs(x, w, y)) != GCONV_OK) return st;
+    if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) return GCONV_ERR_INVALID_ARG;
+    if (aff_scale && (reinterpret_cast<uintptr_t>(aff_scale) & 3u)) return GCONV_ERR_INVALID_ARG;
+    IgemmPlan ig;
+    if (use_igemm(s, false, 1, ig)) {
+        void *ws = nullptr;
+        if ((st = ensure_workspace(ig.ws_bytes, stream, &ws)) != GCONV_OK) return st;
+        ig.prm.aff_scale = aff_scale;
+        ig.prm.clamp = clamp;
+        ig.prm.lo = lo;
+        ig.prm.hi = hi;
+        return run_igemm(s, ig, x, w, bias, nullptr, 0, nullptr, nullptr, 0.f, y, ws, stream);
+    }
+    if (g_force.load(std::memory_order_relaxed) == kForceIgemm) return GCONV_ERR_UNSUPPORTED;
+    DirectPlan pl;
+    const bool x_vec = (s.W % 4 == 0) && aligned16(x);
+    if (!cached_direct_plan(s, x_vec, pl)) return GCONV_ERR_UNSUPPORTED;
+    TensorMap tm;
+    if (!finish_plan(s, false, 1, x, y, pl, tm)) return GCONV_ERR_UNSUPPORTED;
+    DirectParams &p = pl.prm;
+    p.x = x; p.w = w; p.bias = bias; p.y = y;
+    p.aff_scale = aff_scale;
+    p.clamp = clamp;
+    p.lo = lo;
+    p.hi = hi;
+    if (launch_direct(p, tm, pl.geom, pl.KT, 0, pl.grid, pl.threads, pl.smem, stream) != cudaSuccess)
+        return GCONV_ERR_CUDA;
     return GCONV_OK;
 }
 
@@ -639,28 +677,16 @@ const char *gconv2d_plan_name(int N, int C, int H, int W, int K, int R, int S, i
 gconv_status_t gconv2d_fwd(const float *x, const float *w, const float *bias, int N, int C, int H, int W, int K,
                            int R, int S, int stride, int pad, int dilation, int groups, float *y,
                            cudaStream_t stream) {
-    Shape s;
-    gconv_status_t st = make_shape(s, N, C, H, W, K, R, S, stride, pad, dilation, groups);
-    if (st != GCONV_OK) return st;
-    if ((st = validate_ptrs(x, w, y)) != GCONV_OK) return st;
-    if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) return GCONV_ERR_INVALID_ARG;
-    IgemmPlan ig;
-    if (use_igemm(s, false, 1, ig)) {
-        void *ws = nullptr;
-        if ((st = ensure_workspace(ig.ws_bytes, stream, &ws)) != GCONV_OK) return st;
-        return run_igemm(s, ig, x, w, bias, nullptr, 0, nullptr, nullptr, 0.f, y, ws, stream);
-    }
-    if (g_force.load(std::memory_order_relaxed) == kForceIgemm) return GCONV_ERR_UNSUPPORTED;
-    DirectPlan pl;
-    const bool x_vec = (s.W % 4 == 0) && aligned16(x);
-    if (!cached_direct_plan(s, x_vec, pl)) return GCONV_ERR_UNSUPPORTED;
-    TensorMap tm;
-    if (!finish_plan(s, false, 1, x, y, pl, tm)) return GCONV_ERR_UNSUPPORTED;
-    DirectParams &p = pl.prm;
-    p.x = x; p.w = w; p.bias = bias; p.y = y;
-    if (launch_direct(p, tm, pl.geom, pl.KT, 0, pl.grid, pl.threads, pl.smem, stream) != cudaSuccess)
-        return GCONV_ERR_CUDA;
-    return GCONV_OK;
+    return conv_fwd(x, w, bias, nullptr, 0, 0.f, 0.f, N, C, H, W, K, R, S, stride, pad, dilation, groups, y, stream);
+}
+
+gconv_status_t gconv2d_affine_clamp_fwd(const float *x, const float *w, int N, int C, int H, int W, int K, int R,
+                                        int S, int stride, int pad, int dilation, int groups, const float *scale,
+                                        const float *shift, float lo, float hi, float *y, cudaStream_t stream) {
+    if (!(lo <= hi)) return GCONV_ERR_INVALID_ARG;   // also rejects NaN bounds
+    const int clamp = (lo > -INFINITY || hi < INFINITY) ? 1 : 0;
+    return conv_fwd(x, w, shift, scale, clamp, lo, hi, N, C, H, W, K, R, S, stride, pad, dilation, groups, y,
+                    stream);
 }
 
 size_t gconv2d_chain_workspace_size(int N, int C, int H, int W, int K, int R, int S, int stride, int pad,

@@ -56,6 +56,11 @@ struct DirectParams {
 
     // chain bookkeeping
     int gn_groups, kgn, slots, slots_k, n_sp;
+
+    // plain convolution epilogue: y = clamp(acc * aff_scale[k] + bias[k], lo, hi)
+    const float *aff_scale;   // null: 1
+    int clamp;                // apply [lo, hi]
+    float lo, hi;
 };
 
 struct GnParams {
@@ -111,6 +116,10 @@ struct IgemmParams {
     int a_bytes, b_bytes;      // one x operand (hi or lo) tile / one w operand slice
     int tmem_cols;
     int gn_groups, kgn, slots;  // chain: partials per (image, group) = tiles per image x per-tile partials
+    // plain convolution epilogue: y = clamp(acc * aff_scale[k] + bias[k], lo, hi)
+    const float *aff_scale;    // null: 1
+    int clamp;
+    float lo, hi;
 };
 
 int igemm_supported_nt(int kpg);

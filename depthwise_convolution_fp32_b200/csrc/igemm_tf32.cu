@@ -445,7 +445,7 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
                         mul[jj] = -sc * kLog2e;
                         add[jj] = -(b * sc) * kLog2e;
                     } else {
-                        mul[jj] = 1.f;
+                        mul[jj] = p.aff_scale ? __ldg(p.aff_scale + k) : 1.f;
                         add[jj] = b;
                     }
                 }
@@ -478,6 +478,10 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
                         } else {
 #pragma unroll
                             for (int jj = 0; jj < CW; ++jj) v[jj] = fmaf(v[jj], mul[jj], add[jj]);
+                            if (p.clamp) {
+#pragma unroll
+                                for (int jj = 0; jj < CW; ++jj) v[jj] = fminf(fmaxf(v[jj], p.lo), p.hi);
+                            }
                         }
                         if (rvalid && qvalid) {
                             float *yr = ybase + (long long)c0 * plane + (long long)(tl.p0 + i + h) * p.Q;

@@ -85,6 +85,24 @@ GCONV_API gconv_status_t gconv2d_fwd(const float *x, const float *w, const float
                            int stride, int pad, int dilation, int groups,
                            float *y, cudaStream_t stream);
 
+/* Convolution with a per-output-channel affine epilogue and a clamp:
+ *   y[n,k,p,q] = min(max(conv(x, w)[n,k,p,q] * scale[k] + shift[k], lo), hi)
+ * This is the depthwise convolution of a MobileNetV2 inverted-residual block
+ * ("GroupConv Atlas", "Fix the experiment": the block the page substitutes
+ * one convolution in) fused with the BatchNorm in inference form that
+ * follows it, folded into scale = gamma / sqrt(running_var + eps) and
+ * shift = beta - running_mean * scale (+ conv bias * scale), and the ReLU6
+ * (lo = 0, hi = 6).
+ * scale, shift: [K] device pointers, or NULL for 1 and 0.  lo <= hi (either
+ * may be infinite; -INFINITY, +INFINITY gives no clamp).  Shapes, layout,
+ * alignment, streams and errors as gconv2d_fwd; lo > hi or a NaN bound is
+ * GCONV_ERR_INVALID_ARG. */
+GCONV_API gconv_status_t gconv2d_affine_clamp_fwd(const float *x, const float *w,
+                           int N, int C, int H, int W, int K, int R, int S,
+                           int stride, int pad, int dilation, int groups,
+                           const float *scale, const float *shift, float lo, float hi,
+                           float *y, cudaStream_t stream);
+
 /* Fused chain ("Kimi-K2.6__l2_p21", Model forward):
  *   z = conv(x, w) + bias[k]          (bias [K] or NULL; the caller folds the
  *                                       conv bias and the extra [K,1,1] bias)

@@ -179,6 +179,23 @@ def chain(x, w, b_conv, b_extra, scale, gn_groups, gamma, beta, eps=1e-5,
     return dict(y=y, a=a, absacc=acc, mean=mean, var=var)
 
 
+def conv2d_affine_clamp(x, w, scale=None, shift=None, lo=-np.inf, hi=np.inf, stride=1, padding=0,
+                        dilation=1, groups=1, return_absacc=False):
+    """y = min(max(conv(x, w) * scale[k] + shift[k], lo), hi) in float64: the
+    depthwise convolution of the MobileNetV2 inverted-residual block with the
+    BatchNorm (inference form, folded into scale and shift) and the ReLU6
+    that follow it ("GroupConv Atlas", "Fix the experiment").  scale / shift
+    None mean 1 / 0.  The convolution is conv2d above; the affine step and the
+    clamp are written out here on its float64 result."""
+    y, acc = conv2d(x, w, None, stride, padding, dilation, groups, return_absacc=True)
+    K = y.shape[1]
+    s = np.ones(K) if scale is None else _f32(scale).reshape(-1).astype(np.float64)
+    t = np.zeros(K) if shift is None else _f32(shift).reshape(-1).astype(np.float64)
+    y = y * s[None, :, None, None] + t[None, :, None, None]
+    y = np.minimum(np.maximum(y, float(lo)), float(hi))
+    return (y, acc) if return_absacc else y
+
+
 def num_threads() -> int:
     """OpenMP threads the oracle runs with."""
     return int(_load().oracle_num_threads())

@@ -123,3 +123,10 @@ def test_binding_refuses_cpu_tensors(lib):
     w = torch.zeros(4, 1, 3, 3)
     with pytest.raises(ValueError):
         gc.conv2d(x, w, padding=1, groups=4)
+
+
+def test_affine_clamp_rejects_bad_bounds(lib):
+    geo = (1, 4, 8, 8, 4, 3, 3, 1, 1, 1, 4)
+    f = lib.gconv2d_affine_clamp_fwd
+    assert f(FAKE, FAKE, *geo, None, None, 1.0, 0.0, FAKE, None) == gc.ERR_INVALID_ARG
+    assert f(FAKE, FAKE, *geo, None, None, float("nan"), 1.0, FAKE, None) == gc.ERR_INVALID_ARG

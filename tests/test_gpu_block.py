@@ -68,3 +68,23 @@ def test_block_output_matches_float64_block(setup, oracle_mod):
     err = (y - y64).abs()
     # FP32 rounding through two BatchNorms, a ReLU6 and a 144-term 1x1 sum
     assert float((err / (1e-4 * (1.0 + y64.abs()))).max()) <= 1.0, float(err.max())
+
+
+def test_fused_block_matches_float64_block(setup, oracle_mod):
+    # depthwise conv + BatchNorm + ReLU6 in one call (conv2d_affine_clamp with the folded BatchNorm)
+    x, prm = setup
+    dev = block.to_device(prm, "cuda")
+    prev = torch.backends.cudnn.allow_tf32
+    torch.backends.cudnn.allow_tf32 = False
+    try:
+        y = block.forward_fused(x.cuda(), dev).cpu().double()
+    finally:
+        torch.backends.cudnn.allow_tf32 = prev
+    p64 = {k: ({kk: vv.double() for kk, vv in v.items()} if isinstance(v, dict) else v.double())
+           for k, v in prm.items()}
+    x64 = x.double()
+    d64 = torch.from_numpy(oracle_mod.conv2d(block.expand(x64, p64).numpy(), prm["wd"].double().numpy(),
+                                             None, 1, 1, 1, 144))
+    y64 = block.project(x64, d64, p64)
+    err = (y - y64).abs()
+    assert float((err / (1e-4 * (1.0 + y64.abs()))).max()) <= 1.0, float(err.max())

@@ -402,3 +402,43 @@ def test_chain_paths_agree_with_oracle(oracle_mod, mode):
         gc.force_kernel("auto")
     ref = _chain_ref(oracle_mod, d, 1, 0, 1, 1, 1e-5)
     assert_chain_close(y, ref, d["scale"].numpy(), d["gamma"].numpy(), 1e-5, 4, f"{mode} chain")
+
+
+# ------------------------------------------------------------ affine + clamp epilogue
+AFFINE_CASES = [
+    # (N, C, H, W, K, R, S, stride, pad, dil, groups, lo, hi)
+    (4, 144, 56, 56, 144, 3, 3, 1, 1, 1, 144, 0.0, 6.0),            # the depthwise workload + BN + ReLU6
+    (2, 32, 14, 14, 32, 3, 3, 1, 1, 1, 16, -0.5, 0.5),               # W=14: 8-byte cp.async staging
+    (2, 32, 36, 40, 64, 3, 3, 1, 1, 1, 1, 0.0, 6.0),                 # implicit GEMM
+    (2, 32, 36, 40, 64, 3, 3, 1, 1, 1, 1, -math.inf, math.inf),      # implicit GEMM, no clamp
+    (1, 24, 19, 23, 48, 3, 3, 2, 1, 1, 24, 0.0, 6.0),                # stride 2, channel multiplier 2
+]
+
+
+@pytest.mark.parametrize("case", AFFINE_CASES)
+def test_affine_clamp_matches_oracle(oracle_mod, case):
+    N, C, H, W, K, R, S, st, pad, dil, g, lo, hi = case
+    d = inputs.conv_inputs(N, C, H, W, K, R, S, g, seed=4000 + N * C + K)
+    rng = torch.Generator().manual_seed(4100 + K)
+    sc = torch.rand(K, generator=rng) + 0.5
+    sh = torch.randn(K, generator=rng) * 0.5
+    y = gc.conv2d_affine_clamp(d["x"].cuda(), d["w"].cuda(), sc.cuda(), sh.cuda(), lo, hi, st, pad, dil, g)
+    torch.cuda.synchronize()
+    ref, absacc = oracle_mod.conv2d_affine_clamp(d["x"].numpy(), d["w"].numpy(), sc.numpy(), sh.numpy(), lo, hi,
+                                                 st, pad, dil, g, return_absacc=True)
+    s64 = sc.double().numpy()[None, :, None, None]
+    t64 = sh.double().numpy()[None, :, None, None]
+    # conv bound scaled by |scale|, plus one FP32 rounding of acc*scale + shift; the clamp is 1-Lipschitz
+    tol = np.abs(s64) * (1e-5 * absacc + 1e-6) + 2.0 ** -23 * (np.abs(ref) + np.abs(t64)) + 1e-30
+    err = np.abs(y.cpu().double().numpy() - ref)
+    assert np.all(err <= tol), f"max err/tol {np.max(err / tol):.3g}"
+    assert float(y.min()) >= lo and float(y.max()) <= hi
+
+
+def test_affine_without_scale_shift_or_clamp_is_plain_conv():
+    d = inputs.conv_inputs(2, 144, 28, 28, 144, 3, 3, 144, seed=4200)
+    x, w = d["x"].cuda(), d["w"].cuda()
+    a = gc.conv2d_affine_clamp(x, w, None, None, -math.inf, math.inf, 1, 1, 1, 144)
+    b = gc.conv2d(x, w, None, 1, 1, 1, 144)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)

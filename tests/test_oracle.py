@@ -317,3 +317,58 @@ def test_chain_extreme_values_are_finite(oracle_mod):
     out = _chain(oracle_mod, d)
     assert np.all(np.isfinite(out["a"])) and np.all(np.isfinite(out["y"]))
     assert np.all((out["a"] >= 0) & (out["a"] <= 1))
+
+
+# ---------------------------------------------------------------- affine + clamp epilogue
+
+def test_affine_clamp_identity_is_conv(oracle_mod):
+    rng = np.random.default_rng(71)
+    x = rng.standard_normal((2, 6, 9, 11)).astype(np.float32)
+    w = rng.standard_normal((6, 3, 3, 3)).astype(np.float32)
+    a = oracle_mod.conv2d_affine_clamp(x, w, None, None, -np.inf, np.inf, 1, 1, 1, 2)
+    np.testing.assert_array_equal(a, oracle_mod.conv2d(x, w, None, 1, 1, 1, 2))
+
+
+def test_affine_clamp_relu6_closed_form(oracle_mod):
+    # all-ones depthwise 3x3, pad 1: conv = in-bounds tap count (4 corner, 6 edge, 9 inside);
+    # scale 1, shift -5, ReLU6 -> clip(count - 5, 0, 6) = 0, 1, 4
+    x = np.ones((1, 2, 5, 7), np.float32)
+    w = np.ones((2, 1, 3, 3), np.float32)
+    y = oracle_mod.conv2d_affine_clamp(x, w, np.ones(2, np.float32), np.full(2, -5.0, np.float32),
+                                       0.0, 6.0, 1, 1, 1, 2)
+    assert np.all(y[:, :, 0, 0] == 0.0) and np.all(y[:, :, 0, 3] == 1.0) and np.all(y[:, :, 2, 3] == 4.0)
+    # scale 2, shift 0: 2*count clipped at 6 -> 6 everywhere (counts >= 4)
+    y2 = oracle_mod.conv2d_affine_clamp(x, w, np.full(2, 2.0, np.float32), None, 0.0, 6.0, 1, 1, 1, 2)
+    assert np.all(y2 == 6.0)
+
+
+def test_affine_is_folded_batchnorm(oracle_mod):
+    # conv -> BatchNorm (inference) equals conv * scale + shift with the folded constants
+    rng = np.random.default_rng(72)
+    x = rng.standard_normal((2, 4, 8, 8)).astype(np.float32)
+    w = rng.standard_normal((4, 1, 3, 3)).astype(np.float32)
+    gamma, beta = rng.uniform(0.5, 1.5, 4), rng.normal(0, 0.1, 4)
+    mean, var, eps = rng.normal(0, 0.1, 4), rng.uniform(0.5, 1.5, 4), 1e-5
+    c = oracle_mod.conv2d(x, w, None, 1, 1, 1, 4)
+    bn = (c - mean[None, :, None, None]) / np.sqrt(var[None, :, None, None] + eps) * gamma[None, :, None, None] \
+        + beta[None, :, None, None]
+    sc = (gamma / np.sqrt(var + eps)).astype(np.float32)
+    sh = (beta - mean * (gamma / np.sqrt(var + eps))).astype(np.float32)
+    y = oracle_mod.conv2d_affine_clamp(x, w, sc, sh, -np.inf, np.inf, 1, 1, 1, 4)
+    # the folded constants are rounded to FP32 once (|rel| <= 2^-24)
+    assert np.max(np.abs(y - bn)) <= 1e-6 * (1 + np.max(np.abs(bn)))
+
+
+def test_affine_clamp_bounds_and_passthrough(oracle_mod):
+    rng = np.random.default_rng(73)
+    x = rng.standard_normal((1, 8, 10, 10)).astype(np.float32)
+    w = rng.standard_normal((8, 2, 3, 3)).astype(np.float32)
+    sc, sh = rng.standard_normal(8).astype(np.float32), rng.standard_normal(8).astype(np.float32)
+    free = oracle_mod.conv2d_affine_clamp(x, w, sc, sh, -np.inf, np.inf, 1, 1, 1, 4)
+    y = oracle_mod.conv2d_affine_clamp(x, w, sc, sh, -0.5, 0.75, 1, 1, 1, 4)
+    assert y.min() >= -0.5 and y.max() <= 0.75
+    inside = (free >= -0.5) & (free <= 0.75)
+    assert inside.any() and (~inside).any()
+    np.testing.assert_array_equal(y[inside], free[inside])
+    np.testing.assert_array_equal(y[free < -0.5], -0.5)
+    np.testing.assert_array_equal(y[free > 0.75], 0.75)
