@@ -104,13 +104,15 @@ struct Window {
     static constexpr int NCH = (WIN + 3) / 4;                     // chunks per row per thread
 };
 
-template <int G, int KT, int RPT, bool CHAIN, bool TMA>
+// EPI: 0 = plain (+bias), 1 = the chain's epilogue, 2 = affine + clamp
+template <int G, int KT, int RPT, int EPI, bool TMA>
 __global__ void __launch_bounds__(256, 2)
     direct_conv_kernel(const __grid_constant__ TensorMap tm, const DirectParams p) {
     extern __shared__ __align__(128) float smem[];
     using g = Geom<G>;
     using win = Window<G>;
     constexpr bool FAST = win::FAST;
+    constexpr bool CHAIN = EPI == 1;
     constexpr int IR = FAST ? (RPT - 1) * g::ST + (g::R - 1) * g::D + 1 : 1;
 
     const int tid = threadIdx.x;
@@ -189,8 +191,10 @@ __global__ void __launch_bounds__(256, 2)
             const int nw = cc * RS * p.KBtot;
             const int step = blockDim.x;
             const int dq = step / p.KBtot, dr = step - dq * p.KBtot;
-            int kl = tid % p.KBtot, rs = tid / p.KBtot, c = 0;
-            while (rs >= RS) { rs -= RS; ++c; }
+            // start position: one division per thread (only the stride is incremental)
+            int kl = tid % p.KBtot, rs = tid / p.KBtot;
+            int c = rs / RS;
+            rs -= c * RS;
             for (int e = tid; e < nw; e += step) {
                 dev::cp_async4(sw + e, p.w + ((long long)(kc0 + kl) * p.cpg + c0 + c) * RS + rs, true);
                 kl += dr;
@@ -210,8 +214,9 @@ __global__ void __launch_bounds__(256, 2)
             const int total = planes * p.IHt * cols;
             const int step = blockDim.x;
             const int dq = step / cols, dr = step - dq * cols;  // step = dq rows + dr columns
-            int col = tid % cols, row = tid / cols, pl = 0;
-            while (row >= p.IHt) { row -= p.IHt; ++pl; }
+            int col = tid % cols, row = tid / cols;
+            int pl = row / p.IHt;
+            row -= pl * p.IHt;
             int c = pl % cc, gbb = pl / cc;
             for (int e = tid; e < total; e += step) {
                 const int ci = (g0 + gbb) * p.cpg + c0 + c;
@@ -329,7 +334,7 @@ __global__ void __launch_bounds__(256, 2)
             const float b = p.bias ? __ldg(p.bias + kk) : 0.f;
             float sc = 1.f;
             if constexpr (CHAIN) sc = __ldg(p.scale + kk);
-            else if (p.aff_scale) sc = __ldg(p.aff_scale + kk);
+            else if (EPI == 2 && p.aff_scale) sc = __ldg(p.aff_scale + kk);
 #pragma unroll
             for (int rp = 0; rp < RPT; ++rp)
 #pragma unroll
@@ -338,10 +343,11 @@ __global__ void __launch_bounds__(256, 2)
                     if constexpr (CHAIN) {
                         z = acc[rp][v][k] + b;
                         z = __frcp_rn(1.f + __expf(-(z * sc)));
+                    } else if constexpr (EPI == 2) {
+                        // one rounding of acc * scale + shift, then the clamp
+                        z = fminf(fmaxf(fmaf(acc[rp][v][k], sc, b), p.lo), p.hi);
                     } else {
-                        // plain: acc + bias; affine epilogue: one rounding of acc * scale + shift
-                        z = p.aff_scale ? fmaf(acc[rp][v][k], sc, b) : acc[rp][v][k] + b;
-                        if (p.clamp) z = fminf(fmaxf(z, p.lo), p.hi);
+                        z = acc[rp][v][k] + b;
                     }
                     acc[rp][v][k] = z;
                 }
@@ -456,38 +462,38 @@ cudaError_t launch_pdl(Kern kern, dim3 grid, int threads, size_t smem, cudaStrea
     return cudaLaunchKernelEx(&cfg, kern, tm, p);
 }
 
-template <int G, int KT, bool CHAIN>
+template <int G, int KT, int EPI>
 cudaError_t launch_one(const DirectParams &p, const TensorMap &tm, dim3 grid, int threads, size_t smem,
                        cudaStream_t st) {
     constexpr int RPT = (KT >= 4) ? 2 : 4;
     if constexpr (Window<G>::FAST) {
-        if (p.tma) return launch_pdl(direct_conv_kernel<G, KT, RPT, CHAIN, true>, grid, threads, smem, st, tm, p);
+        if (p.tma) return launch_pdl(direct_conv_kernel<G, KT, RPT, EPI, true>, grid, threads, smem, st, tm, p);
     }
-    return launch_pdl(direct_conv_kernel<G, KT, RPT, CHAIN, false>, grid, threads, smem, st, tm, p);
+    return launch_pdl(direct_conv_kernel<G, KT, RPT, EPI, false>, grid, threads, smem, st, tm, p);
 }
 
-template <int G, bool CHAIN>
+template <int G, int EPI>
 cudaError_t launch_kt(const DirectParams &p, const TensorMap &tm, int KT, dim3 grid, int threads, size_t smem,
                       cudaStream_t st) {
     switch (KT) {
-        case 1: return launch_one<G, 1, CHAIN>(p, tm, grid, threads, smem, st);
-        case 2: return launch_one<G, 2, CHAIN>(p, tm, grid, threads, smem, st);
-        case 4: return launch_one<G, 4, CHAIN>(p, tm, grid, threads, smem, st);
-        case 8: return launch_one<G, 8, CHAIN>(p, tm, grid, threads, smem, st);
+        case 1: return launch_one<G, 1, EPI>(p, tm, grid, threads, smem, st);
+        case 2: return launch_one<G, 2, EPI>(p, tm, grid, threads, smem, st);
+        case 4: return launch_one<G, 4, EPI>(p, tm, grid, threads, smem, st);
+        case 8: return launch_one<G, 8, EPI>(p, tm, grid, threads, smem, st);
         default: return cudaErrorInvalidValue;
     }
 }
 
-template <bool CHAIN>
+template <int EPI>
 cudaError_t launch_geom(const DirectParams &p, const TensorMap &tm, int geom, int KT, dim3 grid, int threads,
                         size_t smem, cudaStream_t st) {
     switch (geom) {
-        case kGeom3x3s1p1: return launch_kt<kGeom3x3s1p1, CHAIN>(p, tm, KT, grid, threads, smem, st);
-        case kGeom3x3s1p0: return launch_kt<kGeom3x3s1p0, CHAIN>(p, tm, KT, grid, threads, smem, st);
-        case kGeom3x3s2p1: return launch_kt<kGeom3x3s2p1, CHAIN>(p, tm, KT, grid, threads, smem, st);
-        case kGeom5x9s1p0: return launch_kt<kGeom5x9s1p0, CHAIN>(p, tm, KT, grid, threads, smem, st);
-        case kGeom1x1s1p0: return launch_kt<kGeom1x1s1p0, CHAIN>(p, tm, KT, grid, threads, smem, st);
-        case kDirectGeneric: return launch_kt<kDirectGeneric, CHAIN>(p, tm, KT, grid, threads, smem, st);
+        case kGeom3x3s1p1: return launch_kt<kGeom3x3s1p1, EPI>(p, tm, KT, grid, threads, smem, st);
+        case kGeom3x3s1p0: return launch_kt<kGeom3x3s1p0, EPI>(p, tm, KT, grid, threads, smem, st);
+        case kGeom3x3s2p1: return launch_kt<kGeom3x3s2p1, EPI>(p, tm, KT, grid, threads, smem, st);
+        case kGeom5x9s1p0: return launch_kt<kGeom5x9s1p0, EPI>(p, tm, KT, grid, threads, smem, st);
+        case kGeom1x1s1p0: return launch_kt<kGeom1x1s1p0, EPI>(p, tm, KT, grid, threads, smem, st);
+        case kDirectGeneric: return launch_kt<kDirectGeneric, EPI>(p, tm, KT, grid, threads, smem, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -537,8 +543,9 @@ bool make_x_tensor_map(TensorMap *tm, const float *x, long long planes, int H, i
 
 cudaError_t launch_direct(const DirectParams &p, const TensorMap &tm, int geom, int KT, int chain, dim3 grid,
                           int threads, size_t smem, cudaStream_t stream) {
-    return chain ? launch_geom<true>(p, tm, geom, KT, grid, threads, smem, stream)
-                 : launch_geom<false>(p, tm, geom, KT, grid, threads, smem, stream);
+    if (chain) return launch_geom<1>(p, tm, geom, KT, grid, threads, smem, stream);
+    if (p.aff_scale || p.clamp) return launch_geom<2>(p, tm, geom, KT, grid, threads, smem, stream);
+    return launch_geom<0>(p, tm, geom, KT, grid, threads, smem, stream);
 }
 
 int read_and_clear_device_error() {
