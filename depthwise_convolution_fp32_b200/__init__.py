@@ -80,6 +80,8 @@ def library():
         lib.gconv_force_kernel.argtypes = [s]
         lib.gconv_device_error_status.restype = i
         lib.gconv_device_error_status.argtypes = []
+        lib.gconv_get_last_device_error.restype = i
+        lib.gconv_get_last_device_error.argtypes = [p]
         _lib = lib
         return lib
 

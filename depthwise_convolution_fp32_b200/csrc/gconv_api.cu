@@ -637,6 +637,11 @@ gconv_status_t gconv_device_error_status(void) {
     return (v || u) ? GCONV_ERR_TIMEOUT : GCONV_OK;
 }
 
+gconv_status_t gconv_get_last_device_error(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return GCONV_ERR_CUDA;
+    return gconv_device_error_status();
+}
+
 gconv_status_t gconv2d_output_size(int H, int W, int R, int S, int stride, int pad, int dilation, int *P,
                                    int *Q) {
     if (!P || !Q) return GCONV_ERR_INVALID_ARG;

@@ -190,6 +190,13 @@ GCONV_API gconv_status_t gconv_force_kernel(const char *name);
  * Reading clears the flag.  Synchronises with the current device. */
 GCONV_API gconv_status_t gconv_device_error_status(void);
 
+/* The same status after the work queued on `stream` so far has finished:
+ * synchronises `stream` (NULL: the legacy default stream) first, then reads
+ * and clears the flags as gconv_device_error_status.  GCONV_ERR_CUDA when
+ * the synchronisation itself reports an error (for example a launch that
+ * failed). */
+GCONV_API gconv_status_t gconv_get_last_device_error(cudaStream_t stream);
+
 /* Library version string. */
 GCONV_API const char *gconv_version(void);
 

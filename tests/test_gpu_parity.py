@@ -5,6 +5,7 @@ Small and medium shapes are compared in full; the full-size workloads are
 compared on sampled outputs the oracle computes one by one (and whole
 GroupNorm groups for the chain).  Output buffers are NaN-prefilled and
 surrounded by canary guards, so a missed store or a stray one fails."""
+import ctypes
 import math
 import zlib
 
@@ -442,3 +443,14 @@ def test_affine_without_scale_shift_or_clamp_is_plain_conv():
     b = gc.conv2d(x, w, None, 1, 1, 1, 144)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+def test_device_error_status_after_calls_on_a_stream():
+    # no bounded wait gives up on valid work: both status queries report OK
+    lib = gc.library()
+    d = inputs.conv_inputs(4, 144, 56, 56, 144, 3, 3, 144, seed=4300)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        gc.conv2d(d["x"].cuda(), d["w"].cuda(), None, 1, 1, 1, 144)
+    assert lib.gconv_get_last_device_error(ctypes.c_void_p(s.cuda_stream)) == gc.OK
+    assert lib.gconv_device_error_status() == gc.OK
