@@ -82,3 +82,52 @@ def test_planted_slip_is_caught(tmp_path, name, original, planted, expect):
         except (AssertionError, ValueError):
             caught.append(pin)
     assert caught, f"no pin noticed the planted slip '{name}'"
+
+
+# slips planted in the float64 affine + clamp step of the Python wrapper
+PY_MUTATIONS = [
+    ("shift added before the scale",
+     "y = y * s[None, :, None, None] + t[None, :, None, None]",
+     "y = (y + t[None, :, None, None]) * s[None, :, None, None]",
+     ["affine_bn"]),
+    ("clamp bounds swapped",
+     "y = np.minimum(np.maximum(y, float(lo)), float(hi))",
+     "y = np.maximum(np.minimum(y, float(lo)), float(hi))",
+     ["affine_relu6", "affine_bounds"]),
+    ("scale ignored",
+     "s = np.ones(K) if scale is None else _f32(scale).reshape(-1).astype(np.float64)",
+     "s = np.ones(K)",
+     ["affine_bn", "affine_relu6"]),
+]
+
+PINS.update({
+    "affine_bn": lambda m: pins.test_affine_is_folded_batchnorm(m),
+    "affine_relu6": lambda m: pins.test_affine_clamp_relu6_closed_form(m),
+    "affine_bounds": lambda m: pins.test_affine_clamp_bounds_and_passthrough(m),
+})
+
+
+def _mutated_oracle_py(tmp_path, original, planted):
+    src = open(os.path.join(ORACLE_DIR, "__init__.py")).read()
+    assert src.count(original) == 1, original
+    d = tmp_path / "oracle_mut_py"
+    d.mkdir()
+    shutil.copy(os.path.join(ORACLE_DIR, "oracle.c"), d / "oracle.c")
+    (d / "__init__.py").write_text(src.replace(original, planted))
+    spec = importlib.util.spec_from_file_location(f"oracle_mut_py_{abs(hash(planted))}", d / "__init__.py")
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build(force=True)
+    return mod
+
+
+@pytest.mark.parametrize("name,original,planted,expect", PY_MUTATIONS, ids=[m[0] for m in PY_MUTATIONS])
+def test_planted_affine_slip_is_caught(tmp_path, name, original, planted, expect):
+    mod = _mutated_oracle_py(tmp_path, original, planted)
+    caught = []
+    for pin in expect:
+        try:
+            PINS[pin](mod)
+        except (AssertionError, ValueError):
+            caught.append(pin)
+    assert caught, f"no pin noticed the planted slip '{name}'"
