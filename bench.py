@@ -474,6 +474,47 @@ def bootstrap_ci(samples, reps=2000, seed=0):
     return float(np.percentile(means, 2.5)), float(np.percentile(means, 97.5))
 
 
+def torch_conv_graph_us(r, per_batch, batches):
+    """PyTorch's own FP32 conv2d (cuDNN, autotuned, TF32 off) on the same
+    rotating inputs, timed the same way (a CUDA graph of per_batch calls):
+    the comparison the pages make against tuned PyTorch."""
+    import torch
+    import torch.nn.functional as F
+    s = r.wk.shape
+    prev = (torch.backends.cudnn.benchmark, torch.backends.cudnn.allow_tf32)
+    torch.backends.cudnn.benchmark, torch.backends.cudnn.allow_tf32 = True, False
+    try:
+        def call(i):
+            return F.conv2d(r.xs[i % r.n_sets], r.w, r.bias, s.stride, s.pad, s.dil, s.groups)
+        for i in range(3):
+            call(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        st = torch.cuda.Stream()
+        st.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(st):
+            with torch.cuda.graph(g, stream=st):
+                for i in range(per_batch):
+                    call(i)
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        us = []
+        for b in range(batches):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(st):
+                e0.record(st)
+                g.replay()
+                e1.record(st)
+            torch.cuda.synchronize()
+            us.append(e0.elapsed_time(e1) * 1e3 / per_batch)
+        del g
+        return statistics.mean(us)
+    finally:
+        torch.backends.cudnn.benchmark, torch.backends.cudnn.allow_tf32 = prev
+
+
 def write_records(args, gc, device, l2, hbm_peak, meas, batches=10, per_batch=30):
     """One record per shape: kernel chosen, status, graph-device and synchronized-API
     latency (mean over 10 batches of 30 calls, 95% bootstrap interval), GB/s,
@@ -534,6 +575,9 @@ def write_records(args, gc, device, l2, hbm_peak, meas, batches=10, per_batch=30
             "roofline": roofline_for(wk, gm * 1e-6, plan, hbm_peak, meas),
             "pool_sets": r.n_sets,
         })
+        if not wk.chain:
+            tg = torch_conv_graph_us(r, per_batch, batches)
+            rec.update({"torch_graph_us": round(tg, 3), "speedup_vs_torch": round(tg / gm, 3)})
         out.append(rec)
         del r
         torch.cuda.empty_cache()

@@ -96,7 +96,7 @@ int read_and_clear_device_error();
 int direct_rpt(int KT);   // rows per thread the variant with KT uses
 int direct_fast_window_chunks(int geom);   // 16-byte chunks one thread reads per row
 
-// ---- implicit GEMM on tcgen05 (3xTF32) -------------------------------------
+// ---- implicit GEMM on tcgen05 (tf32 main term + bf16 cross terms) ----------
 struct IgemmParams {
     const float4 *wh, *wl;     // split weights [g][cpg/8][r][s][2][kpg][4]
     const float *bias, *scale; // bias may be null; scale only for the chain
