@@ -4,6 +4,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload depthwise|tiny_grouped|fused_chain|dense_5x9]
                     [--no-shapes] [--sweep] [--force-kernel NAME]
+    python bench.py --profile --workload NAME [--batch B] [--calls C]   (ncu target)
 
 One step = one call of the library's entry point on one batch of the
 workload (default: the depthwise conv of a MobileNetV2 inverted-residual
@@ -609,6 +610,11 @@ def main():
                     help="skip the MobileNetV2 block timing (depthwise workload only)")
     ap.add_argument("--force-kernel", default="auto",
                     help="kernel family for A/B runs: auto, direct, direct_cpasync, generic, igemm")
+    ap.add_argument("--profile", action="store_true",
+                    help="profiler target: run --calls eager calls of --workload (at --batch), each "
+                         "followed by a synchronize, print one line and exit (no timing)")
+    ap.add_argument("--batch", type=int, default=0, help="--profile: override N (0: the workload's own)")
+    ap.add_argument("--calls", type=int, default=2, help="--profile: number of calls")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -644,6 +650,8 @@ def main():
 
     if args.records:
         return write_records(args, gc, device, l2, hbm_peak, meas)
+    if args.profile:
+        return run_profile_case(args, gc, device)
 
     wk = Workload(args.workload)
     runner = DeviceRunner(wk, device, l2)
@@ -725,6 +733,31 @@ def main():
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def run_profile_case(args, gc, device):
+    """A small, self-contained target for one ncu capture: `--calls` eager calls
+    of one workload on the same buffers (optionally at a reduced batch), each
+    followed by a synchronize.  Only the library's kernels run after the
+    one-time input upload."""
+    import dataclasses
+    import torch
+    wk = Workload(args.workload)
+    s = wk.shape
+    if args.batch > 0 and args.batch != s.N:
+        s = dataclasses.replace(s, N=args.batch)
+        wk.shape = s
+        wk.host = {k: (v[:args.batch] if k == "x" else v) for k, v in wk.host.items()}
+        if wk.host["x"].shape[0] < args.batch:
+            raise SystemExit(f"--batch {args.batch} exceeds the workload's N")
+    r = DeviceRunner(wk, device, 0)
+    y = None
+    for i in range(args.calls):
+        y = r.step(0)
+        torch.cuda.synchronize()
+    plan = gc.plan_name(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil, s.groups, wk.chain)
+    print(f"{args.workload} {s.label()} plan={plan} calls={args.calls} "
+          f"mean|y|={float(y.abs().mean()):.6f}", flush=True)
 
 
 def measure_block(device, steps, warmup):

@@ -82,6 +82,8 @@ def library():
         lib.gconv_device_error_status.argtypes = []
         lib.gconv_get_last_device_error.restype = i
         lib.gconv_get_last_device_error.argtypes = [p]
+        lib.gconv_selftest_wait_timeout.restype = i
+        lib.gconv_selftest_wait_timeout.argtypes = [ctypes.c_uint, p]
         _lib = lib
         return lib
 

@@ -38,6 +38,10 @@
 //    (griddepcontrol.wait) before their first global access.
 // A generic variant (all geometry at run time, inputs read straight from
 // global memory) serves every shape the specialised variants do not.
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -103,6 +107,99 @@ struct Window {
     static constexpr int WIN = FAST ? OFF + (kV - 1) * g::ST + (g::S - 1) * g::D + 1 : 4;
     static constexpr int NCH = (WIN + 3) / 4;                     // chunks per row per thread
 };
+
+// Accumulate one staged input plane into a thread's outputs: xs points at
+// the first 16-byte chunk of the thread's window (row ry*RPT*stride, chunk
+// column cx*stride), ws at the plane's weight slice [r][s][channel] offset to
+// the thread's first channel.  The window (IR rows x NCH chunks) is read with
+// 128-bit shared loads; every input value feeds up to R*S*KT FMAs and every
+// weight load (KT channels) feeds RPT*4 FMAs.
+template <int G, int KT, int RPT>
+__device__ __forceinline__ void fma_window(float (&acc)[RPT][kV][KT], const float *xs, const float *ws, int pitch,
+                                           int KBtot) {
+    using g = Geom<G>;
+    using win = Window<G>;
+    constexpr int IR = (RPT - 1) * g::ST + (g::R - 1) * g::D + 1;
+    float xr[IR][win::NCH * 4];
+#pragma unroll
+    for (int ir = 0; ir < IR; ++ir)
+#pragma unroll
+        for (int ch = 0; ch < win::NCH; ++ch) {
+            float4 v4 = *reinterpret_cast<const float4 *>(xs + ir * pitch + ch * 4);
+            xr[ir][4 * ch] = v4.x; xr[ir][4 * ch + 1] = v4.y;
+            xr[ir][4 * ch + 2] = v4.z; xr[ir][4 * ch + 3] = v4.w;
+        }
+#pragma unroll
+    for (int r = 0; r < g::R; ++r)
+#pragma unroll
+        for (int s = 0; s < g::S; ++s) {
+            float wv[KT];
+            load_weights<KT>(wv, ws + (r * g::S + s) * KBtot);
+#pragma unroll
+            for (int rp = 0; rp < RPT; ++rp)
+#pragma unroll
+                for (int v = 0; v < kV; ++v) {
+                    const float xv = xr[rp * g::ST + r * g::D][win::OFF + v * g::ST + s * g::D];
+#pragma unroll
+                    for (int k = 0; k < KT; ++k) acc[rp][v][k] = fmaf(wv[k], xv, acc[rp][v][k]);
+                }
+        }
+}
+
+// Epilogue in registers for the thread's KT channels starting at kfirst:
+// EPI 0: + bias; 1: the chain's logistic of (acc + bias) * scale; 2: the
+// affine + clamp, one rounding of acc * scale + shift.
+template <int KT, int RPT, int EPI>
+__device__ __forceinline__ void epilogue_transform(float (&acc)[RPT][kV][KT], const DirectParams &p, int kfirst) {
+#pragma unroll
+    for (int k = 0; k < KT; ++k) {
+        const int kk = kfirst + k;
+        const float b = p.bias ? __ldg(p.bias + kk) : 0.f;
+        float sc = 1.f;
+        if constexpr (EPI == 1) sc = __ldg(p.scale + kk);
+        else if (EPI == 2 && p.aff_scale) sc = __ldg(p.aff_scale + kk);
+#pragma unroll
+        for (int rp = 0; rp < RPT; ++rp)
+#pragma unroll
+            for (int v = 0; v < kV; ++v) {
+                float z;
+                if constexpr (EPI == 1) {
+                    z = acc[rp][v][k] + b;
+                    z = __frcp_rn(1.f + __expf(-(z * sc)));
+                } else if constexpr (EPI == 2) {
+                    z = fminf(fmaxf(fmaf(acc[rp][v][k], sc, b), p.lo), p.hi);
+                } else {
+                    z = acc[rp][v][k] + b;
+                }
+                acc[rp][v][k] = z;
+            }
+    }
+}
+
+// Store a thread's RPT rows x 4 columns x KT channels (rows from prow, columns
+// from qb, channels from kfirst) of image n; float4 when the rows allow it.
+template <int KT, int RPT>
+__device__ __forceinline__ void store_outputs(const float (&acc)[RPT][kV][KT], const DirectParams &p, int n,
+                                              int kfirst, int prow, int qb) {
+#pragma unroll
+    for (int rp = 0; rp < RPT; ++rp) {
+        const int pp = prow + rp;
+        if (pp >= p.P) continue;
+#pragma unroll
+        for (int k = 0; k < KT; ++k) {
+            const int kk = kfirst + k;
+            float *yr = p.y + (((long long)n * p.K + kk) * p.P + pp) * (long long)p.Q;
+            if (p.vec_out && qb + kV <= p.Q) {
+                *reinterpret_cast<float4 *>(yr + qb) =
+                    make_float4(acc[rp][0][k], acc[rp][1][k], acc[rp][2][k], acc[rp][3][k]);
+            } else {
+#pragma unroll
+                for (int v = 0; v < kV; ++v)
+                    if (qb + v < p.Q) yr[qb + v] = acc[rp][v][k];
+            }
+        }
+    }
+}
 
 // EPI: 0 = plain (+bias), 1 = the chain's epilogue, 2 = affine + clamp
 template <int G, int KT, int RPT, int EPI, bool TMA>
@@ -268,31 +365,7 @@ __global__ void __launch_bounds__(256, 2)
             for (int c = 0; c < cc; ++c) {
                 const float *xs = sx + (long long)(gb * cc + c) * p.pstride + (ry * RPT * g::ST) * p.pitch +
                                   cx * g::ST * 4;
-                const float *ws = sw + c * RS * p.KBtot + kl0;
-                float xr[IR][win::NCH * 4];
-#pragma unroll
-                for (int ir = 0; ir < IR; ++ir)
-#pragma unroll
-                    for (int ch = 0; ch < win::NCH; ++ch) {
-                        float4 v4 = *reinterpret_cast<const float4 *>(xs + ir * p.pitch + ch * 4);
-                        xr[ir][4 * ch] = v4.x; xr[ir][4 * ch + 1] = v4.y;
-                        xr[ir][4 * ch + 2] = v4.z; xr[ir][4 * ch + 3] = v4.w;
-                    }
-#pragma unroll
-                for (int r = 0; r < g::R; ++r)
-#pragma unroll
-                    for (int s = 0; s < g::S; ++s) {
-                        float wv[KT];
-                        load_weights<KT>(wv, ws + (r * g::S + s) * p.KBtot);
-#pragma unroll
-                        for (int rp = 0; rp < RPT; ++rp)
-#pragma unroll
-                            for (int v = 0; v < kV; ++v) {
-                                const float xv = xr[rp * g::ST + r * g::D][win::OFF + v * g::ST + s * g::D];
-#pragma unroll
-                                for (int k = 0; k < KT; ++k) acc[rp][v][k] = fmaf(wv[k], xv, acc[rp][v][k]);
-                            }
-                    }
+                fma_window<G, KT, RPT>(acc, xs, sw + c * RS * p.KBtot + kl0, p.pitch, p.KBtot);
             }
         } else {
             // generic geometry: read x straight from global memory (L1/L2 serve the reuse)
@@ -328,48 +401,8 @@ __global__ void __launch_bounds__(256, 2)
     // ---------------------------------------------------------------- epilogue
     const int qb = q0 + cx * kV;
     if (active && ok_wait) {
-#pragma unroll
-        for (int k = 0; k < KT; ++k) {
-            const int kk = kc0 + kl0 + k;
-            const float b = p.bias ? __ldg(p.bias + kk) : 0.f;
-            float sc = 1.f;
-            if constexpr (CHAIN) sc = __ldg(p.scale + kk);
-            else if (EPI == 2 && p.aff_scale) sc = __ldg(p.aff_scale + kk);
-#pragma unroll
-            for (int rp = 0; rp < RPT; ++rp)
-#pragma unroll
-                for (int v = 0; v < kV; ++v) {
-                    float z;
-                    if constexpr (CHAIN) {
-                        z = acc[rp][v][k] + b;
-                        z = __frcp_rn(1.f + __expf(-(z * sc)));
-                    } else if constexpr (EPI == 2) {
-                        // one rounding of acc * scale + shift, then the clamp
-                        z = fminf(fmaxf(fmaf(acc[rp][v][k], sc, b), p.lo), p.hi);
-                    } else {
-                        z = acc[rp][v][k] + b;
-                    }
-                    acc[rp][v][k] = z;
-                }
-        }
-#pragma unroll
-        for (int rp = 0; rp < RPT; ++rp) {
-            const int pp = p0 + ry * RPT + rp;
-            if (pp >= p.P) continue;
-#pragma unroll
-            for (int k = 0; k < KT; ++k) {
-                const int kk = kc0 + kl0 + k;
-                float *yr = p.y + (((long long)n * p.K + kk) * p.P + pp) * (long long)p.Q;
-                if (p.vec_out && qb + kV <= p.Q) {
-                    *reinterpret_cast<float4 *>(yr + qb) =
-                        make_float4(acc[rp][0][k], acc[rp][1][k], acc[rp][2][k], acc[rp][3][k]);
-                } else {
-#pragma unroll
-                    for (int v = 0; v < kV; ++v)
-                        if (qb + v < p.Q) yr[qb + v] = acc[rp][v][k];
-                }
-            }
-        }
+        epilogue_transform<KT, RPT, EPI>(acc, p, kc0 + kl0);
+        store_outputs<KT, RPT>(acc, p, n, kc0 + kl0, p0 + ry * RPT, qb);
     }
 
     if constexpr (CHAIN) {
@@ -441,12 +474,178 @@ __global__ void __launch_bounds__(256, 2)
     }
 }
 
-template <typename Kern>
-cudaError_t launch_pdl(Kern kern, dim3 grid, int threads, size_t smem, cudaStream_t st, const TensorMap &tm,
+// Streaming variant (plain and affine epilogues): persistent CTAs, each
+// walking the work items blockIdx.x, blockIdx.x + gridDim.x, ... through a
+// ring of `stages` shared-memory stages.  A work item is one tile of the
+// blocked kernel (TP rows x TQ columns x KBtot channels of one image).
+//  * The last warp produces: per item it waits until the item's stage is
+//    free, then lane 0 issues ONE 3-D TMA box holding every input plane, row
+//    and column the item needs (out-of-bounds elements arrive as zeros, so
+//    the padding costs nothing) and all 32 lanes copy the item's weight slice
+//    with 4-byte cp.async; both complete on the stage's `full` barrier.
+//  * The other warps wait on `full`, run the same register-blocked FMA loop
+//    as the blocked kernel, release the stage (one arrival per warp on
+//    `empty`) and then store their outputs from registers.
+// Up to `stages` items per CTA are in flight, so DRAM keeps streaming while
+// a CTA computes and stores (the blocked kernel leaves each CTA idle for a
+// full load latency per tile).  Every wait is bounded; a wait that gives up
+// raises the device error flag, stops the CTA's pipeline and, before the CTA
+// exits, waits (bounded again) for the copies it has in flight.
+template <int G, int KT, int RPT, int EPI>
+__global__ void __launch_bounds__(288, KT >= 8 ? 1 : 2)
+    direct_stream_kernel(const __grid_constant__ TensorMap tm, const DirectParams p) {
+    extern __shared__ __align__(128) float smem[];
+    using g = Geom<G>;
+    using win = Window<G>;
+    constexpr int RS = g::R * g::S;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);     // [8]
+    uint64_t *empty = full + 8;                               // [8]
+    int *flags = reinterpret_cast<int *>(full + 16);          // [0] abort, [1] items issued
+    float *stage0 = smem + kStreamHeaderBytes / 4;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int n_cwarps = (int)(blockDim.x >> 5) - 1;         // the last warp produces
+    const int S = p.stages;
+    const int GY = p.n_kb * (p.groups / p.GB);
+
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) {
+            dev::mbar_init(&full[s], 33);       // lane 0's expect_tx + 32 cp.async arrivals
+            dev::mbar_init(&empty[s], (uint32_t)n_cwarps);
+        }
+        flags[0] = 0;
+        flags[1] = 0;
+        dev::fence_mbar_init();
+    }
+    __syncthreads();
+    dev::griddep_wait();
+    dev::griddep_launch_dependents();
+
+    if (warp == n_cwarps) {
+        // ------------------------------------------------------------ producer
+        const uint32_t x_bytes = (uint32_t)(p.GB * p.cpg) * (uint32_t)p.IHt * (uint32_t)p.pitch * 4u;
+        const int nw = p.cpg * RS * p.KBtot;
+        int j = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; it < p.n_items; it += gridDim.x, ++j) {
+            const int s = j % S;
+            // every lane waits: its cp.async copies below overwrite the stage
+            if (j >= S && !dev::mbar_wait_bounded(&empty[s], (uint32_t)((j / S) - 1) & 1u)) ok = false;
+            if (*(volatile int *)&flags[0]) ok = false;
+            if (!__all_sync(0xffffffffu, ok)) {
+                ok = false;
+                break;
+            }
+            int t = it;
+            const int qt = t % p.n_qt; t /= p.n_qt;
+            const int pt = t % p.n_pt; t /= p.n_pt;
+            const int gy = t % GY;
+            const int n = t / GY;
+            const int g0 = (gy / p.n_kb) * p.GB;
+            const int kc0 = g0 * p.kpg + (gy % p.n_kb) * p.KB;
+            float *st = stage0 + (size_t)s * p.stage_floats;
+            if (lane == 0) {
+                dev::mbar_arrive_expect_tx(&full[s], x_bytes);
+                dev::tma_load_3d(st, &tm, &full[s], qt * p.TQ * g::ST - 4 * win::HL, pt * p.TP * g::ST - g::PAD,
+                                 n * p.C + g0 * p.cpg);
+            }
+            // weight slice transposed to [c][r][s][channel]: KT channels contiguous
+            float *sw = st + p.sw_off;
+            for (int e = lane; e < nw; e += 32) {
+                const int kl = e % p.KBtot;
+                const int crs = e / p.KBtot;   // c * RS + rs
+                const int c = crs / RS;
+                dev::cp_async4(sw + e, p.w + ((long long)(kc0 + kl) * p.cpg + c) * RS + (crs - c * RS), true);
+            }
+            dev::cp_async_mbar_arrive_noinc(&full[s]);
+        }
+        if (lane == 0) {
+            flags[1] = j;
+            if (!ok) {
+                atomicExch(&flags[0], 1);
+                atomicExch(&g_device_error, 1);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ compute
+        int t = tid;
+        const int cx = t % p.CXP; t /= p.CXP;
+        const int ry = t % p.RY; t /= p.RY;
+        const int kz = t % p.KZ;
+        const int gb = t / p.KZ;
+        const bool active = cx < p.CX && gb < p.GB;
+        const int kl0 = gb * p.KB + kz * KT;
+        const int pstride = p.IHt * p.pitch;
+        int j = 0;
+        for (int it = blockIdx.x; it < p.n_items; it += gridDim.x, ++j) {
+            const int s = j % S;
+            if (*(volatile int *)&flags[0]) break;
+            if (!dev::mbar_wait_bounded(&full[s], (uint32_t)(j / S) & 1u)) {
+                atomicExch(&flags[0], 1);
+                atomicExch(&g_device_error, 1);
+                break;
+            }
+            int u = it;
+            const int qt = u % p.n_qt; u /= p.n_qt;
+            const int pt = u % p.n_pt; u /= p.n_pt;
+            const int gy = u % GY;
+            const int n = u / GY;
+            const int kc0 = (gy / p.n_kb) * p.GB * p.kpg + (gy % p.n_kb) * p.KB;
+            const float *st = stage0 + (size_t)s * p.stage_floats;
+            float acc[RPT][kV][KT];
+#pragma unroll
+            for (int a = 0; a < RPT; ++a)
+#pragma unroll
+                for (int v = 0; v < kV; ++v)
+#pragma unroll
+                    for (int k = 0; k < KT; ++k) acc[a][v][k] = 0.f;
+            if (active) {
+                const float *sw = st + p.sw_off;
+                for (int c = 0; c < p.cpg; ++c) {
+                    const float *xs = st + (gb * p.cpg + c) * pstride + (ry * RPT * g::ST) * p.pitch + cx * g::ST * 4;
+                    fma_window<G, KT, RPT>(acc, xs, sw + c * RS * p.KBtot + kl0, p.pitch, p.KBtot);
+                }
+            }
+            // the stage is no longer read by this warp: hand it back before storing
+            __syncwarp();
+            if (lane == 0) dev::mbar_arrive(&empty[s]);
+            if (active) {
+                epilogue_transform<KT, RPT, EPI>(acc, p, kc0 + kl0);
+                store_outputs<KT, RPT>(acc, p, n, kc0 + kl0, pt * p.TP + ry * RPT, qt * p.TQ + cx * kV);
+            }
+        }
+    }
+    __syncthreads();
+    if (tid == 0 && flags[0]) {
+        // after an abort, wait (bounded) for the copies of issued items so no
+        // transfer into this CTA's shared memory is left in flight at exit
+        const int issued = flags[1];
+        for (int j = issued > S ? issued - S : 0; j < issued; ++j)
+            dev::mbar_wait_bounded(&full[j % S], (uint32_t)(j / S) & 1u);
+    }
+}
+
+// Raise a kernel's dynamic shared-memory limit to the opt-in maximum, once per
+// device (the attribute is per function and device; setting it on every
+// launch costs host time on the synchronous path).
+template <auto KERN>
+cudaError_t opt_in_smem() {
+    static std::atomic<unsigned long long> opted{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    const unsigned long long bit = dev < 64 ? 1ull << dev : 0;
+    if (bit && (opted.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e == cudaSuccess && bit) opted.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
+
+template <auto KERN>
+cudaError_t launch_pdl(dim3 grid, int threads, size_t smem, cudaStream_t st, const TensorMap &tm,
                        const DirectParams &p) {
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
+        cudaError_t e = opt_in_smem<KERN>();
         if (e != cudaSuccess) return e;
     }
     cudaLaunchConfig_t cfg = {};
@@ -459,7 +658,21 @@ cudaError_t launch_pdl(Kern kern, dim3 grid, int threads, size_t smem, cudaStrea
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, tm, p);
+    return cudaLaunchKernelEx(&cfg, KERN, tm, p);
+}
+
+template <auto KERN>
+int occupancy_of(int threads, size_t smem) {
+    if (smem > 48 * 1024 && opt_in_smem<KERN>() != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, KERN, threads, smem) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
 }
 
 template <int G, int KT, int EPI>
@@ -467,9 +680,9 @@ cudaError_t launch_one(const DirectParams &p, const TensorMap &tm, dim3 grid, in
                        cudaStream_t st) {
     constexpr int RPT = (KT >= 4) ? 2 : 4;
     if constexpr (Window<G>::FAST) {
-        if (p.tma) return launch_pdl(direct_conv_kernel<G, KT, RPT, EPI, true>, grid, threads, smem, st, tm, p);
+        if (p.tma) return launch_pdl<direct_conv_kernel<G, KT, RPT, EPI, true>>(grid, threads, smem, st, tm, p);
     }
-    return launch_pdl(direct_conv_kernel<G, KT, RPT, EPI, false>, grid, threads, smem, st, tm, p);
+    return launch_pdl<direct_conv_kernel<G, KT, RPT, EPI, false>>(grid, threads, smem, st, tm, p);
 }
 
 template <int G, int EPI>
@@ -494,6 +707,68 @@ cudaError_t launch_geom(const DirectParams &p, const TensorMap &tm, int geom, in
         case kGeom5x9s1p0: return launch_kt<kGeom5x9s1p0, EPI>(p, tm, KT, grid, threads, smem, st);
         case kGeom1x1s1p0: return launch_kt<kGeom1x1s1p0, EPI>(p, tm, KT, grid, threads, smem, st);
         case kDirectGeneric: return launch_kt<kDirectGeneric, EPI>(p, tm, KT, grid, threads, smem, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+// Streaming variants: (geometry, KT, epilogue) -> launch or occupancy query.
+// Resident CTAs per SM of one kernel at a block size and shared memory,
+// queried once per (device, block size, shared memory) and kept.
+template <auto KERN>
+int cached_occupancy(int threads, size_t smem) {
+    struct Entry {
+        int dev, threads;
+        size_t smem;
+        int occ;
+    };
+    static std::mutex mu;
+    static Entry cache[8] = {};
+    static int next = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry &e : cache)
+        if (e.occ > 0 && e.dev == dev && e.threads == threads && e.smem == smem) return e.occ;
+    const int occ = occupancy_of<KERN>(threads, smem);
+    if (occ > 0) {
+        cache[next] = Entry{dev, threads, smem, occ};
+        next = (next + 1) % 8;
+    }
+    return occ;
+}
+
+template <int G, int KT, int EPI>
+cudaError_t stream_one(const DirectParams &p, const TensorMap &tm, int sms, int threads, size_t smem,
+                       cudaStream_t st) {
+    constexpr int RPT = (KT >= 4) ? 2 : 4;
+    constexpr auto K = direct_stream_kernel<G, KT, RPT, EPI>;
+    const int occ = cached_occupancy<K>(threads, smem);
+    if (occ < 1 || p.stages < 1 || p.stages > 8) return cudaErrorInvalidConfiguration;
+    const long long ctas = std::min<long long>(p.n_items, (long long)sms * occ);
+    return launch_pdl<K>(dim3((unsigned)ctas), threads, smem, st, tm, p);
+}
+
+template <int G, int EPI>
+cudaError_t stream_kt(int KT, const DirectParams &p, const TensorMap &tm, int sms, int threads, size_t smem,
+                      cudaStream_t st) {
+    switch (KT) {
+        case 1: return stream_one<G, 1, EPI>(p, tm, sms, threads, smem, st);
+        case 2: return stream_one<G, 2, EPI>(p, tm, sms, threads, smem, st);
+        case 4: return stream_one<G, 4, EPI>(p, tm, sms, threads, smem, st);
+        case 8: return stream_one<G, 8, EPI>(p, tm, sms, threads, smem, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int EPI>
+cudaError_t stream_geom(int geom, int KT, const DirectParams &p, const TensorMap &tm, int sms, int threads,
+                        size_t smem, cudaStream_t st) {
+    switch (geom) {
+        case kGeom3x3s1p1: return stream_kt<kGeom3x3s1p1, EPI>(KT, p, tm, sms, threads, smem, st);
+        case kGeom3x3s1p0: return stream_kt<kGeom3x3s1p0, EPI>(KT, p, tm, sms, threads, smem, st);
+        case kGeom3x3s2p1: return stream_kt<kGeom3x3s2p1, EPI>(KT, p, tm, sms, threads, smem, st);
+        case kGeom5x9s1p0: return stream_kt<kGeom5x9s1p0, EPI>(KT, p, tm, sms, threads, smem, st);
+        case kGeom1x1s1p0: return stream_kt<kGeom1x1s1p0, EPI>(KT, p, tm, sms, threads, smem, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -527,13 +802,15 @@ int direct_fast_window_chunks(int geom) {
     }
 }
 
-bool make_x_tensor_map(TensorMap *tm, const float *x, long long planes, int H, int W, int box_w, int box_h) {
+bool make_x_tensor_map(TensorMap *tm, const float *x, long long planes, int H, int W, int box_w, int box_h,
+                       int box_planes) {
     static_assert(sizeof(TensorMap) == sizeof(CUtensorMap), "tensor map size");
     auto fn = encode_fn();
-    if (!fn) return false;
+    if (!fn || box_w < 1 || box_w > 256 || box_h < 1 || box_h > 256 || box_planes < 1 || box_planes > 256)
+        return false;
     cuuint64_t dims[3] = {(cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)planes};
     cuuint64_t strides[2] = {(cuuint64_t)W * 4, (cuuint64_t)W * H * 4};
-    cuuint32_t box[3] = {(cuuint32_t)box_w, (cuuint32_t)box_h, 1};
+    cuuint32_t box[3] = {(cuuint32_t)box_w, (cuuint32_t)box_h, (cuuint32_t)box_planes};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(reinterpret_cast<CUtensorMap *>(tm), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(x),
                     dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -546,6 +823,35 @@ cudaError_t launch_direct(const DirectParams &p, const TensorMap &tm, int geom, 
     if (chain) return launch_geom<1>(p, tm, geom, KT, grid, threads, smem, stream);
     if (p.aff_scale || p.clamp) return launch_geom<2>(p, tm, geom, KT, grid, threads, smem, stream);
     return launch_geom<0>(p, tm, geom, KT, grid, threads, smem, stream);
+}
+
+cudaError_t launch_direct_stream(const DirectParams &p, const TensorMap &tm, int geom, int KT, int sms,
+                                 int threads, size_t smem, cudaStream_t stream) {
+    if (p.aff_scale || p.clamp) return stream_geom<2>(geom, KT, p, tm, sms, threads, smem, stream);
+    return stream_geom<0>(geom, KT, p, tm, sms, threads, smem, stream);
+}
+
+namespace {
+
+// Self-test of the bounded-wait failure path: one warp waits on an mbarrier
+// that no thread ever arrives on, with the same bounded wait the kernels use
+// (at most `spins` polls).  The wait runs out, the kernel raises the device
+// error flag and returns; nothing else is touched.
+__global__ void wait_timeout_probe_kernel(unsigned spins) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        dev::mbar_init(&bar, 1);
+        dev::fence_mbar_init();
+    }
+    __syncthreads();
+    if (!dev::mbar_wait_bounded(&bar, 0, spins) && threadIdx.x == 0) atomicExch(&g_device_error, 1);
+}
+
+}  // namespace
+
+cudaError_t launch_wait_timeout_probe(unsigned spins, cudaStream_t stream) {
+    wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(spins);
+    return cudaGetLastError();
 }
 
 int read_and_clear_device_error() {

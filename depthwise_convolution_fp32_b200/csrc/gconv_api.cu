@@ -21,7 +21,10 @@ constexpr size_t kSmemBudget = 100 * 1024;   // keep two CTAs per SM where possi
 constexpr size_t kSmemMax = 227 * 1024;
 constexpr int kBarFloats = 32;               // shared memory reserved for mbarriers
 
-enum ForceMode : int { kForceAuto = 0, kForceDirect = 1, kForceGeneric = 2, kForceCpAsync = 3, kForceIgemm = 4 };
+enum ForceMode : int {
+    kForceAuto = 0, kForceDirect = 1, kForceGeneric = 2, kForceCpAsync = 3, kForceIgemm = 4,
+    kForceBlocked = 5, kForceStream = 6
+};
 std::atomic<int> g_force{kForceAuto};
 
 struct Shape {
@@ -73,6 +76,17 @@ const char *geom_name(int geom) {
     }
 }
 
+const char *geom_name_stream(int geom) {
+    switch (geom) {
+        case kGeom3x3s1p1: return "direct_stream_3x3s1p1";
+        case kGeom3x3s1p0: return "direct_stream_3x3s1p0";
+        case kGeom3x3s2p1: return "direct_stream_3x3s2p1";
+        case kGeom5x9s1p0: return "direct_stream_5x9s1p0";
+        case kGeom1x1s1p0: return "direct_stream_1x1s1p0";
+        default: return "direct_generic";
+    }
+}
+
 const char *geom_name_tma(int geom) {
     switch (geom) {
         case kGeom3x3s1p1: return "direct_tma_3x3s1p1";
@@ -92,13 +106,14 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 
-// A complete launch plan for the direct kernel.
+// A complete launch plan for the direct kernel (blocked or streaming).
 struct DirectPlan {
     DirectParams prm;
     int geom, KT;
-    dim3 grid;
+    dim3 grid;        // streaming: grid.x is set at launch from the occupancy
     int threads;
     size_t smem;
+    int stream = 0;   // 1: direct_stream_kernel
 };
 
 int sm_count() {
@@ -284,11 +299,118 @@ bool plan_direct(const Shape &s, bool chain, int gn_groups, int geom, bool x_vec
     return true;
 }
 
+// Plan for the streaming direct kernel (plain and affine epilogues, fast
+// geometries, rows TMA can describe, one pass over a group's input channels).
+// A work item is a blocked-kernel tile; its input (GB*cpg planes x IHt rows x
+// 4*tpc columns, one TMA box) and its weight slice form one ring stage.
+// Returns false when the shape does not fit this variant.
+bool plan_stream(const Shape &s, int geom, bool x_vec, DirectPlan &pl) {
+    if (geom == kDirectGeneric || !x_vec) return false;
+    DirectParams &p = pl.prm;
+    std::memset(&p, 0, sizeof(p));
+    // channels per thread: the blocked kernel's rule
+    int KT = 1;
+    const long long want = (long long)sm_count() * (kMaxThreads / 2);
+    for (int c : {8, 4, 2, 1}) {
+        if (s.kpg % c != 0) continue;
+        KT = c;
+        if ((long long)s.N * (s.K / c) * ceil_div(s.P, direct_rpt(c)) * ceil_div(s.Q, 4) >= want) break;
+    }
+    const int RPT = direct_rpt(KT);
+    const int nch = direct_fast_window_chunks(geom);
+    const int qchunks = ceil_div(s.Q, 4);
+    int n_qt = ceil_div(qchunks, 32), CX = 0, tpc = 0;
+    for (;; ++n_qt) {   // column tiles until the staged row fits one 256-element box row
+        CX = ceil_div(qchunks, n_qt);
+        tpc = ((CX - 1) * s.stride + nch + 7) / 8 * 8;
+        if (4 * tpc <= 256) break;
+    }
+    n_qt = ceil_div(qchunks, CX);
+    const int CXP = CX <= 4 ? CX : (CX + 7) / 8 * 8;
+    const int m = s.kpg / KT;
+    int KZ = 1;
+    for (int z = 1; z <= m; ++z)
+        if (m % z == 0 && KT * z <= 32 && CXP * z <= kMaxThreads) KZ = z;
+    const int strips = ceil_div(s.P, RPT);
+    int n_pt = 1;
+    auto pick_ry = [&](int cap) {
+        const int ry_max = std::max(1, std::min(cap, kMaxThreads / (CXP * KZ)));
+        n_pt = ceil_div(strips, ry_max);
+        return ceil_div(strips, n_pt);
+    };
+    int RY = pick_ry(strips);
+    auto pick_gb = [&](int cap) {
+        int gb = 1;
+        if (s.kpg / (KT * KZ) == 1)
+            for (int gc = 1; gc <= std::min(s.groups, cap); ++gc) {
+                if (s.groups % gc) continue;
+                if (CXP * RY * KZ * gc > kMaxThreads || gc * s.cpg > 256) break;
+                gb = gc;
+            }
+        return gb;
+    };
+    int GB = pick_gb(s.groups);
+    // enough items for about two CTAs per SM: fewer groups, rows, then slices per item
+    const long long target = 2LL * sm_count();
+    auto items = [&]() { return (long long)s.N * (m / KZ) * (s.groups / GB) * n_qt * n_pt; };
+    for (int guard = 0; guard < 64 && items() < target; ++guard) {
+        if (GB > 1) {
+            GB = pick_gb(GB - 1);
+        } else if (RY > 1) {
+            RY = pick_ry((RY + 1) / 2);
+        } else if (KZ > 1) {
+            int z = KZ - 1;
+            while (z > 1 && m % z != 0) --z;
+            KZ = z;
+            RY = pick_ry(strips);
+        } else {
+            break;
+        }
+    }
+    const int TP = RY * RPT;
+    const int KB = KT * KZ;
+    const int KBtot = GB * KB;
+    const int IHt = (TP - 1) * s.stride + (s.R - 1) * s.dil + 1;
+    const int planes = GB * s.cpg;
+    if (IHt > 256 || planes > 256 || items() > 0x7fffffffLL) return false;
+    const size_t x_floats = (size_t)planes * IHt * 4 * tpc;
+    const size_t w_floats = ((size_t)s.cpg * s.R * s.S * KBtot + 31) / 32 * 32;
+    const size_t stage_bytes = (x_floats + w_floats) * sizeof(float);
+    if (stage_bytes > 96 * 1024) return false;
+    const int S = stage_bytes <= 24 * 1024 ? 4 : (stage_bytes <= 36 * 1024 ? 3 : 2);
+
+    p.N = s.N; p.C = s.C; p.H = s.H; p.W = s.W; p.K = s.K; p.R = s.R; p.S = s.S;
+    p.stride = s.stride; p.pad = s.pad; p.dil = s.dil; p.groups = s.groups;
+    p.cpg = s.cpg; p.kpg = s.kpg; p.P = s.P; p.Q = s.Q;
+    p.CX = CX; p.CXP = CXP; p.RY = RY; p.KZ = KZ; p.GB = GB;
+    p.TP = TP; p.TQ = 4 * CX; p.KB = KB; p.KBtot = KBtot;
+    p.n_qt = n_qt; p.n_pt = n_pt; p.n_kb = m / KZ;
+    p.IHt = IHt; p.PC = tpc; p.pitch = 4 * tpc; p.cchunk = s.cpg;
+    p.pstride = IHt * 4 * tpc;
+    p.tma = 1;
+    p.n_items = (int)items();
+    p.stages = S;
+    p.stage_floats = (int)(x_floats + w_floats);
+    p.sw_off = (int)x_floats;
+    pl.geom = geom;
+    pl.KT = KT;
+    pl.threads = (CXP * RY * KZ * GB + 31) / 32 * 32 + 32;
+    pl.smem = kStreamHeaderBytes + (size_t)S * stage_bytes;
+    pl.grid = dim3(0);
+    pl.stream = 1;
+    return true;
+}
+
 // Direct-kernel plan for the current forcing mode.
 bool choose_direct(const Shape &s, bool chain, int gn_groups, bool x_vec, DirectPlan &pl) {
     const int force = g_force.load(std::memory_order_relaxed);
     int geom = (force == kForceGeneric) ? (int)kDirectGeneric : match_geom(s);
     if (force == kForceCpAsync) x_vec = false;
+    if (!chain && force != kForceBlocked && force != kForceGeneric && force != kForceCpAsync &&
+        plan_stream(s, geom, x_vec, pl))
+        return true;
+    if (force == kForceStream) return false;
+    pl.stream = 0;
     if (plan_direct(s, chain, gn_groups, geom, x_vec, pl)) return true;
     if (geom != kDirectGeneric && force == kForceAuto)
         return plan_direct(s, chain, gn_groups, kDirectGeneric, x_vec, pl);
@@ -332,11 +454,12 @@ bool cached_direct_plan(const Shape &s, bool x_vec, DirectPlan &pl) {
     return true;
 }
 
-bool cached_x_tensor_map(TensorMap *tm, const float *x, long long planes, int H, int W, int box_w, int box_h) {
+bool cached_x_tensor_map(TensorMap *tm, const float *x, long long planes, int H, int W, int box_w, int box_h,
+                         int box_planes = 1) {
     struct Entry {
         const float *x;
         long long planes;
-        int H, W, box_w, box_h, dev;
+        int H, W, box_w, box_h, box_planes, dev;
         TensorMap tm;
         bool valid;
     };
@@ -344,12 +467,12 @@ bool cached_x_tensor_map(TensorMap *tm, const float *x, long long planes, int H,
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
     if (last.valid && last.x == x && last.planes == planes && last.H == H && last.W == W && last.box_w == box_w &&
-        last.box_h == box_h && last.dev == dev) {
+        last.box_h == box_h && last.box_planes == box_planes && last.dev == dev) {
         *tm = last.tm;
         return true;
     }
-    if (!make_x_tensor_map(tm, x, planes, H, W, box_w, box_h)) return false;
-    last = Entry{x, planes, H, W, box_w, box_h, dev, *tm, true};
+    if (!make_x_tensor_map(tm, x, planes, H, W, box_w, box_h, box_planes)) return false;
+    last = Entry{x, planes, H, W, box_w, box_h, box_planes, dev, *tm, true};
     return true;
 }
 
@@ -362,6 +485,19 @@ bool finish_plan(const Shape &s, bool chain, int gn_groups, const float *x, floa
     p.vec2_in = !p.vec_in && (s.W % 2 == 0) && (reinterpret_cast<uintptr_t>(x) & 7u) == 0;
     p.vec_out = (s.Q % 4 == 0) && aligned16(y);
     std::memset(&tm, 0, sizeof(tm));
+    if (pl.stream) {
+        // one box per work item: 4*tpc columns x IHt rows x GB*cpg planes
+        if (cached_x_tensor_map(&tm, x, (long long)s.N * s.C, s.H, s.W, p.pitch, p.IHt, p.GB * s.cpg)) return true;
+        // a map the driver rejects: the blocked kernel with cp.async staging
+        DirectPlan again;
+        if (!plan_direct(s, chain, gn_groups, pl.geom, false, again)) return false;
+        again.stream = 0;
+        again.prm.vec_in = p.vec_in;
+        again.prm.vec2_in = p.vec2_in;
+        again.prm.vec_out = p.vec_out;
+        pl = again;
+        return true;
+    }
     if (p.tma && !cached_x_tensor_map(&tm, x, (long long)s.N * s.C, s.H, s.W, 4 * p.PC, p.bh)) {
         DirectPlan again;
         if (!plan_direct(s, chain, gn_groups, pl.geom, false, again)) return false;
@@ -517,7 +653,9 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
 // Whether the dispatcher sends a shape to the implicit GEMM.
 bool use_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     const int force = g_force.load(std::memory_order_relaxed);
-    if (force == kForceDirect || force == kForceGeneric || force == kForceCpAsync) return false;
+    if (force == kForceDirect || force == kForceGeneric || force == kForceCpAsync || force == kForceBlocked ||
+        force == kForceStream)
+        return false;
     if (!plan_igemm(s, chain, gn_groups, pl)) return false;
     if (force == kForceIgemm) return true;
     // auto: enough reduction depth and output channels for the tensor cores to win
@@ -526,20 +664,32 @@ bool use_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
 
 // Launch the split passes and the GEMM; chain additionally runs the GroupNorm
 // finalize and normalize passes.
+// Tensor maps over the split x operands in the workspace (x_hi, cross terms).
+bool igemm_maps(const Shape &s, const IgemmPlan &pl, void *ws, TensorMap *tm) {
+    char *base = reinterpret_cast<char *>(ws);
+    const IgemmParams &p = pl.prm;
+    const long long quads = (long long)s.N * (s.C / 4);
+    return make_nc4hw4_tile_map(&tm[0], reinterpret_cast<float *>(base), quads, p.Hp, p.Wp, p.COLS, p.AR) &&
+           make_nc4hw4_tile_map(&tm[1], reinterpret_cast<float *>(base + pl.off_xl), quads, p.Hp, p.Wp, p.COLS,
+                                p.AR);
+}
+
 gconv_status_t run_igemm(const Shape &s, IgemmPlan &pl, const float *x, const float *w, const float *bias,
                          const float *scale, int gn_groups, const float *gamma, const float *beta, float eps,
-                         float *y, void *ws, cudaStream_t stream) {
+                         float *y, void *ws, cudaStream_t stream, const TensorMap *maps = nullptr,
+                         bool split_w = true) {
     char *base = reinterpret_cast<char *>(ws);
     float *xh = reinterpret_cast<float *>(base);
     float *xl = reinterpret_cast<float *>(base + pl.off_xl);
     float *wh = reinterpret_cast<float *>(base + pl.off_wh);
     float *wl = reinterpret_cast<float *>(base + pl.off_wl);
     IgemmParams &p = pl.prm;
-    const long long quads = (long long)s.N * (s.C / 4);
-    TensorMap tm[2];
-    if (!make_nc4hw4_tile_map(&tm[0], xh, quads, p.Hp, p.Wp, p.COLS, p.AR) ||
-        !make_nc4hw4_tile_map(&tm[1], xl, quads, p.Hp, p.Wp, p.COLS, p.AR))
-        return GCONV_ERR_UNSUPPORTED;
+    TensorMap own[2];
+    const TensorMap *tm = maps;
+    if (!tm) {
+        if (!igemm_maps(s, pl, ws, own)) return GCONV_ERR_UNSUPPORTED;
+        tm = own;
+    }
     p.wh = reinterpret_cast<const float4 *>(wh);
     p.wl = reinterpret_cast<const float4 *>(wl);
     p.bias = bias;
@@ -549,7 +699,8 @@ gconv_status_t run_igemm(const Shape &s, IgemmPlan &pl, const float *x, const fl
     p.gn_part = chain ? reinterpret_cast<float4 *>(base + pl.off_part) : nullptr;
     if (launch_split_x(x, xh, xl, s.N, s.C, s.H, s.W, s.pad, p.Hp, p.Wp, stream) != cudaSuccess)
         return GCONV_ERR_CUDA;
-    if (launch_split_w(w, wh, wl, s.K, s.cpg, s.R, s.S, s.groups, stream) != cudaSuccess) return GCONV_ERR_CUDA;
+    if (split_w && launch_split_w(w, wh, wl, s.K, s.cpg, s.R, s.S, s.groups, stream) != cudaSuccess)
+        return GCONV_ERR_CUDA;
     if (launch_igemm(p, tm, chain ? 1 : 0, pl.grid, pl.smem, stream) != cudaSuccess) return GCONV_ERR_CUDA;
     if (!chain) return GCONV_OK;
     GnParams g;
@@ -565,6 +716,59 @@ gconv_status_t run_igemm(const Shape &s, IgemmPlan &pl, const float *x, const fl
     g.chunks = (int)std::max<long long>(1, (g.PQ + per_cta - 1) / per_cta);
     if (launch_gn_finalize(g, stream) != cudaSuccess) return GCONV_ERR_CUDA;
     if (launch_gn_normalize(g, stream) != cudaSuccess) return GCONV_ERR_CUDA;
+    return GCONV_OK;
+}
+
+// Images per chunk of the fused chain on the implicit-GEMM path: the chunk's
+// conv output and split operands take about half of the L2 cache, so the
+// normalize pass reads the conv output back from L2 and y goes out to HBM
+// once (plus the chunk's own split operands, which the next chunk overwrites
+// in place).  Returns N when the whole batch already fits.
+int chain_chunk_images(const Shape &s, const IgemmPlan &pl) {
+    static const int budget_mb = [] {
+        const int v = env_int("GCONV_CHAIN_L2_MB");
+        return v > 0 ? v : 56;
+    }();
+    const double per_img = 4.0 * s.K * s.P * s.Q + 8.0 * s.C * pl.prm.Hp * (double)pl.prm.Wp;
+    const long long B = (long long)(budget_mb * 1048576.0 / per_img);
+    return (int)std::max<long long>(1, std::min<long long>(B, s.N));
+}
+
+// The fused chain on the implicit-GEMM path, one chunk of images at a time
+// (split x -> GEMM with the fused epilogue -> statistics merge -> normalize);
+// the workspace holds one chunk.
+gconv_status_t run_chain_igemm(const Shape &s, const IgemmPlan &full, const float *x, const float *w,
+                               const float *bias, const float *scale, int gn_groups, const float *gamma,
+                               const float *beta, float eps, float *y, cudaStream_t stream) {
+    const int B = chain_chunk_images(s, full);
+    Shape sc = s;
+    sc.N = B;
+    IgemmPlan first;
+    if (B == s.N) first = full;
+    else if (!plan_igemm(sc, true, gn_groups, first)) return GCONV_ERR_UNSUPPORTED;
+    void *ws = nullptr;
+    gconv_status_t st = ensure_workspace(first.ws_bytes, stream, &ws);
+    if (st != GCONV_OK) return st;
+    TensorMap maps[2];
+    if (!igemm_maps(sc, first, ws, maps)) return GCONV_ERR_UNSUPPORTED;
+    const long long x_img = (long long)s.C * s.H * s.W, y_img = (long long)s.K * s.P * s.Q;
+    for (int n0 = 0; n0 < s.N; n0 += B) {
+        const int nb = std::min(B, s.N - n0);
+        if (nb == B) {
+            IgemmPlan cur = first;
+            st = run_igemm(sc, cur, x + n0 * x_img, w, bias, scale, gn_groups, gamma, beta, eps, y + n0 * y_img, ws,
+                           stream, maps, n0 == 0);
+        } else {
+            // a shorter last chunk: its own plan (workspace offsets and maps follow N)
+            Shape sl = s;
+            sl.N = nb;
+            IgemmPlan cur;
+            if (!plan_igemm(sl, true, gn_groups, cur)) return GCONV_ERR_UNSUPPORTED;
+            st = run_igemm(sl, cur, x + n0 * x_img, w, bias, scale, gn_groups, gamma, beta, eps, y + n0 * y_img, ws,
+                           stream);
+        }
+        if (st != GCONV_OK) return st;
+    }
     return GCONV_OK;
 }
 
@@ -607,9 +811,10 @@ gconv_status_t conv_fwd(const float *x, const float *w, const float *bias, const
     p.clamp = clamp;
     p.lo = lo;
     p.hi = hi;
-    if (launch_direct(p, tm, pl.geom, pl.KT, 0, pl.grid, pl.threads, pl.smem, stream) != cudaSuccess)
-        return GCONV_ERR_CUDA;
-    return GCONV_OK;
+    const cudaError_t e = pl.stream
+                              ? launch_direct_stream(p, tm, pl.geom, pl.KT, sm_count(), pl.threads, pl.smem, stream)
+                              : launch_direct(p, tm, pl.geom, pl.KT, 0, pl.grid, pl.threads, pl.smem, stream);
+    return e == cudaSuccess ? GCONV_OK : GCONV_ERR_CUDA;
 }
 
 }  // namespace
@@ -642,6 +847,11 @@ gconv_status_t gconv_get_last_device_error(cudaStream_t stream) {
     return gconv_device_error_status();
 }
 
+gconv_status_t gconv_selftest_wait_timeout(unsigned int spins, cudaStream_t stream) {
+    if (spins < 1 || spins > (1u << 24)) return GCONV_ERR_INVALID_ARG;
+    return launch_wait_timeout_probe(spins, stream) == cudaSuccess ? GCONV_OK : GCONV_ERR_CUDA;
+}
+
 gconv_status_t gconv2d_output_size(int H, int W, int R, int S, int stride, int pad, int dilation, int *P,
                                    int *Q) {
     if (!P || !Q) return GCONV_ERR_INVALID_ARG;
@@ -661,6 +871,8 @@ gconv_status_t gconv_force_kernel(const char *name) {
     else if (!std::strcmp(name, "generic")) g_force = kForceGeneric;
     else if (!std::strcmp(name, "direct_cpasync")) g_force = kForceCpAsync;
     else if (!std::strcmp(name, "igemm")) g_force = kForceIgemm;
+    else if (!std::strcmp(name, "direct_blocked")) g_force = kForceBlocked;
+    else if (!std::strcmp(name, "direct_stream")) g_force = kForceStream;
     else return GCONV_ERR_INVALID_ARG;
     return GCONV_OK;
 }
@@ -676,6 +888,7 @@ const char *gconv2d_plan_name(int N, int C, int H, int W, int K, int R, int S, i
     DirectPlan pl;
     int gn = 1;
     if (!choose_direct(s, chain != 0, gn, s.W % 4 == 0, pl)) return "unsupported";
+    if (pl.stream) return geom_name_stream(pl.geom);
     return pl.prm.tma ? geom_name_tma(pl.geom) : geom_name(pl.geom);
 }
 
@@ -700,7 +913,14 @@ size_t gconv2d_chain_workspace_size(int N, int C, int H, int W, int K, int R, in
     if (make_shape(s, N, C, H, W, K, R, S, stride, pad, dilation, groups) != GCONV_OK) return 0;
     if (gn_groups < 1 || K % gn_groups) return 0;
     IgemmPlan ig;
-    if (use_igemm(s, true, gn_groups, ig)) return ig.ws_bytes;
+    if (use_igemm(s, true, gn_groups, ig)) {
+        const int B = chain_chunk_images(s, ig);
+        if (B == s.N) return ig.ws_bytes;
+        Shape sc = s;
+        sc.N = B;
+        IgemmPlan first;
+        return plan_igemm(sc, true, gn_groups, first) ? first.ws_bytes : 0;
+    }
     DirectPlan pl;
     if (!choose_direct(s, true, gn_groups, s.W % 4 == 0, pl)) return 0;
     return chain_ws_bytes(pl.prm);
@@ -726,11 +946,8 @@ gconv_status_t gconv2d_bias_scale_sigmoid_groupnorm_fwd(const float *x, const fl
     for (const void *q : {(const void *)bias, (const void *)scale, (const void *)gamma, (const void *)beta})
         if (q && (reinterpret_cast<uintptr_t>(q) & 3u)) return GCONV_ERR_INVALID_ARG;
     IgemmPlan ig;
-    if (use_igemm(s, true, gn_groups, ig)) {
-        void *ws = nullptr;
-        if ((st = ensure_workspace(ig.ws_bytes, stream, &ws)) != GCONV_OK) return st;
-        return run_igemm(s, ig, x, w, bias, scale, gn_groups, gamma, beta, eps, y, ws, stream);
-    }
+    if (use_igemm(s, true, gn_groups, ig))
+        return run_chain_igemm(s, ig, x, w, bias, scale, gn_groups, gamma, beta, eps, y, stream);
     if (g_force.load(std::memory_order_relaxed) == kForceIgemm) return GCONV_ERR_UNSUPPORTED;
     DirectPlan pl;
     const bool x_vec = (s.W % 4 == 0) && aligned16(x);

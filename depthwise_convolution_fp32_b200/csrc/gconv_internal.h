@@ -54,6 +54,16 @@ struct DirectParams {
     int x_off;        // float offset of the x tile in shared memory
     int pstride;      // floats between staged planes
 
+    // streaming variant (persistent CTAs over a ring of stages; plain and
+    // affine epilogues): a work item is one CTA tile of the blocked kernel,
+    // staged by ONE 3-D TMA box of 4*PC columns x IHt rows x GB*cpg planes
+    int n_items;      // N * (groups/GB) * n_kb * n_pt * n_qt
+    int stages;       // ring depth
+    int stage_floats; // floats per stage: x planes, then the weight slice (multiple of 32)
+    int sw_off;       // float offset of the weight slice inside a stage
+    int CXP;          // threads per row strip: CX, rounded up to 8 when CX > 4 so that no
+                      // quarter-warp's 128-bit shared loads straddle two row strips
+
     // chain bookkeeping
     int gn_groups, kgn, slots, slots_k, n_sp;
 
@@ -83,16 +93,26 @@ struct alignas(64) TensorMap {
 // Encode a 3-D tensor map over x viewed as [N*C][H][W] with a box of
 // box_w x box_h x 1 elements (zero fill out of bounds).  Returns false when
 // the driver entry point is unavailable or rejects the map.
-bool make_x_tensor_map(TensorMap *tm, const float *x, long long planes, int H, int W, int box_w, int box_h);
+bool make_x_tensor_map(TensorMap *tm, const float *x, long long planes, int H, int W, int box_w, int box_h,
+                       int box_planes = 1);
 
 // Launch one direct-kernel variant (programmatic dependent launch enabled);
 // returns the launch status.
 cudaError_t launch_direct(const DirectParams &p, const TensorMap &tm, int geom, int KT, int chain,
                           dim3 grid, int threads, size_t smem, cudaStream_t stream);
 
+// Streaming direct kernel: threads = compute threads + one producer warp.
+// The grid is min(work items, sms x resident CTAs per SM), the occupancy
+// being queried once per variant, block size, shared memory and device.
+cudaError_t launch_direct_stream(const DirectParams &p, const TensorMap &tm, int geom, int KT, int sms,
+                                 int threads, size_t smem, cudaStream_t stream);
+constexpr int kStreamHeaderBytes = 256;   // barriers + bookkeeping ahead of the stages
+
 // Device error flag raised by bounded waits that gave up (0 = none); reading
 // clears it.  Synchronises with the device.
 int read_and_clear_device_error();
+// One CTA whose bounded mbarrier wait runs out after `spins` polls (raises the flag).
+cudaError_t launch_wait_timeout_probe(unsigned spins, cudaStream_t stream);
 int direct_rpt(int KT);   // rows per thread the variant with KT uses
 int direct_fast_window_chunks(int geom);   // 16-byte chunks one thread reads per row
 

@@ -59,7 +59,7 @@ typedef enum gconv_status {
     GCONV_ERR_UNSUPPORTED = 2,   /* valid shape that no kernel implements */
     GCONV_ERR_CUDA = 3,          /* the CUDA runtime reported an error */
     GCONV_ERR_WORKSPACE = 4,     /* workspace too small and cannot grow now */
-    GCONV_ERR_TIMEOUT = 5        /* reserved: a bounded device wait gave up */
+    GCONV_ERR_TIMEOUT = 5        /* a bounded device wait gave up (see gconv_get_last_device_error) */
 } gconv_status_t;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -196,6 +196,20 @@ GCONV_API gconv_status_t gconv_device_error_status(void);
  * the synchronisation itself reports an error (for example a launch that
  * failed). */
 GCONV_API gconv_status_t gconv_get_last_device_error(cudaStream_t stream);
+
+/* Self-test of the device-side failure path.  Every wait inside the kernels
+ * (on TMA and cp.async completion, on pipeline stages, on tensor-core
+ * commits) is bounded: a wait that runs out raises a device error flag,
+ * stops the kernel's pipeline and returns, instead of hanging the GPU.  This
+ * call launches one CTA (one warp) on `stream` that waits on an mbarrier no
+ * thread ever arrives on, with that same bounded wait limited to `spins`
+ * polls (1 .. 2^24); the wait runs out, the flag is raised and the kernel
+ * returns.  The next gconv_get_last_device_error(stream) then reports
+ * GCONV_ERR_TIMEOUT (and clears the flag) while the CUDA context stays
+ * usable.  The pages have no counterpart: this exists so the failure path
+ * can be tested without faulting a GPU.  Returns GCONV_ERR_INVALID_ARG for
+ * `spins` out of range, GCONV_ERR_CUDA when the launch fails. */
+GCONV_API gconv_status_t gconv_selftest_wait_timeout(unsigned int spins, cudaStream_t stream);
 
 /* Library version string. */
 GCONV_API const char *gconv_version(void);

@@ -101,8 +101,11 @@ def test_chain_rejects_invalid_arguments(lib):
 
 
 def test_plan_names(lib):
-    assert gc.plan_name(4, 144, 56, 56, 144, 3, 3, 1, 1, 1, 144) == "direct_tma_3x3s1p1"
-    assert gc.plan_name(2, 16, 14, 14, 16, 3, 3, 1, 1, 1, 16) == "direct_3x3s1p1"
+    assert gc.plan_name(4, 144, 56, 56, 144, 3, 3, 1, 1, 1, 144) == "direct_stream_3x3s1p1"
+    assert gc.plan_name(2, 16, 14, 14, 16, 3, 3, 1, 1, 1, 16) == "direct_3x3s1p1"   # rows not 16-byte multiples
+    assert gc.plan_name(1, 8, 29, 32, 8, 3, 3, 2, 1, 1, 8) == "direct_stream_3x3s2p1"
+    # the fused chain's conv stage never streams (its epilogue reduces statistics per CTA)
+    assert not gc.plan_name(2, 16, 30, 32, 16, 3, 3, 1, 1, 1, 16, chain=True).startswith("direct_stream")
     assert gc.plan_name(1, 8, 16, 16, 8, 3, 3, 1, 1, 2, 4) == "direct_generic"
     assert gc.plan_name(1, 8, 16, 16, 8, 3, 3, 1, 1, 1, 3) == "invalid"
     assert gc.chain_workspace_size(128, 8, 256, 256, 32, 3, 3, 1, 0, 1, 1, 8) > 0
@@ -110,8 +113,13 @@ def test_plan_names(lib):
 
 
 def test_force_kernel_names(lib):
-    for n in ("generic", "direct", "direct_cpasync", "auto"):
+    for n in ("generic", "direct", "direct_cpasync", "direct_blocked", "direct_stream", "igemm", "auto"):
         gc.force_kernel(n)
+    gc.force_kernel("direct_blocked")
+    try:
+        assert gc.plan_name(4, 144, 56, 56, 144, 3, 3, 1, 1, 1, 144) == "direct_tma_3x3s1p1"
+    finally:
+        gc.force_kernel("auto")
     with pytest.raises(gc.GconvError):
         gc.force_kernel("cudnn")
     gc.force_kernel("auto")
@@ -130,3 +138,9 @@ def test_affine_clamp_rejects_bad_bounds(lib):
     f = lib.gconv2d_affine_clamp_fwd
     assert f(FAKE, FAKE, *geo, None, None, 1.0, 0.0, FAKE, None) == gc.ERR_INVALID_ARG
     assert f(FAKE, FAKE, *geo, None, None, float("nan"), 1.0, FAKE, None) == gc.ERR_INVALID_ARG
+
+
+def test_selftest_wait_timeout_rejects_bad_limits(lib):
+    # validated on the host: nothing is launched
+    assert lib.gconv_selftest_wait_timeout(0, None) == gc.ERR_INVALID_ARG
+    assert lib.gconv_selftest_wait_timeout((1 << 24) + 1, None) == gc.ERR_INVALID_ARG

@@ -209,6 +209,80 @@ def test_forced_cpasync_staging_matches_oracle(oracle_mod, geo):
         gc.force_kernel("auto")
 
 
+# shapes the streaming kernel takes: every fast geometry, ragged tiles, several
+# work items per CTA (the stage ring wraps many times), grouped and multiplied
+# channels, the largest channel slices
+STREAM_GEOMS = [
+    # N, C, H, W, K, R, S, stride, pad, dil, groups, bias
+    (1, 32, 28, 28, 32, 3, 3, 1, 1, 1, 8, True),
+    (3, 12, 17, 24, 12, 3, 3, 1, 1, 1, 12, True),     # ragged rows
+    (2, 8, 33, 132, 8, 3, 3, 1, 1, 1, 8, False),     # two column tiles
+    (1, 16, 56, 56, 32, 3, 3, 1, 1, 1, 16, False),   # channel multiplier 2
+    (2, 24, 20, 20, 48, 3, 3, 1, 1, 1, 3, True),     # cpg 8, kpg 16
+    (2, 16, 56, 56, 16, 3, 3, 2, 1, 1, 16, True),    # stride 2
+    (1, 8, 32, 36, 8, 3, 3, 2, 1, 1, 8, False),
+    (1, 8, 20, 24, 16, 3, 3, 1, 0, 1, 1, True),      # pad 0 dense
+    (1, 16, 12, 40, 16, 1, 1, 1, 0, 1, 4, True),     # pointwise grouped
+    (1, 64, 12, 12, 64, 3, 3, 1, 1, 1, 1, False),    # dense 3x3, 64 channels per group
+    (32, 64, 56, 56, 64, 3, 3, 1, 1, 1, 64, True),   # 1024 work items: many per CTA
+    (8, 256, 28, 28, 256, 3, 3, 1, 1, 1, 128, False),
+    (2, 32, 112, 112, 32, 3, 3, 1, 1, 1, 8, True),   # 112-wide rows, cpg 4
+    (1, 8, 64, 1028, 8, 3, 3, 2, 1, 1, 8, False),    # wide rows: column tiles, stride 2
+]
+
+
+@pytest.mark.parametrize("geo", STREAM_GEOMS, ids=lambda g: "x".join(map(str, g[:11])))
+def test_forced_stream_matches_oracle(oracle_mod, geo):
+    N, C, H, W, K, R, S, st, pad, dil, g, bias = geo
+    d = inputs.conv_inputs(N, C, H, W, K, R, S, g, seed=13 + zlib.crc32(repr(geo).encode()) % 1000,
+                           x_dist="normal", bias=bias)
+    gc.force_kernel("direct_stream")
+    try:
+        assert gc.plan_name(N, C, H, W, K, R, S, st, pad, dil, g).startswith("direct_stream")
+        full_check(oracle_mod, d, st, pad, dil, g, "stream " + str(geo))
+    finally:
+        gc.force_kernel("auto")
+    assert gc.library().gconv_device_error_status() == gc.OK
+
+
+@pytest.mark.parametrize("geo", GEOMS[:10] + STREAM_GEOMS[10:], ids=lambda g: "x".join(map(str, g[:11])))
+def test_forced_blocked_matches_oracle(oracle_mod, geo):
+    """The blocked (one tile per CTA) direct kernel on shapes the dispatcher streams."""
+    N, C, H, W, K, R, S, st, pad, dil, g, bias = geo
+    d = inputs.conv_inputs(N, C, H, W, K, R, S, g, seed=17 + zlib.crc32(repr(geo).encode()) % 1000,
+                           x_dist="normal", bias=bias)
+    gc.force_kernel("direct_blocked")
+    try:
+        assert not gc.plan_name(N, C, H, W, K, R, S, st, pad, dil, g).startswith("direct_stream")
+        full_check(oracle_mod, d, st, pad, dil, g, "blocked " + str(geo))
+    finally:
+        gc.force_kernel("auto")
+
+
+def test_stream_affine_clamp_and_misaligned_output(oracle_mod):
+    """Streaming kernel with the affine + clamp epilogue, y not 16-byte aligned (scalar stores)."""
+    d = inputs.conv_inputs(4, 64, 56, 56, 64, 3, 3, 64, seed=4500)
+    rng = torch.Generator().manual_seed(4501)
+    sc = torch.rand(64, generator=rng) + 0.5
+    sh = torch.randn(64, generator=rng) * 0.5
+    out = Guarded((4, 64, 56, 56), misalign=1)
+    gc.force_kernel("direct_stream")
+    try:
+        gc.conv2d_affine_clamp(d["x"].cuda(), d["w"].cuda(), sc.cuda(), sh.cuda(), 0.0, 6.0, 1, 1, 1, 64,
+                               out=out.y)
+        torch.cuda.synchronize()
+    finally:
+        gc.force_kernel("auto")
+    out.check()
+    ref, absacc = oracle_mod.conv2d_affine_clamp(d["x"].numpy(), d["w"].numpy(), sc.numpy(), sh.numpy(), 0.0,
+                                                 6.0, 1, 1, 1, 64, return_absacc=True)
+    s64 = sc.double().numpy()[None, :, None, None]
+    t64 = sh.double().numpy()[None, :, None, None]
+    tol = np.abs(s64) * (1e-5 * absacc + 1e-6) + 2.0 ** -23 * (np.abs(ref) + np.abs(t64)) + 1e-30
+    err = np.abs(out.y.cpu().double().numpy() - ref)
+    assert np.all(err <= tol), f"max err/tol {np.max(err / tol):.3g}"
+
+
 def test_forced_cpasync_chain(oracle_mod):
     d = inputs.chain_inputs(2, 8, 40, 40, 32, 3, 3, 1, 8, seed=64, bias_scale_std=1.0, affine="random")
     gc.force_kernel("direct_cpasync")
