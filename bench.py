@@ -615,6 +615,10 @@ def main():
                          "followed by a synchronize, print one line and exit (no timing)")
     ap.add_argument("--batch", type=int, default=0, help="--profile: override N (0: the workload's own)")
     ap.add_argument("--calls", type=int, default=2, help="--profile: number of calls")
+    ap.add_argument("--profile-graph", action="store_true",
+                    help="profiler target: capture --steps calls of --workload (rotating buffers, as the "
+                         "timed region) in one CUDA graph and replay it once inside the NVTX range "
+                         "'gconv_graph' (ncu --nvtx --nvtx-include gconv_graph/ --graph-profiling graph)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -652,6 +656,8 @@ def main():
         return write_records(args, gc, device, l2, hbm_peak, meas)
     if args.profile:
         return run_profile_case(args, gc, device)
+    if args.profile_graph:
+        return run_profile_graph(args, gc, device, l2)
 
     wk = Workload(args.workload)
     runner = DeviceRunner(wk, device, l2)
@@ -758,6 +764,36 @@ def run_profile_case(args, gc, device):
     plan = gc.plan_name(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil, s.groups, wk.chain)
     print(f"{args.workload} {s.label()} plan={plan} calls={args.calls} "
           f"mean|y|={float(y.abs().mean()):.6f}", flush=True)
+
+
+def run_profile_graph(args, gc, device, l2):
+    """The timed region of the benchmark as one profiler workload: --steps calls
+    over the rotating buffer pool captured in one CUDA graph, uploaded by one
+    untimed replay, then replayed once inside the NVTX range 'gconv_graph'.
+    Only that replay falls inside the range."""
+    import torch
+    wk = Workload(args.workload)
+    r = DeviceRunner(wk, device, l2)
+    r.step(0)                      # one eager call: workspace and plans ready before capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        with torch.cuda.graph(g, stream=st):
+            for i in range(args.steps):
+                r.step(i)
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("gconv_graph")
+    with torch.cuda.stream(st):
+        g.replay()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
+    del g
+    print(f"{args.workload} graph of {args.steps} calls over {r.n_sets} buffer sets "
+          f"({r.pool_bytes / 2**20:.0f} MiB)", flush=True)
 
 
 def measure_block(device, steps, warmup):

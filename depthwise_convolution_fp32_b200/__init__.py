@@ -66,6 +66,10 @@ def library():
         lib.gconv2d_output_size.argtypes = [i] * 7 + [ctypes.POINTER(i), ctypes.POINTER(i)]
         lib.gconv2d_fwd.restype = i
         lib.gconv2d_fwd.argtypes = [p, p, p] + geo + [p, p]
+        lib.gconv2d_fwd_ex.restype = i
+        lib.gconv2d_fwd_ex.argtypes = [p, p, p] + [i] * 14 + [p, p]
+        lib.gconv2d_plan_name_ex.restype = s
+        lib.gconv2d_plan_name_ex.argtypes = [i] * 14
         lib.gconv2d_affine_clamp_fwd.restype = i
         lib.gconv2d_affine_clamp_fwd.argtypes = [p, p] + geo + [p, p, f, f, p, p]
         lib.gconv2d_bias_scale_sigmoid_groupnorm_fwd.restype = i
@@ -109,8 +113,12 @@ def output_size(H, W, R, S, stride=1, pad=0, dilation=1):
 
 
 def plan_name(N, C, H, W, K, R, S, stride=1, pad=0, dilation=1, groups=1, chain=False) -> str:
-    return library().gconv2d_plan_name(N, C, H, W, K, R, S, stride, pad, dilation, groups,
-                                       1 if chain else 0).decode()
+    (sh, sw), (ph, pw), (dh, dw) = _pair(stride, "stride"), _pair(pad, "pad"), _pair(dilation, "dilation")
+    if sh == sw and ph == pw and dh == dw:
+        return library().gconv2d_plan_name(N, C, H, W, K, R, S, sh, ph, dh, groups, 1 if chain else 0).decode()
+    if chain:
+        raise ValueError("the fused chain takes the same stride, padding and dilation on both axes")
+    return library().gconv2d_plan_name_ex(N, C, H, W, K, R, S, sh, sw, ph, pw, dh, dw, groups).decode()
 
 
 def force_kernel(name: str):
@@ -161,6 +169,15 @@ def _stream(t):
     return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
 
 
+def _pair(v, name):
+    """(h, w) of an int or a 2-tuple argument."""
+    if isinstance(v, (tuple, list)):
+        if len(v) != 2:
+            raise ValueError(f"{name} must be an int or an (h, w) pair")
+        return int(v[0]), int(v[1])
+    return int(v), int(v)
+
+
 def _scalar(v, name):
     if isinstance(v, (tuple, list)):
         if len(v) != 2 or v[0] != v[1]:
@@ -191,20 +208,28 @@ def _output(x, out, shape):
 
 
 def conv2d(x, w, bias=None, stride=1, padding=0, dilation=1, groups=1, out=None):
-    """y = conv2d(x, w) (+ bias) on the GPU; x[N,C,H,W], w[K,C/groups,R,S]."""
+    """y = conv2d(x, w) (+ bias) on the GPU; x[N,C,H,W], w[K,C/groups,R,S].
+    stride, padding and dilation are ints or (h, w) pairs."""
     N, C, H, W = x.shape
     K, cpg, R, S = w.shape
-    stride, padding, dilation = (_scalar(stride, "stride"), _scalar(padding, "padding"),
-                                 _scalar(dilation, "dilation"))
+    (sh, sw), (ph, pw), (dh, dw) = _pair(stride, "stride"), _pair(padding, "padding"), _pair(dilation, "dilation")
     if cpg * groups != C:
         raise ValueError("w.shape[1] * groups must equal C")
-    P, Q = _out_size(H, W, R, S, stride, padding, dilation)
+    if sh == sw and ph == pw and dh == dw:
+        P, Q = _out_size(H, W, R, S, sh, ph, dh)
+        out = _output(x, out, (N, K, P, Q))
+        st = library().gconv2d_fwd(_dev(x, "x"), _dev(w, "w"), _dev(bias, "bias", True),
+                                   N, C, H, W, K, R, S, sh, ph, dh, groups, _dev(out, "out"), _stream(x))
+        if st:
+            _check(st, "gconv2d_fwd")
+        return out
+    P = _out_size(H, H, R, R, sh, ph, dh)[0]
+    Q = _out_size(W, W, S, S, sw, pw, dw)[0]
     out = _output(x, out, (N, K, P, Q))
-    st = library().gconv2d_fwd(_dev(x, "x"), _dev(w, "w"), _dev(bias, "bias", True),
-                               N, C, H, W, K, R, S, stride, padding, dilation, groups,
-                               _dev(out, "out"), _stream(x))
+    st = library().gconv2d_fwd_ex(_dev(x, "x"), _dev(w, "w"), _dev(bias, "bias", True),
+                                  N, C, H, W, K, R, S, sh, sw, ph, pw, dh, dw, groups, _dev(out, "out"), _stream(x))
     if st:
-        _check(st, "gconv2d_fwd")
+        _check(st, "gconv2d_fwd_ex")
     return out
 
 

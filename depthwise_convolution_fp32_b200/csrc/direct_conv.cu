@@ -384,7 +384,7 @@ __global__ void __launch_bounds__(256, 2)
                             const int ih = pp * p.stride - p.pad + r * p.dil;
                             if (ih < 0 || ih >= p.H) continue;
                             for (int s = 0; s < Ss; ++s) {
-                                const int iw = qq * p.stride - p.pad + s * p.dil;
+                                const int iw = qq * p.sw - p.pw + s * p.dw;
                                 if (iw < 0 || iw >= p.W) continue;
                                 const float xv = __ldg(xp + (long long)ih * p.W + iw);
                                 const float *wr = ws + (r * Ss + s) * p.KBtot;
@@ -395,6 +395,16 @@ __global__ void __launch_bounds__(256, 2)
                     }
                 }
             }
+        }
+    }
+
+    if constexpr (TMA) {
+        // a band wait that gave up: wait (bounded) for every band's copies
+        // before shared memory is reused by the statistics or the CTA exits
+        if (__syncthreads_or(!ok_wait)) {
+            if (tid == 0)
+                for (int b = 0; b < p.nb; ++b) dev::mbar_wait_bounded(&bars[b], 0);
+            __syncthreads();
         }
     }
 

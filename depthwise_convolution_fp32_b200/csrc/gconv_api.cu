@@ -27,9 +27,13 @@ enum ForceMode : int {
 };
 std::atomic<int> g_force{kForceAuto};
 
+// Convolution geometry.  stride, pad and dil are the H-axis values; sw, pw
+// and dw the W-axis ones (equal to them for the symmetric entry points).
 struct Shape {
     int N, C, H, W, K, R, S, stride, pad, dil, groups;
     int cpg, kpg, P, Q;
+    int sw, pw, dw;
+    bool square() const { return stride == sw && pad == pw && dil == dw; }
 };
 
 long long out_extent(long long in, long long k, long long s, long long p, long long d) {
@@ -38,25 +42,30 @@ long long out_extent(long long in, long long k, long long s, long long p, long l
     return span / s + 1;
 }
 
-gconv_status_t make_shape(Shape &s, int N, int C, int H, int W, int K, int R, int S, int stride, int pad,
-                          int dil, int groups) {
+gconv_status_t make_shape_ex(Shape &s, int N, int C, int H, int W, int K, int R, int S, int sh, int sw, int ph,
+                             int pw, int dh, int dw, int groups) {
     if (N < 1 || C < 1 || H < 1 || W < 1 || K < 1 || R < 1 || S < 1) return GCONV_ERR_INVALID_ARG;
-    if (stride < 1 || pad < 0 || dil < 1 || groups < 1) return GCONV_ERR_INVALID_ARG;
+    if (sh < 1 || sw < 1 || ph < 0 || pw < 0 || dh < 1 || dw < 1 || groups < 1) return GCONV_ERR_INVALID_ARG;
     if (C % groups != 0 || K % groups != 0) return GCONV_ERR_INVALID_ARG;
-    long long P = out_extent(H, R, stride, pad, dil);
-    long long Q = out_extent(W, S, stride, pad, dil);
+    long long P = out_extent(H, R, sh, ph, dh);
+    long long Q = out_extent(W, S, sw, pw, dw);
     if (P < 1 || Q < 1 || P > 0x7fffffff || Q > 0x7fffffff) return GCONV_ERR_INVALID_ARG;
     // index arithmetic: per-plane offsets fit in int64 comfortably; keep the
     // element counts below 2^62 and the staged-tile arithmetic in int
     if ((long long)N * C * H * W >= (1LL << 62) || (long long)N * K * P * Q >= (1LL << 62))
         return GCONV_ERR_INVALID_ARG;
     if ((long long)H * W >= (1LL << 31) || P * Q >= (1LL << 31)) return GCONV_ERR_UNSUPPORTED;
-    s = {N, C, H, W, K, R, S, stride, pad, dil, groups, C / groups, K / groups, (int)P, (int)Q};
+    s = {N, C, H, W, K, R, S, sh, ph, dh, groups, C / groups, K / groups, (int)P, (int)Q, sw, pw, dw};
     return GCONV_OK;
 }
 
+gconv_status_t make_shape(Shape &s, int N, int C, int H, int W, int K, int R, int S, int stride, int pad,
+                          int dil, int groups) {
+    return make_shape_ex(s, N, C, H, W, K, R, S, stride, stride, pad, pad, dil, dil, groups);
+}
+
 int match_geom(const Shape &s) {
-    if (s.dil != 1) return kDirectGeneric;
+    if (s.dil != 1 || !s.square()) return kDirectGeneric;
     if (s.R == 3 && s.S == 3 && s.stride == 1 && s.pad == 1) return kGeom3x3s1p1;
     if (s.R == 3 && s.S == 3 && s.stride == 1 && s.pad == 0) return kGeom3x3s1p0;
     if (s.R == 3 && s.S == 3 && s.stride == 2 && s.pad == 1) return kGeom3x3s2p1;
@@ -271,6 +280,7 @@ bool plan_direct(const Shape &s, bool chain, int gn_groups, int geom, bool x_vec
 
     p.N = s.N; p.C = s.C; p.H = s.H; p.W = s.W; p.K = s.K; p.R = s.R; p.S = s.S;
     p.stride = s.stride; p.pad = s.pad; p.dil = s.dil; p.groups = s.groups;
+    p.sw = s.sw; p.pw = s.pw; p.dw = s.dw;
     p.cpg = s.cpg; p.kpg = s.kpg; p.P = s.P; p.Q = s.Q;
     p.CX = CX; p.RY = RY; p.KZ = KZ; p.GB = GB;
     p.TP = TP; p.TQ = 4 * CX; p.KB = KB; p.KBtot = KBtot;
@@ -381,6 +391,7 @@ bool plan_stream(const Shape &s, int geom, bool x_vec, DirectPlan &pl) {
 
     p.N = s.N; p.C = s.C; p.H = s.H; p.W = s.W; p.K = s.K; p.R = s.R; p.S = s.S;
     p.stride = s.stride; p.pad = s.pad; p.dil = s.dil; p.groups = s.groups;
+    p.sw = s.sw; p.pw = s.pw; p.dw = s.dw;
     p.cpg = s.cpg; p.kpg = s.kpg; p.P = s.P; p.Q = s.Q;
     p.CX = CX; p.CXP = CXP; p.RY = RY; p.KZ = KZ; p.GB = GB;
     p.TP = TP; p.TQ = 4 * CX; p.KB = KB; p.KBtot = KBtot;
@@ -422,7 +433,7 @@ bool choose_direct(const Shape &s, bool chain, int gn_groups, bool x_vec, Direct
 // last TMA descriptor by input pointer and box (encoding goes through the
 // driver).  Keys hold everything the cached value depends on.
 struct DirectKey {
-    int v[11];
+    int v[14];
     int x_vec, force, dev, sms;
     bool operator==(const DirectKey &o) const { return std::memcmp(this, &o, sizeof(*this)) == 0; }
 };
@@ -437,7 +448,7 @@ bool cached_direct_plan(const Shape &s, bool x_vec, DirectPlan &pl) {
     thread_local int next = 0;
     DirectKey k;
     std::memset(&k, 0, sizeof(k));
-    const int vals[11] = {s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil, s.groups};
+    const int vals[14] = {s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil, s.groups, s.sw, s.pw, s.dw};
     std::memcpy(k.v, vals, sizeof(vals));
     k.x_vec = x_vec ? 1 : 0;
     k.force = g_force.load(std::memory_order_relaxed);
@@ -510,9 +521,30 @@ bool finish_plan(const Shape &s, bool chain, int gn_groups, const float *x, floa
 }
 
 // ----------------------------------------------------------------- workspace
+// Device addresses cached per device are only valid in the context they were
+// obtained in: after cudaDeviceReset (or a primary-context reset) the device
+// gets a new context and the cached address is dropped and looked up again.
+void *current_context() {
+    using Fn = int (*)(void **);
+    static Fn fn = [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            return (Fn) nullptr;
+        }
+        return reinterpret_cast<Fn>(ptr);
+    }();
+    void *ctx = nullptr;
+    if (!fn || fn(&ctx) != 0) return nullptr;
+    return ctx;
+}
+
 struct Workspace {
     void *ptr = nullptr;
     size_t bytes = 0;
+    void *ctx = nullptr;
 };
 constexpr int kMaxDevices = 64;
 Workspace g_ws[kMaxDevices];
@@ -522,8 +554,10 @@ gconv_status_t ensure_workspace(size_t bytes, cudaStream_t stream, void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return GCONV_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return GCONV_ERR_UNSUPPORTED;
+    void *ctx = current_context();
     std::lock_guard<std::mutex> lock(g_ws_mutex);
     Workspace &ws = g_ws[dev];
+    if (ws.ptr && ws.ctx != ctx) ws = Workspace{};   // allocated in a context that no longer exists
     if (ws.bytes >= bytes && ws.ptr) {
         *out = ws.ptr;
         return GCONV_OK;
@@ -544,6 +578,7 @@ gconv_status_t ensure_workspace(size_t bytes, cudaStream_t stream, void **out) {
     }
     ws.ptr = p;
     ws.bytes = want;
+    ws.ctx = ctx;
     *out = p;
     return GCONV_OK;
 }
@@ -572,18 +607,18 @@ int env_int(const char *name) {
 // Stride-1 convolutions whose groups hold a multiple of 8 input channels and
 // 32/64/128/256 output channels run as an implicit GEMM on the tensor cores.
 bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
-    if (s.stride != 1 || s.cpg % 8 != 0 || !igemm_supported_nt(s.kpg)) return false;
+    if (s.stride != 1 || s.sw != 1 || s.cpg % 8 != 0 || !igemm_supported_nt(s.kpg)) return false;
     const int kgn = chain ? s.K / gn_groups : 1;
     // chain epilogue: groups nest inside a conv group, widths 1..16 or multiples of 16
     if (chain && (s.kpg > 64 || s.kpg % kgn != 0 || (kgn > 16 && kgn % 16 != 0))) return false;
     const int NT = s.kpg;
-    int COLS = 128 + (s.S - 1) * s.dil;
+    int COLS = 128 + (s.S - 1) * s.dw;
     COLS = (COLS + 15) / 16 * 16;   // whole 16-pixel groups of the tile box
     if (COLS > 256) return false;
     // padded split operands: every tile box starts at a 16-pixel group and a
     // non-negative row, the zero border supplies the padding
     const long long Hp = (long long)s.H + s.pad;
-    const long long Wp = ((long long)s.W + s.pad + 15) / 16 * 16;
+    const long long Wp = ((long long)s.W + s.pw + 15) / 16 * 16;
     if (Hp > 0x7fffffffLL || Wp / 16 > 0x7fffffffLL) return false;
     static const int force_th = env_int("GCONV_IGEMM_TH");
     static const int force_sa = env_int("GCONV_IGEMM_SA");
@@ -615,6 +650,7 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     std::memset(&p, 0, sizeof(p));
     p.N = s.N; p.C = s.C; p.H = s.H; p.W = s.W; p.K = s.K; p.R = s.R; p.S = s.S;
     p.pad = s.pad; p.dil = s.dil; p.groups = s.groups; p.cpg = s.cpg; p.kpg = s.kpg; p.P = s.P; p.Q = s.Q;
+    p.pad_w = s.pw; p.dil_w = s.dw;
     p.CC8 = s.cpg / 8;
     p.TH = TH;
     p.COLS = COLS;
@@ -697,7 +733,7 @@ gconv_status_t run_igemm(const Shape &s, IgemmPlan &pl, const float *x, const fl
     p.y = y;
     const bool chain = gn_groups > 0;
     p.gn_part = chain ? reinterpret_cast<float4 *>(base + pl.off_part) : nullptr;
-    if (launch_split_x(x, xh, xl, s.N, s.C, s.H, s.W, s.pad, p.Hp, p.Wp, stream) != cudaSuccess)
+    if (launch_split_x(x, xh, xl, s.N, s.C, s.H, s.W, s.pad, s.pw, p.Hp, p.Wp, stream) != cudaSuccess)
         return GCONV_ERR_CUDA;
     if (split_w && launch_split_w(w, wh, wl, s.K, s.cpg, s.R, s.S, s.groups, stream) != cudaSuccess)
         return GCONV_ERR_CUDA;
@@ -780,12 +816,9 @@ gconv_status_t validate_ptrs(const float *x, const float *w, const float *y) {
 }
 
 // Plain convolution, optionally with the affine + clamp epilogue.
-gconv_status_t conv_fwd(const float *x, const float *w, const float *bias, const float *aff_scale, int clamp,
-                        float lo, float hi, int N, int C, int H, int W, int K, int R, int S, int stride, int pad,
-                        int dilation, int groups, float *y, cudaStream_t stream) {
-    Shape s;
-    gconv_status_t st = make_shape(s, N, C, H, W, K, R, S, stride, pad, dilation, groups);
-    if (st != GCONV_OK) return st;
+gconv_status_t conv_fwd_shape(const Shape &s, const float *x, const float *w, const float *bias,
+                              const float *aff_scale, int clamp, float lo, float hi, float *y, cudaStream_t stream) {
+    gconv_status_t st;
     if ((st = validate_ptrs(x, w, y)) != GCONV_OK) return st;
     if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) return GCONV_ERR_INVALID_ARG;
     if (aff_scale && (reinterpret_cast<uintptr_t>(aff_scale) & 3u)) return GCONV_ERR_INVALID_ARG;
@@ -815,6 +848,15 @@ gconv_status_t conv_fwd(const float *x, const float *w, const float *bias, const
                               ? launch_direct_stream(p, tm, pl.geom, pl.KT, sm_count(), pl.threads, pl.smem, stream)
                               : launch_direct(p, tm, pl.geom, pl.KT, 0, pl.grid, pl.threads, pl.smem, stream);
     return e == cudaSuccess ? GCONV_OK : GCONV_ERR_CUDA;
+}
+
+gconv_status_t conv_fwd(const float *x, const float *w, const float *bias, const float *aff_scale, int clamp,
+                        float lo, float hi, int N, int C, int H, int W, int K, int R, int S, int stride, int pad,
+                        int dilation, int groups, float *y, cudaStream_t stream) {
+    Shape s;
+    gconv_status_t st = make_shape(s, N, C, H, W, K, R, S, stride, pad, dilation, groups);
+    if (st != GCONV_OK) return st;
+    return conv_fwd_shape(s, x, w, bias, aff_scale, clamp, lo, hi, y, stream);
 }
 
 }  // namespace
@@ -896,6 +938,31 @@ gconv_status_t gconv2d_fwd(const float *x, const float *w, const float *bias, in
                            int R, int S, int stride, int pad, int dilation, int groups, float *y,
                            cudaStream_t stream) {
     return conv_fwd(x, w, bias, nullptr, 0, 0.f, 0.f, N, C, H, W, K, R, S, stride, pad, dilation, groups, y, stream);
+}
+
+gconv_status_t gconv2d_fwd_ex(const float *x, const float *w, const float *bias, int N, int C, int H, int W, int K,
+                              int R, int S, int stride_h, int stride_w, int pad_h, int pad_w, int dil_h, int dil_w,
+                              int groups, float *y, cudaStream_t stream) {
+    Shape s;
+    gconv_status_t st =
+        make_shape_ex(s, N, C, H, W, K, R, S, stride_h, stride_w, pad_h, pad_w, dil_h, dil_w, groups);
+    if (st != GCONV_OK) return st;
+    return conv_fwd_shape(s, x, w, bias, nullptr, 0, 0.f, 0.f, y, stream);
+}
+
+const char *gconv2d_plan_name_ex(int N, int C, int H, int W, int K, int R, int S, int stride_h, int stride_w,
+                                 int pad_h, int pad_w, int dil_h, int dil_w, int groups) {
+    Shape s;
+    gconv_status_t st =
+        make_shape_ex(s, N, C, H, W, K, R, S, stride_h, stride_w, pad_h, pad_w, dil_h, dil_w, groups);
+    if (st == GCONV_ERR_INVALID_ARG) return "invalid";
+    if (st != GCONV_OK) return "unsupported";
+    IgemmPlan ig;
+    if (use_igemm(s, false, 1, ig)) return "igemm_tf32_bf16x";
+    DirectPlan pl;
+    if (!choose_direct(s, false, 1, s.W % 4 == 0, pl)) return "unsupported";
+    if (pl.stream) return geom_name_stream(pl.geom);
+    return pl.prm.tma ? geom_name_tma(pl.geom) : geom_name(pl.geom);
 }
 
 gconv_status_t gconv2d_affine_clamp_fwd(const float *x, const float *w, int N, int C, int H, int W, int K, int R,
@@ -997,22 +1064,26 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 namespace {
 
 void *g_noalloc_ptr[kMaxDevices];
+void *g_noalloc_ctx[kMaxDevices];
 std::mutex g_noalloc_mutex;
 
 // Device address of the scratch array on the current device; the first call
-// per device performs the lookup.
+// per device (and the first after the device's context was reset) performs
+// the lookup.
 gconv_status_t noalloc_scratch(void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return GCONV_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return GCONV_ERR_UNSUPPORTED;
+    void *ctx = current_context();
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
+    if (!g_noalloc_ptr[dev] || g_noalloc_ctx[dev] != ctx) {
         void *ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
             cudaGetLastError();
             return GCONV_ERR_CUDA;
         }
         g_noalloc_ptr[dev] = ptr;
+        g_noalloc_ctx[dev] = ctx;
     }
     *out = g_noalloc_ptr[dev];
     return GCONV_OK;

@@ -27,8 +27,9 @@ struct DirectParams {
     const float *scale;         // chain only: [K]
     float4 *gn_part;            // chain only: [N*gn_groups][slots] (count, mean, M2, 0)
 
-    int N, C, H, W, K, R, S, stride, pad, dil, groups;
+    int N, C, H, W, K, R, S, stride, pad, dil, groups;   // stride, pad, dil: H axis
     int cpg, kpg, P, Q;
+    int sw, pw, dw;   // W-axis stride, padding, dilation (the specialised variants need them equal to H's)
 
     // CTA tile: CX chunk-columns of 4 outputs, RY row strips of RPT rows,
     // KZ channel slices of KT channels, GB conv groups.
@@ -122,7 +123,8 @@ struct IgemmParams {
     const float *bias, *scale; // bias may be null; scale only for the chain
     float *y;
     float4 *gn_part;           // chain only
-    int N, C, H, W, K, R, S, pad, dil, groups, cpg, kpg, P, Q;
+    int N, C, H, W, K, R, S, pad, dil, groups, cpg, kpg, P, Q;   // pad, dil: H axis
+    int pad_w, dil_w;          // W axis
     int CC8;                   // cpg / 8 (K-steps of 8 channels)
     int TH;                    // output rows per tile (one 128-pixel M tile each)
     int AR;                    // staged x rows per channel step: TH + (R-1)*dil
@@ -153,8 +155,8 @@ int igemm_threads(int nt);
 // step: 2 quads x box_rows rows x box_cols (multiple of 16) pixels.
 bool make_nc4hw4_tile_map(TensorMap *tm, const float *base, long long quads, int Hp, int Wp, int box_cols,
                           int box_rows);
-cudaError_t launch_split_x(const float *x, float *xh, float *xl, int N, int C, int H, int W, int pad, int Hp,
-                           int Wp, cudaStream_t st);
+cudaError_t launch_split_x(const float *x, float *xh, float *xl, int N, int C, int H, int W, int pad_h, int pad_w,
+                           int Hp, int Wp, cudaStream_t st);
 cudaError_t launch_split_w(const float *w, float *wh, float *wl, int K, int cpg, int R, int S, int groups,
                            cudaStream_t st);
 // tm: x_hi tile map, cross-term tile map

@@ -68,14 +68,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo_half, float hi_half) {
 }
 
 // x[N][C][H][W] -> per 8 input channels (octet c8) and padded pixel (hp, wp)
-// of a [Hp][Wp] plane holding x[h][w] at (h + pad, w + pad) and zeros
+// of a [Hp][Wp] plane holding x[h][w] at (h + pad_h, w + pad_w) and zeros
 // elsewhere:
 //   xh: tf32 parts in NC4HW4 cells, [n][2*c8 + q][hp][wp][4]  (q = channel quad)
 //   xc: bf16 parts, [n][c8][2][hp][wp][8]: chunk 0 = bf16(x_hi), chunk 1 = bf16(x - x_hi)
 // Both tensors have the same geometry when read as 32-bit words.
 __global__ void __launch_bounds__(256) split_x_kernel(const float *__restrict__ x, float4 *__restrict__ xh,
-                                                      uint4 *__restrict__ xc, int C8, int H, int W, int pad,
-                                                      int Hp, int Wp, long long cells) {
+                                                      uint4 *__restrict__ xc, int C8, int H, int W, int pad_h,
+                                                      int pad_w, int Hp, int Wp, long long cells) {
     dev::griddep_wait();
     dev::griddep_launch_dependents();
     const long long HW = (long long)H * W, HWp = (long long)Hp * Wp;
@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(256) split_x_kernel(const float *__restrict__ 
          i += (long long)gridDim.x * blockDim.x) {
         const long long pix = i % HWp;         // hp*Wp + wp
         const long long nc8 = i / HWp;         // n*C8 + c8
-        const int h = (int)(pix / Wp) - pad, w = (int)(pix % Wp) - pad;
+        const int h = (int)(pix / Wp) - pad_h, w = (int)(pix % Wp) - pad_w;
         const bool in = h >= 0 && h < H && w >= 0 && w < W;
         const float *src = x + nc8 * 8 * HW + (in ? (long long)h * W + w : 0);
         float hi[8], lo[8];
@@ -206,7 +206,7 @@ __device__ __forceinline__ bool ig_mma_loop(const IgemmParams &p, uint32_t tmem,
     constexpr uint32_t idesc_c = dev::idesc_bf16(128, NT);
     constexpr bool FIX = TH_ > 0;
     const int TH = FIX ? TH_ : p.TH, R = FIX ? R_ : p.R, S = FIX ? S_ : p.S;
-    const int dil = FIX ? 1 : p.dil;
+    const int dil = FIX ? 1 : p.dil, dil_w = FIX ? 1 : p.dil_w;
     const int COLS = FIX ? (128 + S_ - 1 + 15) / 16 * 16 : p.COLS;
     const uint32_t a_bytes = 32u * (uint32_t)COLS * (uint32_t)(TH + (R - 1) * dil);
     const uint32_t a_lbo = a_bytes / 2;          // one channel quad / bf16 chunk apart
@@ -242,8 +242,8 @@ __device__ __forceinline__ bool ig_mma_loop(const IgemmParams &p, uint32_t tmem,
                     const uint32_t d = dbase + (uint32_t)(i * NT);
 #pragma unroll
                     for (int s = 0; s < S; ++s) {
-                        // 16-byte units: staged row i + r*dil, column s*dil
-                        const uint64_t ao = (uint64_t)((i + r * dil) * COLS + s * dil);
+                        // 16-byte units: staged row i + r*dil, column s*dil_w
+                        const uint64_t ao = (uint64_t)((i + r * dil) * COLS + s * dil_w);
                         const uint64_t bo = (uint64_t)(s * 2 * NT);
                         const uint32_t acc = (cc8 > 0 || r > 0 || s > 0) ? 1u : 0u;
                         // cross terms x_hi*w_lo + x_lo*w_hi: one bf16 MMA over K = 16
@@ -281,6 +281,7 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
     uint64_t *acce = fullA + 18;                            // [2] accumulator drained
     uint32_t *tslot = reinterpret_cast<uint32_t *>(fullA + 20);
     int *abort_flag = reinterpret_cast<int *>(fullA + 21);
+    uint64_t *drain = fullA + 22;                           // every issued MMA has completed
     constexpr bool CHAIN = KGN > 0;
     unsigned char *stages = smem + ig_header(NT, CHAIN);
 
@@ -304,6 +305,7 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
             dev::mbar_init(&accf[b], 1);
             dev::mbar_init(&acce[b], ig_epi_warps(NT));
         }
+        dev::mbar_init(drain, 1);
         *abort_flag = 0;
         dev::fence_mbar_init();
     }
@@ -370,6 +372,18 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
             *abort_flag = 1;
             atomicExch(&g_igemm_error, 1);
         }
+        if (lane == 0) {
+            // copies still in flight (only after an abort): wait, bounded, for the
+            // last phase issued on every slot before the CTA may exit
+            for (int j = ia > p.sa ? ia - p.sa : 0; j < ia; ++j)
+                dev::mbar_wait_bounded(&fullA[j % p.sa], (uint32_t)(j / p.sa) & 1u);
+            if (p.b_resident) {
+                for (int j = 0; j < ib; ++j) dev::mbar_wait_bounded(&fullB[j], 0);
+            } else {
+                for (int j = ib > p.sb ? ib - p.sb : 0; j < ib; ++j)
+                    dev::mbar_wait_bounded(&fullB[j % p.sb], (uint32_t)(j / p.sb) & 1u);
+            }
+        }
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
@@ -378,7 +392,7 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
             // (dilation 1, default rows per tile): the issue loop then runs
             // back to back on constant operand offsets
             constexpr int THD = ig_default_th(NT);
-            const bool d1 = p.dil == 1 && p.TH == THD;
+            const bool d1 = p.dil == 1 && p.dil_w == 1 && p.TH == THD;
             bool ok;
             if (d1 && p.R == 3 && p.S == 3) ok = ig_mma_loop<NT, THD, 3, 3>(p, tmem, ringA, ringB, a_slot, b_slot, fullA, emptyA, fullB, emptyB, accf, acce);
             else if (d1 && p.R == 5 && p.S == 9) ok = ig_mma_loop<NT, THD, 5, 9>(p, tmem, ringA, ringB, a_slot, b_slot, fullA, emptyA, fullB, emptyB, accf, acce);
@@ -388,6 +402,10 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
                 *abort_flag = 1;
                 atomicExch(&g_igemm_error, 1);
             }
+            // no MMA may still be running when TMEM is released: one more commit
+            // arrives once every MMA this thread issued has completed
+            dev::mma_commit(drain);
+            dev::mbar_wait_bounded(drain, 0);
         }
         __syncwarp();
     } else {
@@ -626,12 +644,12 @@ bool make_nc4hw4_tile_map(TensorMap *tm, const float *base, long long quads, int
     return r == CUDA_SUCCESS;
 }
 
-cudaError_t launch_split_x(const float *x, float *xh, float *xl, int N, int C, int H, int W, int pad, int Hp,
-                           int Wp, cudaStream_t st) {
+cudaError_t launch_split_x(const float *x, float *xh, float *xl, int N, int C, int H, int W, int pad_h, int pad_w,
+                           int Hp, int Wp, cudaStream_t st) {
     const long long cells = (long long)N * (C / 8) * Hp * Wp;
     const long long blocks = std::min<long long>((cells + 255) / 256, 148LL * 64);
     return launch_ex(split_x_kernel, dim3((unsigned)blocks), dim3(256), 0, st, x, reinterpret_cast<float4 *>(xh),
-                     reinterpret_cast<uint4 *>(xl), C / 8, H, W, pad, Hp, Wp, cells);
+                     reinterpret_cast<uint4 *>(xl), C / 8, H, W, pad_h, pad_w, Hp, Wp, cells);
 }
 
 cudaError_t launch_split_w(const float *w, float *wh, float *wl, int K, int cpg, int R, int S, int groups,

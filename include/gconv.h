@@ -26,8 +26,9 @@
  *  - The operation is a cross-correlation (no kernel flip): output channel k
  *    belongs to group k / (K/groups) and reads input channels
  *    [gi*C/groups, (gi+1)*C/groups); taps outside the image read zero.
- *  - Stride, padding and dilation are the same along H and W; the kernel may
- *    be non-square (R != S).
+ *  - Stride, padding and dilation are the same along H and W, except in
+ *    gconv2d_fwd_ex, which takes them per axis; the kernel may be non-square
+ *    (R != S).
  *  - Every call is asynchronous on `stream` (0 = legacy default stream).  It
  *    performs no host synchronisation and no device allocation, except the
  *    one-time workspace allocation described at gconv_reserve_workspace.
@@ -84,6 +85,25 @@ GCONV_API gconv_status_t gconv2d_fwd(const float *x, const float *w, const float
                            int N, int C, int H, int W, int K, int R, int S,
                            int stride, int pad, int dilation, int groups,
                            float *y, cudaStream_t stream);
+
+/* Convolution forward with stride, padding and dilation given per axis
+ * ("Kimi-K2.6__l1_p62", ModelNew.forward: the layer's padding, stride and
+ * dilation may each be an (h, w) tuple, which a single int cannot carry; the
+ * transcript's fix is a signature taking padding_h, padding_w, dilation_h,
+ * dilation_w, stride_h and stride_w):
+ *   y[n,k,p,q] = bias[k] + sum_{c,r,s} w[k,c,r,s] * x[n, gi*C/g + c,
+ *                       p*stride_h - pad_h + r*dil_h, q*stride_w - pad_w + s*dil_w]
+ *   P = floor((H + 2*pad_h - dil_h*(R-1) - 1)/stride_h) + 1,
+ *   Q = floor((W + 2*pad_w - dil_w*(S-1) - 1)/stride_w) + 1.
+ * Equal values on both axes give exactly gconv2d_fwd (same kernels, same
+ * bits).  Unequal ones run on the general-geometry direct kernel, or on the
+ * implicit GEMM when both strides are 1 and the groups are wide enough.
+ * Arguments, layout, alignment, streams, workspace and errors as
+ * gconv2d_fwd (each stride and dilation >= 1, each padding >= 0). */
+GCONV_API gconv_status_t gconv2d_fwd_ex(const float *x, const float *w, const float *bias,
+                           int N, int C, int H, int W, int K, int R, int S,
+                           int stride_h, int stride_w, int pad_h, int pad_w, int dil_h, int dil_w,
+                           int groups, float *y, cudaStream_t stream);
 
 /* Convolution with a per-output-channel affine epilogue and a clamp:
  *   y[n,k,p,q] = min(max(conv(x, w)[n,k,p,q] * scale[k] + shift[k], lo), hi)
@@ -177,6 +197,11 @@ GCONV_API gconv_status_t gconv_reserve_workspace(size_t bytes);
  * `chain` != 0 asks about the fused chain's conv stage. */
 GCONV_API const char *gconv2d_plan_name(int N, int C, int H, int W, int K, int R, int S,
                               int stride, int pad, int dilation, int groups, int chain);
+
+/* gconv2d_plan_name for the per-axis geometry of gconv2d_fwd_ex. */
+GCONV_API const char *gconv2d_plan_name_ex(int N, int C, int H, int W, int K, int R, int S,
+                              int stride_h, int stride_w, int pad_h, int pad_w, int dil_h, int dil_w,
+                              int groups);
 
 /* Force a kernel family for subsequent calls on this process, by name
  * ("auto" restores per-shape dispatch).  A forced family that cannot run a

@@ -144,3 +144,17 @@ def test_selftest_wait_timeout_rejects_bad_limits(lib):
     # validated on the host: nothing is launched
     assert lib.gconv_selftest_wait_timeout(0, None) == gc.ERR_INVALID_ARG
     assert lib.gconv_selftest_wait_timeout((1 << 24) + 1, None) == gc.ERR_INVALID_ARG
+
+
+def test_per_axis_entry_point_validates_and_plans(lib):
+    f = lib.gconv2d_fwd_ex
+    geo = (1, 4, 8, 8, 4, 3, 3)
+    # each per-axis value checked on its own
+    for bad in [(0, 1, 1, 1, 1, 1), (1, 0, 1, 1, 1, 1), (1, 1, -1, 1, 1, 1), (1, 1, 1, -1, 1, 1),
+                (1, 1, 1, 1, 0, 1), (1, 1, 1, 1, 1, 0), (1, 1, 0, 0, 5, 1)]:
+        assert f(FAKE, FAKE, None, *geo, *bad, 4, FAKE, None) == gc.ERR_INVALID_ARG, bad
+    # unequal axes use the general-geometry kernel; equal axes plan like gconv2d_fwd
+    assert gc.plan_name(2, 16, 30, 34, 16, 3, 3, (1, 2), (1, 0), 1, 16) == "direct_generic"
+    assert gc.plan_name(2, 32, 24, 36, 64, 5, 9, 1, (2, 4), 1, 1) == "igemm_tf32_bf16x"
+    assert gc.plan_name(4, 144, 56, 56, 144, 3, 3, (1, 1), (1, 1), (1, 1), 144) == \
+        gc.plan_name(4, 144, 56, 56, 144, 3, 3, 1, 1, 1, 144)

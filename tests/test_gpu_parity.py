@@ -283,6 +283,45 @@ def test_stream_affine_clamp_and_misaligned_output(oracle_mod):
     assert np.all(err <= tol), f"max err/tol {np.max(err / tol):.3g}"
 
 
+# per-axis stride / padding / dilation ("Kimi-K2.6__l1_p62", padding as an (h, w) tuple)
+AXIS_GEOMS = [
+    # N, C, H, W, K, R, S, (sh, sw), (ph, pw), (dh, dw), groups, bias
+    (2, 16, 30, 34, 16, 3, 3, (1, 2), (1, 0), (1, 1), 16, True),      # depthwise, generic kernel
+    (1, 8, 21, 40, 16, 3, 5, (2, 1), (0, 2), (1, 2), 4, False),
+    (2, 32, 24, 36, 64, 5, 9, (1, 1), (2, 4), (1, 1), 1, True),       # "same" 5x9: implicit GEMM
+    (1, 16, 17, 29, 32, 3, 3, (1, 1), (2, 1), (2, 1), 1, False),      # implicit GEMM, dilation (2, 1)
+    (1, 8, 16, 16, 8, 3, 3, (1, 1), (1, 1), (1, 1), 8, True),         # equal axes: the plain entry point
+]
+
+
+@pytest.mark.parametrize("geo", AXIS_GEOMS, ids=lambda g: "x".join(map(str, g[:7])) + f"_s{g[7]}_p{g[8]}_d{g[9]}")
+def test_per_axis_geometry_matches_oracle(oracle_mod, geo):
+    N, C, H, W, K, R, S, st, pad, dil, g, bias = geo
+    d = inputs.conv_inputs(N, C, H, W, K, R, S, g, seed=19 + zlib.crc32(repr(geo).encode()) % 1000,
+                           x_dist="normal", bias=bias)
+    ref, acc = oracle_mod.conv2d(d["x"], d["w"], d.get("bias"), st, pad, dil, g, return_absacc=True)
+    out = Guarded(ref.shape)
+    gc.conv2d(d["x"].cuda(), d["w"].cuda(), d["bias"].cuda() if bias else None, st, pad, dil, g, out=out.y)
+    torch.cuda.synchronize()
+    out.check()
+    assert_conv_close(out.y.cpu().numpy(), ref, acc, "per-axis " + str(geo))
+
+
+def test_per_axis_equal_values_are_bitwise_the_plain_entry_point():
+    d = inputs.conv_inputs(2, 32, 28, 28, 32, 3, 3, 32, seed=4700, x_dist="normal")
+    x, w = d["x"].cuda(), d["w"].cuda()
+    lib = gc.library()
+    a = torch.empty(2, 32, 28, 28, device="cuda")
+    b = torch.empty(2, 32, 28, 28, device="cuda")
+    h = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert lib.gconv2d_fwd(x.data_ptr(), w.data_ptr(), None, 2, 32, 28, 28, 32, 3, 3, 1, 1, 1, 32,
+                           a.data_ptr(), h) == gc.OK
+    assert lib.gconv2d_fwd_ex(x.data_ptr(), w.data_ptr(), None, 2, 32, 28, 28, 32, 3, 3, 1, 1, 1, 1, 1, 1, 32,
+                              b.data_ptr(), h) == gc.OK
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
 def test_forced_cpasync_chain(oracle_mod):
     d = inputs.chain_inputs(2, 8, 40, 40, 32, 3, 3, 1, 8, seed=64, bias_scale_std=1.0, affine="random")
     gc.force_kernel("direct_cpasync")

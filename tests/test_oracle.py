@@ -134,6 +134,67 @@ def test_library_float64_conv(oracle_mod):
         np.testing.assert_allclose(y, _tconv(x, w, b, st, pad, dil, g), rtol=1e-11, atol=1e-11)
 
 
+# ---------------------------------------------------------------- per-axis geometry
+# ("Kimi-K2.6__l1_p62", ModelNew.forward: padding, stride and dilation as (h, w)
+# tuples).  Each check takes different values on the two axes, so an axis mix-up
+# (the W index reading the H padding, swapped strides) fails it.
+
+def test_per_axis_all_ones_counts_in_bounds_taps(oracle_mod):
+    for (H, W, R, S, sh, sw, ph, pw, dh, dw) in [(9, 12, 3, 5, 1, 2, 0, 2, 1, 1), (11, 8, 5, 3, 2, 1, 3, 0, 1, 2),
+                                                 (7, 13, 3, 3, 1, 1, 1, 0, 2, 1), (12, 12, 1, 3, 3, 1, 0, 1, 1, 3)]:
+        x = np.ones((1, 2, H, W), np.float32)
+        w = np.ones((2, 1, R, S), np.float32)
+        y = oracle_mod.conv2d(x, w, None, (sh, sw), (ph, pw), (dh, dw), 2)
+        P, Q = y.shape[2:]
+        assert P == (H + 2 * ph - dh * (R - 1) - 1) // sh + 1 and Q == (W + 2 * pw - dw * (S - 1) - 1) // sw + 1
+        for p in range(P):
+            nr = sum(1 for r in range(R) if 0 <= p * sh - ph + r * dh < H)
+            for q in range(Q):
+                ns = sum(1 for s_ in range(S) if 0 <= q * sw - pw + s_ * dw < W)
+                assert y[0, 0, p, q] == nr * ns and y[0, 1, p, q] == nr * ns, (p, q)
+
+
+def test_per_axis_shifted_delta_is_shift(oracle_mod):
+    g = inputs.generator(3)
+    x = inputs.normal((1, 2, 9, 14), 1.0, g).numpy()
+    # a 3x5 kernel, padding (1, 2), tap (r, s) = (2, 0): y[p, q] = x[p + 1, q - 2] (zero outside)
+    w = np.zeros((2, 1, 3, 5), np.float32)
+    w[:, 0, 2, 0] = 1.0
+    y = oracle_mod.conv2d(x, w, None, 1, (1, 2), 1, 2)
+    want = np.zeros_like(y)
+    want[:, :, :-1, 2:] = x[:, :, 1:, :-2]
+    np.testing.assert_array_equal(y, want)
+    # strides (2, 3) with the centre tap of a 3x3 and padding (1, 1): y[p, q] = x[2p, 3q]
+    w = np.zeros((2, 1, 3, 3), np.float32)
+    w[:, 0, 1, 1] = 1.0
+    y = oracle_mod.conv2d(x, w, None, (2, 3), 1, 1, 2)
+    np.testing.assert_array_equal(y, x[:, :, ::2, ::3][:, :, :y.shape[2], :y.shape[3]].astype(np.float64))
+
+
+def test_per_axis_library_float64_conv(oracle_mod):
+    rng = np.random.default_rng(8)
+    for (N, C, H, W, K, R, S, st, pad, dil, g, bias) in [
+            (2, 8, 15, 17, 8, 3, 3, (1, 2), (1, 0), (1, 1), 8, False),
+            (1, 6, 13, 19, 12, 5, 9, (1, 1), (2, 4), (1, 1), 1, True),     # "same" padding of the 5x9 kernel
+            (2, 8, 14, 12, 16, 3, 3, (2, 1), (0, 1), (2, 1), 2, True),
+            (1, 4, 10, 16, 8, 3, 5, (1, 3), (2, 1), (1, 2), 4, False)]:
+        x = rng.standard_normal((N, C, H, W)).astype(np.float32)
+        w = rng.standard_normal((K, C // g, R, S)).astype(np.float32)
+        b = rng.standard_normal(K).astype(np.float32) if bias else None
+        y = oracle_mod.conv2d(x, w, b, st, pad, dil, g)
+        np.testing.assert_allclose(y, _tconv(x, w, b, st, pad, dil, g), rtol=1e-11, atol=1e-11)
+
+
+def test_per_axis_same_padding_of_the_5x9_kernel(oracle_mod):
+    # the dense transcript's 512x512 input and (5, 9) kernel: padding (2, 4) keeps 512x512
+    assert oracle_mod.out_extent(512, 5, 1, 2, 1) == 512 and oracle_mod.out_extent(512, 9, 1, 4, 1) == 512
+    x = np.ones((1, 1, 6, 10), np.float32)
+    w = np.ones((1, 1, 5, 9), np.float32)
+    y = oracle_mod.conv2d(x, w, None, 1, (2, 4), 1, 1)
+    assert y.shape == (1, 1, 6, 10)
+    assert y[0, 0, 2, 4] == 5 * 9 and y[0, 0, 0, 0] == 3 * 5
+
+
 def test_grouped_equals_concatenated_dense(oracle_mod):
     rng = np.random.default_rng(7)
     N, C, H, W, K, g = 2, 12, 9, 10, 18, 3

@@ -26,6 +26,14 @@ MUTATIONS = [
      "if (ih < 0 || ih >= g->H) continue;",
      "if (ih < 0) ih = 0; if (ih >= g->H) ih = g->H - 1;",
      ["all_ones", "shifted_delta", "library"]),
+    ("W index reads the H padding",
+     "long iw = q * g->sw - g->pw + s * g->dw;",
+     "long iw = q * g->sw - g->ph + s * g->dw;",
+     ["axis_all_ones", "axis_shift", "axis_library"]),
+    ("row index takes the W stride",
+     "long ih = p * g->sh - g->ph + r * g->dh;",
+     "long ih = p * g->sw - g->ph + r * g->dh;",
+     ["axis_all_ones", "axis_shift", "axis_library"]),
     ("output size rounded up",
      "return span / stride + 1;",
      "return (span + stride - 1) / stride + 1;",
@@ -55,6 +63,9 @@ PINS = {
     "gn_closed": lambda m: pins.test_chain_groupnorm_closed_forms(m),
     "chain_library": lambda m: pins.test_chain_matches_float64_library(m, 1.0, "random"),
     "bias_before_scale": lambda m: pins.test_chain_bias_before_scale(m),
+    "axis_all_ones": lambda m: pins.test_per_axis_all_ones_counts_in_bounds_taps(m),
+    "axis_shift": lambda m: pins.test_per_axis_shifted_delta_is_shift(m),
+    "axis_library": lambda m: pins.test_per_axis_library_float64_conv(m),
 }
 
 

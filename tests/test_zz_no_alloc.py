@@ -4,10 +4,11 @@ Callers that cannot allocate device memory while they run (a CUDA graph being
 recorded, an engine with a fixed memory budget, a host whose allocator belongs
 to another framework) use gconv2d_bias_scale_sigmoid_groupnorm_fwd_noalloc,
 which keeps its GroupNorm partial statistics in a fixed scratch array instead
-of a cudaMalloc'd workspace.  These tests check that it returns what the
-regular entry point returns, on two calls in a row (the second call must not
-see anything the first left in the shared scratch), and that shapes needing
-more scratch than the array holds are refused without launching.
+of a cudaMalloc'd workspace.  These tests check, on two calls in a row (the
+second call must not see anything the first left in the shared scratch), that
+it returns what the regular entry point returns and that both agree with the
+FP64 oracle within the chain's error bound, and that shapes needing more
+scratch than the array holds are refused without launching.
 
 This file is named so that pytest collects it last."""
 import ctypes
@@ -19,7 +20,7 @@ import torch
 import depthwise_convolution_fp32_b200 as gc
 from depthwise_convolution_fp32_b200 import build, inputs
 
-from tolerance import chain_tols
+from tolerance import assert_chain_close, chain_tols
 
 pytestmark = pytest.mark.gpu
 
@@ -60,8 +61,6 @@ def test_noalloc_matches_regular_entry_point_twice(lib, oracle_mod, geo, gn, std
     N, C, H, W, K, R, S, st, pad, dil, g = geo
     P, Q = gc.output_size(H, W, R, S, st, pad, dil)
     eps = 1e-5
-    assert gc.chain_workspace_size(N, C, H, W, K, R, S, st, pad, dil, g, gn) <= \
-        lib.gconv_noalloc_scratch_capacity()
     for call in range(2):        # two calls in a row on different inputs
         d = inputs.chain_inputs(N, C, H, W, K, R, S, g, gn, seed=900 + 17 * call,
                                 bias_scale_std=std, affine="random")
@@ -78,6 +77,9 @@ def test_noalloc_matches_regular_entry_point_twice(lib, oracle_mod, geo, gn, std
         a = y_new.cpu().numpy().astype(np.float64)
         b = y_ref.cpu().numpy().astype(np.float64)
         assert np.all(np.abs(a - b) <= tau_y), f"call {call}: max diff {np.nanmax(np.abs(a - b))}"
+        # and each result against the oracle directly, so a fault both paths share cannot hide
+        assert_chain_close(a, ref, d["scale"].numpy(), d["gamma"].numpy(), eps, K // gn, f"noalloc call {call}")
+        assert_chain_close(b, ref, d["scale"].numpy(), d["gamma"].numpy(), eps, K // gn, f"regular call {call}")
     assert lib.gconv_device_error_status() == gc.OK
 
 
@@ -88,8 +90,7 @@ def test_noalloc_refuses_shapes_beyond_capacity(lib):
     geo = (16384, 8, 4, 4, 32, 3, 3, 1, 0, 1, 1)
     gn = 32
     N, C, H, W, K, R, S, st, pad, dil, g = geo
-    need = gc.chain_workspace_size(N, C, H, W, K, R, S, st, pad, dil, g, gn)
-    assert need > lib.gconv_noalloc_scratch_capacity()
+    assert N * gn * 16 > lib.gconv_noalloc_scratch_capacity()
     P, Q = gc.output_size(H, W, R, S, st, pad, dil)
     # real, correctly sized buffers: nothing may be launched, but nothing
     # could go out of bounds if it were
