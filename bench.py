@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload depthwise|tiny_grouped|fused_chain|dense_5x9]
-                    [--no-shapes] [--sweep] [--force-kernel NAME]
+                    [--no-shapes] [--force-kernel NAME]
     python bench.py --profile --workload NAME [--batch B] [--calls C]   (ncu target)
 
 One step = one call of the library's entry point on one batch of the
@@ -114,17 +114,50 @@ def weak_scaling_rate(units_per_step, world, steps, ms):
 
 TF32_OVER_BF16 = 1.1 / 2.25      # nominal dense tf32 / bf16 tensor throughput on B200
 
+# Compute rates measured on this GPU at start-up by libgconv_peaks.so (FP32
+# FMA; tcgen05 kind::tf32 and kind::f16/bf16 MMA), reported beside the roofline
+# denominators to corroborate them.
+MEASURED_COMPUTE = {}
+
+
+def measure_compute_peaks():
+    """FP32 CUDA-core and tensor-core MMA rates of this GPU (TFLOP/s), each
+    from one timed launch of a throughput microbenchmark (a few ms each)."""
+    import ctypes
+    from depthwise_convolution_fp32_b200 import build
+    lib = ctypes.CDLL(build.build_peaks())
+    out = {}
+    for name, fn, iters in (("fp32_fma", lib.gpeaks_ffma, 4096), ("tf32_mma", lib.gpeaks_mma_tf32, 20000),
+                            ("bf16_mma", lib.gpeaks_mma_bf16, 20000)):
+        fn.restype = ctypes.c_int
+        fn.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]
+        ms, fl = ctypes.c_double(0), ctypes.c_double(0)
+        rc = fn(iters, ctypes.byref(ms), ctypes.byref(fl))
+        if rc == 0 and ms.value > 0:
+            out[name + "_tflops"] = round(fl.value / (ms.value * 1e-3) / 1e12, 2)
+            out[name + "_ms"] = round(ms.value, 3)
+    if "tf32_mma_tflops" in out and "bf16_mma_tflops" in out:
+        # one useful FP32-accurate multiply-add = one tf32 MAC + two bf16 MACs
+        t, b = out["tf32_mma_tflops"], out["bf16_mma_tflops"]
+        out["fp32_accurate_tensor_tflops"] = round(1.0 / (1.0 / t + 2.0 / b), 2)
+    MEASURED_COMPUTE.update(out)
+    return out
+
 
 def fp32_peak_tflops():
-    """CUDA-core FP32 peak: 148 SMs x 128 FMA lanes x 2 FLOP x 1965 MHz."""
+    """Roofline denominator of the CUDA-core path (bound "alu"): 148 SMs x 128
+    FP32 FMA lanes x 2 FLOP x 1965 MHz, from unit counts and the clock.  The
+    FMA microbenchmark's measured rate is reported beside it (compute_peaks)."""
     return wl.fp32_fma_peak_tflops()
 
 
 def tensor_fp32_peak_tflops(meas):
-    """Useful FP32 FLOP/s ceiling of the tensor-core path: each multiply-add
-    costs one tf32 MAC (main term) plus two bf16 MACs (the two cross terms,
-    one K=16 bf16 MMA per 8 channels).  With the measured bf16 GEMM peak and
-    the nominal tf32/bf16 ratio r, the ceiling is bf16 / (1/r + 2)."""
+    """Roofline denominator of the tensor-core path: useful FP32 FLOP/s when
+    each multiply-add costs one tf32 MAC (main term) plus two bf16 MACs (the
+    two cross terms, one K=16 bf16 MMA per 8 channels).  With the measured bf16
+    GEMM peak (MEASURED_PEAKS.json, else the 1.59 PFLOP/s fallback) and the
+    nominal tf32/bf16 ratio r: bf16 / (1/r + 2).  The tcgen05 MMA
+    microbenchmarks' tf32 and bf16 rates are reported beside it."""
     bf16 = float(meas.get("bf16_tflops", 1590.0)) if meas else 1590.0
     return bf16 / (1.0 / TF32_OVER_BF16 + 2.0)
 
@@ -242,6 +275,12 @@ class Workload:
             d = inputs.chain_inputs(s.N, s.C, s.H, s.W, s.K, s.R, s.S, 1, wl.FUSED_CHAIN.gn_groups,
                                     seed=wl.SEEDS["fused_chain"])
             self.host = d
+        elif name.startswith("ring"):
+            N, C, H, W, K, R, pad, g = THRESHOLD_RING[int(name[4:])]
+            s = wl.ConvShape(N=N, C=C, H=H, W=W, K=K, R=R, S=R, stride=1, pad=pad, groups=g)
+            self.shape = s
+            self.host = inputs.conv_inputs(s.N, s.C, s.H, s.W, s.K, R, R, g, 5000 + int(name[4:]),
+                                           x_dist="normal", w_bound=1 / math.sqrt(R * R * s.cpg))
         elif name.startswith("sweep"):
             i = int(name[5:])
             s = wl.sweep80()[i]
@@ -425,10 +464,22 @@ def time_sync_api(runner: DeviceRunner, steps: int):
     return statistics.median(lat) * 1e6
 
 
-def cpu_oracle_rate(wk: Workload, budget_s: float):
-    """Time the FP64 oracle, as it stands, on this host's cores on a bounded
-    sample of the workload; returns (GB/s, sample description, threads)."""
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_oracle_rate(wk: Workload, budget_s: float, threads: int = 0):
+    """Time the FP64 oracle, as it stands, on this host's cores (all of them, or
+    `threads`) on a bounded sample of the workload; returns (GB/s, sample
+    description, threads used)."""
     import oracle
+    oracle.set_num_threads(threads if threads > 0 else (os.cpu_count() or 1))
     s = wk.shape
     h = wk.host
     x = h["x"].numpy()
@@ -589,6 +640,109 @@ def write_records(args, gc, device, l2, hbm_peak, meas, batches=10, per_batch=30
     print(json.dumps({"records": len(out), "file": args.records}))
 
 
+# shapes around the implicit-GEMM threshold (channels per group x taps near 64,
+# output channels per group at the tensor path's minimum of 32): x[N,C,H,W], K,
+# R=S, pad, groups
+THRESHOLD_RING = [
+    (8, 32, 56, 56, 32, 3, 1, 1), (8, 64, 56, 56, 64, 3, 1, 1), (8, 128, 28, 28, 128, 3, 1, 4),
+    (8, 16, 56, 56, 32, 3, 1, 1), (8, 8, 128, 128, 32, 3, 1, 1), (8, 64, 56, 56, 64, 1, 0, 1),
+    (8, 128, 28, 28, 128, 1, 0, 1), (8, 256, 28, 28, 256, 3, 1, 8),
+]
+
+
+def tuning_workloads():
+    out = [Workload(n) for n in ("tiny_grouped", "depthwise", "fused_chain", "dense_5x9")]
+    out += [Workload(f"sweep{i}") for i in range(80)]
+    for j, (N, C, H, W, K, R, pad, g) in enumerate(THRESHOLD_RING):
+        out.append(Workload(f"ring{j}"))
+    return out
+
+
+def candidate_families(gc, s, chain):
+    """Kernel families (force names) that can run the shape, direct ones per
+    channels-per-thread choice."""
+    c = []
+    for fam in ("direct_stream", "direct_blocked"):
+        if chain and fam == "direct_stream":
+            continue
+        for kt in (1, 2, 4, 8):
+            if s.kpg % kt:
+                continue
+            if chain and (wl.FUSED_CHAIN.conv.K // wl.FUSED_CHAIN.gn_groups) % kt and \
+                    kt % (wl.FUSED_CHAIN.conv.K // wl.FUSED_CHAIN.gn_groups):
+                continue
+            name = f"{fam}:kt{kt}"
+            gc.force_kernel(name)
+            plan = gc.plan_name(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil, s.groups, chain)
+            if plan not in ("unsupported", "invalid") and (fam != "direct_stream" or "stream" in plan):
+                c.append(name)
+    gc.force_kernel("igemm")
+    if gc.plan_name(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil, s.groups, chain).startswith("igemm"):
+        c.append("igemm")
+    gc.force_kernel("auto")
+    return c
+
+
+def write_dispatch_table(args, gc, device, l2, batches=3, per_batch=20):
+    """Per tuning shape: time every candidate family under the benchmark's own
+    graph timing (rotating buffers larger than L2, `per_batch` calls per graph,
+    mean over `batches` replays) and keep the fastest.  Candidates within 1% of
+    the fastest keep the planner's own default order (streaming, blocked,
+    implicit GEMM) so the table only overrides where the measurement says so."""
+    import torch
+    entries = []
+    for wk in tuning_workloads():
+        s = wk.shape
+        cands = candidate_families(gc, s, wk.chain)
+        if not cands:
+            continue
+        r = DeviceRunner(wk, device, l2)
+        us = {}
+        for name in cands:
+            gc.force_kernel(name)
+            try:
+                for i in range(3):
+                    r.step(i)
+                torch.cuda.synchronize()
+                g = torch.cuda.CUDAGraph()
+                st = torch.cuda.Stream()
+                st.wait_stream(torch.cuda.current_stream())
+                with torch.cuda.stream(st):
+                    with torch.cuda.graph(g, stream=st):
+                        for i in range(per_batch):
+                            r.step(i)
+                torch.cuda.synchronize()
+                g.replay()
+                torch.cuda.synchronize()
+                t = []
+                for b in range(batches):
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    with torch.cuda.stream(st):
+                        e0.record(st)
+                        g.replay()
+                        e1.record(st)
+                    torch.cuda.synchronize()
+                    t.append(e0.elapsed_time(e1) * 1e3 / per_batch)
+                del g
+                us[name] = round(statistics.mean(t), 3)
+            finally:
+                gc.force_kernel("auto")
+        best = min(us, key=us.get)
+        entries.append({"workload": wk.name, "shape": [s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil,
+                                                       s.groups],
+                        "chain": 1 if wk.chain else 0, "best": best, "us": us})
+        print(json.dumps({"workload": wk.name, "best": best, "us": us[best]}), flush=True)
+        del r
+        torch.cuda.empty_cache()
+    with open(args.dispatch_table, "w") as f:
+        json.dump({"about": "per-shape kernel choice measured on B200 with bench.py --dispatch-table: graph "
+                            "device time per call (rotating buffers larger than L2), every family that can "
+                            "run the shape; 'best' is compiled into libgconv.so, other shapes follow the "
+                            "planner's rules",
+                   "device": torch.cuda.get_device_name(device), "batches": batches, "per_batch": per_batch,
+                   "entries": entries}, f, indent=1)
+
+
 # ------------------------------------------------------------------ main
 
 def main():
@@ -599,8 +753,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="depthwise")
     ap.add_argument("--no-shapes", action="store_true",
-                    help="skip timing the other page workloads (tiny grouped, depthwise, chain, dense)")
-    ap.add_argument("--sweep", action="store_true", help="also time the 80-shape sweep")
+                    help="skip the other page workloads (tiny grouped, depthwise, chain, dense) and the "
+                         "80-shape sweep")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--records", default=None,
                     help="write per-shape records (page workloads + 80-shape sweep) to this JSON file "
@@ -615,6 +769,11 @@ def main():
                          "followed by a synchronize, print one line and exit (no timing)")
     ap.add_argument("--batch", type=int, default=0, help="--profile: override N (0: the workload's own)")
     ap.add_argument("--calls", type=int, default=2, help="--profile: number of calls")
+    ap.add_argument("--dispatch-table", default=None,
+                    help="time every kernel family (and direct-kernel channels per thread) on the tuning "
+                         "shapes (page workloads, 80-shape sweep, shapes around the implicit-GEMM "
+                         "threshold) and write the per-shape choices to this JSON file "
+                         "(depthwise_convolution_fp32_b200/dispatch_table.json is the compiled-in copy)")
     ap.add_argument("--profile-graph", action="store_true",
                     help="profiler target: capture --steps calls of --workload (rotating buffers, as the "
                          "timed region) in one CUDA graph and replay it once inside the NVTX range "
@@ -651,9 +810,13 @@ def main():
     props = torch.cuda.get_device_properties(device)
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
     hbm_peak, peak_kind, meas = peaks()
+    if not (args.profile or args.profile_graph):
+        measure_compute_peaks()
 
     if args.records:
         return write_records(args, gc, device, l2, hbm_peak, meas)
+    if args.dispatch_table:
+        return write_dispatch_table(args, gc, device, l2)
     if args.profile:
         return run_profile_case(args, gc, device)
     if args.profile_graph:
@@ -699,46 +862,97 @@ def main():
                 "d2h_bytes_per_step": d2h},
         "roofline": roof,
         "gpu_launches": launches * args.steps,
+        "compute_peaks": dict(MEASURED_COMPUTE, note="microbenchmarks on this GPU, reported beside the "
+                              "roofline denominators (alu: unit counts x clock; tensor: bf16 GEMM peak x "
+                              "nominal tf32 ratio)", alu_peak_tflops=round(fp32_peak_tflops(), 2),
+                              tensor_peak_tflops=round(tensor_fp32_peak_tflops(meas), 2)),
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         "clock_samples": {"n": clocks.get("samples"), "window": clocks.get("window")},
     }
 
-    if not args.no_shapes or args.sweep:
-        extra = {}
-        names = [] if args.no_shapes else ["tiny_grouped", "depthwise", "fused_chain", "dense_5x9"]
-        if args.sweep:
-            names += [f"sweep{i}" for i in range(80)]
-        for nm in names:
+    if not args.no_shapes:
+        # every page workload with the headline's fields: graph time, roofline,
+        # end-to-end through the public API, synchronous API, CPU oracle baseline
+        cfgs = {}
+        for nm in ("tiny_grouped", "depthwise", "fused_chain", "dense_5x9"):
             if nm == args.workload:
                 continue
-            w2 = Workload(nm)
-            r2 = DeviceRunner(w2, device, l2)
-            k2 = max(3, min(args.steps, 20))
-            ms2, _, _ = time_graph(r2, k2, 3, barrier)
-            sec = ms2 / 1e3 / k2
-            s2 = w2.shape
-            plan2 = gc.plan_name(s2.N, s2.C, s2.H, s2.W, s2.K, s2.R, s2.S, s2.stride, s2.pad, s2.dil,
-                                 s2.groups, w2.chain)
-            extra[nm] = {"us": round(sec * 1e6, 3), "GB/s": round(w2.bytes / sec / 1e9, 1),
-                         "GFLOP/s": round(w2.flops / sec / 1e9, 1), "kernel": plan2,
-                         "roofline": roofline_for(w2, sec, plan2, hbm_peak, meas),
-                         "label": s2.label()}
-            del r2
+            cfgs[nm] = measure_config(nm, gc, device, l2, hbm_peak, meas, barrier, args, rank, world)
             torch.cuda.empty_cache()
-        result["shapes"] = extra
+        result["configs"] = cfgs
+        result["sweep80"] = measure_sweep(gc, device, l2, hbm_peak, meas, barrier)
 
     if args.workload == "depthwise" and not args.no_block:
         result["mobilenetv2_block"] = measure_block(device, max(20, min(args.steps, 200)), args.warmup)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gbs, desc, thr = cpu_oracle_rate(wk, args.cpu_budget)
+        gbs1, _, _ = cpu_oracle_rate(wk, args.cpu_budget / 4, threads=1)
         result["cpu_baseline"] = {"value": round(gbs, 4), "unit": UNIT, "cores": thr,
-                                  "kind": "oracle", "sample": desc}
+                                  "kind": "oracle", "sample": desc, "single_thread_value": round(gbs1, 4),
+                                  "cpu_model": cpu_model()}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def measure_config(name, gc, device, l2, hbm_peak, meas, barrier, args, rank, world):
+    """One page workload with the headline's fields (fewer calls): device time
+    in a CUDA graph, roofline, end-to-end GB/s through the public API with the
+    step's host copies, synchronous-API latency and the CPU oracle baseline
+    (all host cores and one)."""
+    import torch
+    wk = Workload(name)
+    r = DeviceRunner(wk, device, l2)
+    s = wk.shape
+    k = max(3, min(args.steps, 20))
+    ms, _, _ = time_graph(r, k, 3, barrier)
+    sec = ms / 1e3 / k
+    plan = gc.plan_name(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil, s.groups, wk.chain)
+    e2e_ms, h2d, d2h = time_e2e(r, k, 3, barrier)
+    out = {"label": s.label(), "kernel": plan, "us": round(sec * 1e6, 3),
+           "GB/s": round(wk.bytes / sec / 1e9, 1), "GFLOP/s": round(wk.flops / sec / 1e9, 1),
+           "roofline": roofline_for(wk, sec, plan, hbm_peak, meas),
+           "e2e": {"value": round(wk.bytes * k / (e2e_ms / 1e3) / 1e9, 2), "unit": UNIT,
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+           "sync_api_us": round(time_sync_api(r, k), 2)}
+    del r
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, desc, thr = cpu_oracle_rate(wk, max(1.0, args.cpu_budget / 4))
+        gbs1, _, _ = cpu_oracle_rate(wk, max(0.5, args.cpu_budget / 8), threads=1)
+        out["cpu_baseline"] = {"value": round(gbs, 4), "unit": UNIT, "cores": thr, "kind": "oracle",
+                               "sample": desc, "single_thread_value": round(gbs1, 4)}
+    return out
+
+
+def measure_sweep(gc, device, l2, hbm_peak, meas, barrier, k=20):
+    """The 80-shape sweep under graph timing (k calls per shape, rotating
+    buffers): per-shape time and roofline fraction, and their summary."""
+    import torch
+    per = []
+    for i in range(80):
+        wk = Workload(f"sweep{i}")
+        s = wk.shape
+        r = DeviceRunner(wk, device, l2)
+        ms, _, _ = time_graph(r, k, 3, barrier)
+        sec = ms / 1e3 / k
+        plan = gc.plan_name(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil, s.groups, False)
+        roof = roofline_for(wk, sec, plan, hbm_peak, meas)
+        per.append({"i": i, "us": round(sec * 1e6, 3), "MB": round(wk.bytes / 1e6, 2), "kernel": plan,
+                    "bound": roof["bound"], "frac": roof["frac"]})
+        del r
+        torch.cuda.empty_cache()
+
+    def gmean(v):
+        return round(math.exp(sum(math.log(x) for x in v) / len(v)), 4) if v else None
+    big = [p["frac"] for p in per if p["MB"] >= 50]
+    big_hbm = [p["frac"] for p in per if p["MB"] >= 50 and p["bound"] == "hbm"]
+    return {"calls_per_shape": k, "geomean_frac": gmean([p["frac"] for p in per]),
+            "geomean_frac_ge_50MB": gmean(big), "geomean_frac_ge_50MB_hbm_bound": gmean(big_hbm),
+            "n_ge_50MB": len(big), "n_ge_50MB_at_0.70": sum(1 for f in big if f >= 0.70),
+            "shapes": per}
 
 
 def run_profile_case(args, gc, device):

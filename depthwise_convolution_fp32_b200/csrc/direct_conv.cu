@@ -113,37 +113,72 @@ struct Window {
 // column cx*stride), ws at the plane's weight slice [r][s][channel] offset to
 // the thread's first channel.  The window (IR rows x NCH chunks) is read with
 // 128-bit shared loads; every input value feeds up to R*S*KT FMAs and every
-// weight load (KT channels) feeds RPT*4 FMAs.
+// weight feeds RPT*4 FMAs.
+// When the plane's weights fit in registers (R*S*KT <= 36) they are loaded
+// once and the input rows are streamed one at a time, each row feeding every
+// output row whose taps cover it; otherwise the whole window is held and the
+// weights are loaded tap by tap.
 template <int G, int KT, int RPT>
 __device__ __forceinline__ void fma_window(float (&acc)[RPT][kV][KT], const float *xs, const float *ws, int pitch,
                                            int KBtot) {
     using g = Geom<G>;
     using win = Window<G>;
     constexpr int IR = (RPT - 1) * g::ST + (g::R - 1) * g::D + 1;
-    float xr[IR][win::NCH * 4];
+    constexpr int RS = g::R * g::S;
+    if constexpr (RS * KT <= 36) {
+        float wr[RS][KT];
 #pragma unroll
-    for (int ir = 0; ir < IR; ++ir)
+        for (int t = 0; t < RS; ++t) load_weights<KT>(wr[t], ws + t * KBtot);
 #pragma unroll
-        for (int ch = 0; ch < win::NCH; ++ch) {
-            float4 v4 = *reinterpret_cast<const float4 *>(xs + ir * pitch + ch * 4);
-            xr[ir][4 * ch] = v4.x; xr[ir][4 * ch + 1] = v4.y;
-            xr[ir][4 * ch + 2] = v4.z; xr[ir][4 * ch + 3] = v4.w;
+        for (int ir = 0; ir < IR; ++ir) {
+            float xr[win::NCH * 4];
+#pragma unroll
+            for (int ch = 0; ch < win::NCH; ++ch) {
+                const float4 v4 = *reinterpret_cast<const float4 *>(xs + ir * pitch + ch * 4);
+                xr[4 * ch] = v4.x; xr[4 * ch + 1] = v4.y; xr[4 * ch + 2] = v4.z; xr[4 * ch + 3] = v4.w;
+            }
+#pragma unroll
+            for (int r = 0; r < g::R; ++r) {
+                // input row ir is tap row r of output row rp when rp*ST + r*D == ir
+                const int rem = ir - r * g::D;
+                if (rem < 0 || rem % g::ST != 0 || rem / g::ST >= RPT) continue;
+                const int rp = rem / g::ST;
+#pragma unroll
+                for (int s = 0; s < g::S; ++s)
+#pragma unroll
+                    for (int v = 0; v < kV; ++v) {
+                        const float xv = xr[win::OFF + v * g::ST + s * g::D];
+#pragma unroll
+                        for (int k = 0; k < KT; ++k) acc[rp][v][k] = fmaf(wr[r * g::S + s][k], xv, acc[rp][v][k]);
+                    }
+            }
         }
+    } else {
+        float xr[IR][win::NCH * 4];
 #pragma unroll
-    for (int r = 0; r < g::R; ++r)
+        for (int ir = 0; ir < IR; ++ir)
 #pragma unroll
-        for (int s = 0; s < g::S; ++s) {
-            float wv[KT];
-            load_weights<KT>(wv, ws + (r * g::S + s) * KBtot);
+            for (int ch = 0; ch < win::NCH; ++ch) {
+                float4 v4 = *reinterpret_cast<const float4 *>(xs + ir * pitch + ch * 4);
+                xr[ir][4 * ch] = v4.x; xr[ir][4 * ch + 1] = v4.y;
+                xr[ir][4 * ch + 2] = v4.z; xr[ir][4 * ch + 3] = v4.w;
+            }
 #pragma unroll
-            for (int rp = 0; rp < RPT; ++rp)
+        for (int r = 0; r < g::R; ++r)
 #pragma unroll
-                for (int v = 0; v < kV; ++v) {
-                    const float xv = xr[rp * g::ST + r * g::D][win::OFF + v * g::ST + s * g::D];
+            for (int s = 0; s < g::S; ++s) {
+                float wv[KT];
+                load_weights<KT>(wv, ws + (r * g::S + s) * KBtot);
 #pragma unroll
-                    for (int k = 0; k < KT; ++k) acc[rp][v][k] = fmaf(wv[k], xv, acc[rp][v][k]);
-                }
-        }
+                for (int rp = 0; rp < RPT; ++rp)
+#pragma unroll
+                    for (int v = 0; v < kV; ++v) {
+                        const float xv = xr[rp * g::ST + r * g::D][win::OFF + v * g::ST + s * g::D];
+#pragma unroll
+                        for (int k = 0; k < KT; ++k) acc[rp][v][k] = fmaf(wv[k], xv, acc[rp][v][k]);
+                    }
+            }
+    }
 }
 
 // Epilogue in registers for the thread's KT channels starting at kfirst:
@@ -181,21 +216,23 @@ __device__ __forceinline__ void epilogue_transform(float (&acc)[RPT][kV][KT], co
 template <int KT, int RPT>
 __device__ __forceinline__ void store_outputs(const float (&acc)[RPT][kV][KT], const DirectParams &p, int n,
                                               int kfirst, int prow, int qb) {
+    // one 64-bit base per thread, then per-channel / per-row increments
+    const long long plane = (long long)p.P * p.Q;
+    float *y0 = p.y + (((long long)n * p.K + kfirst) * p.P + prow) * (long long)p.Q + qb;
+    const bool vec = p.vec_out && qb + kV <= p.Q;
 #pragma unroll
-    for (int rp = 0; rp < RPT; ++rp) {
-        const int pp = prow + rp;
-        if (pp >= p.P) continue;
+    for (int k = 0; k < KT; ++k) {
+        float *yr = y0 + k * plane;
 #pragma unroll
-        for (int k = 0; k < KT; ++k) {
-            const int kk = kfirst + k;
-            float *yr = p.y + (((long long)n * p.K + kk) * p.P + pp) * (long long)p.Q;
-            if (p.vec_out && qb + kV <= p.Q) {
-                *reinterpret_cast<float4 *>(yr + qb) =
+        for (int rp = 0; rp < RPT; ++rp, yr += p.Q) {
+            if (prow + rp >= p.P) continue;
+            if (vec) {
+                *reinterpret_cast<float4 *>(yr) =
                     make_float4(acc[rp][0][k], acc[rp][1][k], acc[rp][2][k], acc[rp][3][k]);
             } else {
 #pragma unroll
                 for (int v = 0; v < kV; ++v)
-                    if (qb + v < p.Q) yr[qb + v] = acc[rp][v][k];
+                    if (qb + v < p.Q) yr[v] = acc[rp][v][k];
             }
         }
     }
@@ -502,7 +539,7 @@ __global__ void __launch_bounds__(256, 2)
 // raises the device error flag, stops the CTA's pipeline and, before the CTA
 // exits, waits (bounded again) for the copies it has in flight.
 template <int G, int KT, int RPT, int EPI>
-__global__ void __launch_bounds__(288, KT >= 8 ? 1 : 2)
+__global__ void __launch_bounds__(288, KT >= 8 ? 1 : (KT >= 4 ? 2 : 3))
     direct_stream_kernel(const __grid_constant__ TensorMap tm, const DirectParams p) {
     extern __shared__ __align__(128) float smem[];
     using g = Geom<G>;
@@ -511,13 +548,13 @@ __global__ void __launch_bounds__(288, KT >= 8 ? 1 : 2)
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);     // [8]
     uint64_t *empty = full + 8;                               // [8]
     int *flags = reinterpret_cast<int *>(full + 16);          // [0] abort, [1] items issued
+    int4 *item_hdr = reinterpret_cast<int4 *>(full + 18);     // [8] per stage: n, kc0, first row, first column
     float *stage0 = smem + kStreamHeaderBytes / 4;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int n_cwarps = (int)(blockDim.x >> 5) - 1;         // the last warp produces
     const int S = p.stages;
-    const int GY = p.n_kb * (p.groups / p.GB);
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
@@ -536,6 +573,7 @@ __global__ void __launch_bounds__(288, KT >= 8 ? 1 : 2)
         // ------------------------------------------------------------ producer
         const uint32_t x_bytes = (uint32_t)(p.GB * p.cpg) * (uint32_t)p.IHt * (uint32_t)p.pitch * 4u;
         const int nw = p.cpg * RS * p.KBtot;
+        const int GY = p.n_kb * (p.groups / p.GB);
         int j = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < p.n_items; it += gridDim.x, ++j) {
@@ -556,6 +594,8 @@ __global__ void __launch_bounds__(288, KT >= 8 ? 1 : 2)
             const int kc0 = g0 * p.kpg + (gy % p.n_kb) * p.KB;
             float *st = stage0 + (size_t)s * p.stage_floats;
             if (lane == 0) {
+                // the decoded item, published to the compute warps by the barrier's release
+                item_hdr[s] = make_int4(n, kc0, pt * p.TP, qt * p.TQ);
                 dev::mbar_arrive_expect_tx(&full[s], x_bytes);
                 dev::tma_load_3d(st, &tm, &full[s], qt * p.TQ * g::ST - 4 * win::HL, pt * p.TP * g::ST - g::PAD,
                                  n * p.C + g0 * p.cpg);
@@ -596,12 +636,7 @@ __global__ void __launch_bounds__(288, KT >= 8 ? 1 : 2)
                 atomicExch(&g_device_error, 1);
                 break;
             }
-            int u = it;
-            const int qt = u % p.n_qt; u /= p.n_qt;
-            const int pt = u % p.n_pt; u /= p.n_pt;
-            const int gy = u % GY;
-            const int n = u / GY;
-            const int kc0 = (gy / p.n_kb) * p.GB * p.kpg + (gy % p.n_kb) * p.KB;
+            const int4 hd = item_hdr[s];   // n, kc0, first output row, first output column
             const float *st = stage0 + (size_t)s * p.stage_floats;
             float acc[RPT][kV][KT];
 #pragma unroll
@@ -621,8 +656,8 @@ __global__ void __launch_bounds__(288, KT >= 8 ? 1 : 2)
             __syncwarp();
             if (lane == 0) dev::mbar_arrive(&empty[s]);
             if (active) {
-                epilogue_transform<KT, RPT, EPI>(acc, p, kc0 + kl0);
-                store_outputs<KT, RPT>(acc, p, n, kc0 + kl0, pt * p.TP + ry * RPT, qt * p.TQ + cx * kV);
+                epilogue_transform<KT, RPT, EPI>(acc, p, hd.y + kl0);
+                store_outputs<KT, RPT>(acc, p, hd.x, hd.y + kl0, hd.z + ry * RPT, hd.w + cx * kV);
             }
         }
     }

@@ -26,6 +26,8 @@ enum ForceMode : int {
     kForceBlocked = 5, kForceStream = 6
 };
 std::atomic<int> g_force{kForceAuto};
+std::atomic<int> g_force_kt{0};   // channels per thread forced for the direct kernels (0: planner's rule)
+
 
 // Convolution geometry.  stride, pad and dil are the H-axis values; sw, pw
 // and dw the W-axis ones (equal to them for the symmetric entry points).
@@ -62,6 +64,30 @@ gconv_status_t make_shape_ex(Shape &s, int N, int C, int H, int W, int K, int R,
 gconv_status_t make_shape(Shape &s, int N, int C, int H, int W, int K, int R, int S, int stride, int pad,
                           int dil, int groups) {
     return make_shape_ex(s, N, C, H, W, K, R, S, stride, stride, pad, pad, dil, dil, groups);
+}
+
+// Per-shape kernel choices measured on B200 (dispatch_table.json, compiled in
+// at build time): the fastest of the streaming direct kernel, the blocked
+// direct kernel and the implicit GEMM, with the direct kernels' channels per
+// thread, timed per shape; shapes not in the table follow the planner's rules.
+enum TableFamily : int { kTabStream = 1, kTabBlocked = 2, kTabIgemm = 3 };
+struct DispatchEntry {
+    int key[12];   // N, C, H, W, K, R, S, stride, pad, dilation, groups, chain
+    int family;
+    int kt;
+};
+const DispatchEntry kDispatchTable[] = {
+#include "gconv_dispatch_table.inc"
+    {{0}, 0, 0}   // end marker
+};
+
+// The measured choice for a shape with equal axes, or nullptr.
+const DispatchEntry *table_choice(const Shape &s, bool chain) {
+    if (!s.square()) return nullptr;
+    const int key[12] = {s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil, s.groups, chain ? 1 : 0};
+    for (const DispatchEntry *e = kDispatchTable; e->family; ++e)
+        if (!std::memcmp(e->key, key, sizeof(key))) return e;
+    return nullptr;
 }
 
 int match_geom(const Shape &s) {
@@ -140,7 +166,7 @@ int sm_count() {
 
 // Choose the CTA tile for a direct-kernel launch.  Returns false when no tile
 // fits the shared-memory limit (the shape is then unsupported by this family).
-bool plan_direct(const Shape &s, bool chain, int gn_groups, int geom, bool x_vec, DirectPlan &pl) {
+bool plan_direct(const Shape &s, bool chain, int gn_groups, int geom, bool x_vec, DirectPlan &pl, int kt_req = 0) {
     const bool fast = geom != kDirectGeneric;
     const int kgn = chain ? s.K / gn_groups : 1;
     DirectParams &p = pl.prm;
@@ -162,6 +188,7 @@ bool plan_direct(const Shape &s, bool chain, int gn_groups, int geom, bool x_vec
                 (long long)s.N * (s.K / c) * ceil_div(s.P, direct_rpt(c)) * ceil_div(s.Q, 4);
             if (threads >= want) break;
         }
+        if (kt_req > 0 && s.kpg % kt_req == 0 && (!chain || compat(kgn, kt_req))) KT = kt_req;
     }
     const int RPT = fast ? direct_rpt(KT) : direct_rpt(1);
     if (!fast) KT = 1;
@@ -314,7 +341,7 @@ bool plan_direct(const Shape &s, bool chain, int gn_groups, int geom, bool x_vec
 // A work item is a blocked-kernel tile; its input (GB*cpg planes x IHt rows x
 // 4*tpc columns, one TMA box) and its weight slice form one ring stage.
 // Returns false when the shape does not fit this variant.
-bool plan_stream(const Shape &s, int geom, bool x_vec, DirectPlan &pl) {
+bool plan_stream(const Shape &s, int geom, bool x_vec, DirectPlan &pl, int kt_req = 0) {
     if (geom == kDirectGeneric || !x_vec) return false;
     DirectParams &p = pl.prm;
     std::memset(&p, 0, sizeof(p));
@@ -326,6 +353,7 @@ bool plan_stream(const Shape &s, int geom, bool x_vec, DirectPlan &pl) {
         KT = c;
         if ((long long)s.N * (s.K / c) * ceil_div(s.P, direct_rpt(c)) * ceil_div(s.Q, 4) >= want) break;
     }
+    if (kt_req > 0 && s.kpg % kt_req == 0) KT = kt_req;
     const int RPT = direct_rpt(KT);
     const int nch = direct_fast_window_chunks(geom);
     const int qchunks = ceil_div(s.Q, 4);
@@ -387,7 +415,8 @@ bool plan_stream(const Shape &s, int geom, bool x_vec, DirectPlan &pl) {
     const size_t w_floats = ((size_t)s.cpg * s.R * s.S * KBtot + 31) / 32 * 32;
     const size_t stage_bytes = (x_floats + w_floats) * sizeof(float);
     if (stage_bytes > 96 * 1024) return false;
-    const int S = stage_bytes <= 24 * 1024 ? 4 : (stage_bytes <= 36 * 1024 ? 3 : 2);
+    // about 64 KB of stages per CTA, 2 to 4 deep, so that 3 CTAs fit an SM
+    const int S = (int)std::max<size_t>(2, std::min<size_t>(4, (64 * 1024) / stage_bytes));
 
     p.N = s.N; p.C = s.C; p.H = s.H; p.W = s.W; p.K = s.K; p.R = s.R; p.S = s.S;
     p.stride = s.stride; p.pad = s.pad; p.dil = s.dil; p.groups = s.groups;
@@ -412,17 +441,32 @@ bool plan_stream(const Shape &s, int geom, bool x_vec, DirectPlan &pl) {
     return true;
 }
 
-// Direct-kernel plan for the current forcing mode.
+// Direct-kernel plan for the current forcing mode: in automatic mode the
+// measured table decides streaming vs blocked and the channels per thread;
+// shapes outside it stream whenever the streaming kernel can take them.
 bool choose_direct(const Shape &s, bool chain, int gn_groups, bool x_vec, DirectPlan &pl) {
     const int force = g_force.load(std::memory_order_relaxed);
+    int kt = g_force_kt.load(std::memory_order_relaxed);
+    bool try_stream = !chain && force != kForceBlocked && force != kForceGeneric && force != kForceCpAsync;
+    if (force == kForceAuto) {
+        if (const DispatchEntry *e = table_choice(s, chain)) {
+            if (e->family == kTabBlocked) try_stream = false;
+            kt = e->kt;
+        }
+    }
+    const DispatchEntry *te = force == kForceAuto ? table_choice(s, chain) : nullptr;
     int geom = (force == kForceGeneric) ? (int)kDirectGeneric : match_geom(s);
     if (force == kForceCpAsync) x_vec = false;
-    if (!chain && force != kForceBlocked && force != kForceGeneric && force != kForceCpAsync &&
-        plan_stream(s, geom, x_vec, pl))
-        return true;
+    if (try_stream && plan_stream(s, geom, x_vec, pl, kt)) {
+        // outside the table, stream only where it measured faster: problems
+        // moving at least 24 MB with at most 4 channels per thread (small ones
+        // are latency-bound, where the blocked kernel's per-band waits win)
+        const double mb = 4.0 * ((double)s.N * s.C * s.H * s.W + (double)s.N * s.K * s.P * s.Q) / 1048576.0;
+        if (force != kForceAuto || te || (pl.KT <= 4 && mb >= 24.0)) return true;
+    }
     if (force == kForceStream) return false;
     pl.stream = 0;
-    if (plan_direct(s, chain, gn_groups, geom, x_vec, pl)) return true;
+    if (plan_direct(s, chain, gn_groups, geom, x_vec, pl, kt)) return true;
     if (geom != kDirectGeneric && force == kForceAuto)
         return plan_direct(s, chain, gn_groups, kDirectGeneric, x_vec, pl);
     return false;
@@ -434,7 +478,7 @@ bool choose_direct(const Shape &s, bool chain, int gn_groups, bool x_vec, Direct
 // driver).  Keys hold everything the cached value depends on.
 struct DirectKey {
     int v[14];
-    int x_vec, force, dev, sms;
+    int x_vec, force, force_kt, dev, sms;
     bool operator==(const DirectKey &o) const { return std::memcmp(this, &o, sizeof(*this)) == 0; }
 };
 
@@ -452,6 +496,7 @@ bool cached_direct_plan(const Shape &s, bool x_vec, DirectPlan &pl) {
     std::memcpy(k.v, vals, sizeof(vals));
     k.x_vec = x_vec ? 1 : 0;
     k.force = g_force.load(std::memory_order_relaxed);
+    k.force_kt = g_force_kt.load(std::memory_order_relaxed);
     if (cudaGetDevice(&k.dev) != cudaSuccess) return false;
     k.sms = sm_count();
     for (const Entry &e : cache)
@@ -694,7 +739,8 @@ bool use_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
         return false;
     if (!plan_igemm(s, chain, gn_groups, pl)) return false;
     if (force == kForceIgemm) return true;
-    // auto: enough reduction depth and output channels for the tensor cores to win
+    if (const DispatchEntry *e = table_choice(s, chain)) return e->family == kTabIgemm;
+    // outside the table: enough reduction depth and output channels for the tensor cores to win
     return s.cpg * s.R * s.S >= 64;
 }
 
@@ -755,16 +801,16 @@ gconv_status_t run_igemm(const Shape &s, IgemmPlan &pl, const float *x, const fl
     return GCONV_OK;
 }
 
-// Images per chunk of the fused chain on the implicit-GEMM path: the chunk's
-// conv output and split operands take about half of the L2 cache, so the
-// normalize pass reads the conv output back from L2 and y goes out to HBM
-// once (plus the chunk's own split operands, which the next chunk overwrites
-// in place).  Returns N when the whole batch already fits.
+// Images per chunk of the fused chain on the implicit-GEMM path.  With a
+// budget set (GCONV_CHAIN_L2_MB), each chunk's conv output and split operands
+// take about that much of the L2 cache, so the normalize pass could read the
+// conv output back from L2.  Measured on B200 this loses to one pass over the
+// whole batch at every budget tried (24-112 MB: 1.0-1.6 ms against 0.91 ms;
+// per-chunk GEMM ramp and tail, statistics merge and launch costs outweigh
+// the saved HBM traffic), so by default the whole batch is one chunk.
 int chain_chunk_images(const Shape &s, const IgemmPlan &pl) {
-    static const int budget_mb = [] {
-        const int v = env_int("GCONV_CHAIN_L2_MB");
-        return v > 0 ? v : 56;
-    }();
+    static const int budget_mb = env_int("GCONV_CHAIN_L2_MB");
+    if (budget_mb <= 0) return s.N;
     const double per_img = 4.0 * s.K * s.P * s.Q + 8.0 * s.C * pl.prm.Hp * (double)pl.prm.Wp;
     const long long B = (long long)(budget_mb * 1048576.0 / per_img);
     return (int)std::max<long long>(1, std::min<long long>(B, s.N));
@@ -908,14 +954,33 @@ gconv_status_t gconv2d_output_size(int H, int W, int R, int S, int stride, int p
 
 gconv_status_t gconv_force_kernel(const char *name) {
     if (!name) return GCONV_ERR_INVALID_ARG;
-    if (!std::strcmp(name, "auto")) g_force = kForceAuto;
-    else if (!std::strcmp(name, "direct")) g_force = kForceDirect;
-    else if (!std::strcmp(name, "generic")) g_force = kForceGeneric;
-    else if (!std::strcmp(name, "direct_cpasync")) g_force = kForceCpAsync;
-    else if (!std::strcmp(name, "igemm")) g_force = kForceIgemm;
-    else if (!std::strcmp(name, "direct_blocked")) g_force = kForceBlocked;
-    else if (!std::strcmp(name, "direct_stream")) g_force = kForceStream;
+    // optional ":ktN" suffix: channels per thread of the direct kernels
+    char fam[32];
+    int kt = 0;
+    const char *colon = std::strchr(name, ':');
+    const size_t n = colon ? (size_t)(colon - name) : std::strlen(name);
+    if (n >= sizeof(fam)) return GCONV_ERR_INVALID_ARG;
+    std::memcpy(fam, name, n);
+    fam[n] = 0;
+    if (colon) {
+        if (std::strcmp(colon + 1, "kt1") == 0) kt = 1;
+        else if (std::strcmp(colon + 1, "kt2") == 0) kt = 2;
+        else if (std::strcmp(colon + 1, "kt4") == 0) kt = 4;
+        else if (std::strcmp(colon + 1, "kt8") == 0) kt = 8;
+        else return GCONV_ERR_INVALID_ARG;
+    }
+    int mode;
+    if (!std::strcmp(fam, "auto")) mode = kForceAuto;
+    else if (!std::strcmp(fam, "direct")) mode = kForceDirect;
+    else if (!std::strcmp(fam, "generic")) mode = kForceGeneric;
+    else if (!std::strcmp(fam, "direct_cpasync")) mode = kForceCpAsync;
+    else if (!std::strcmp(fam, "igemm")) mode = kForceIgemm;
+    else if (!std::strcmp(fam, "direct_blocked")) mode = kForceBlocked;
+    else if (!std::strcmp(fam, "direct_stream")) mode = kForceStream;
     else return GCONV_ERR_INVALID_ARG;
+    if (kt && (mode == kForceAuto || mode == kForceIgemm)) return GCONV_ERR_INVALID_ARG;
+    g_force = mode;
+    g_force_kt = kt;
     return GCONV_OK;
 }
 

@@ -107,7 +107,10 @@ cudaError_t launch_direct(const DirectParams &p, const TensorMap &tm, int geom, 
 // being queried once per variant, block size, shared memory and device.
 cudaError_t launch_direct_stream(const DirectParams &p, const TensorMap &tm, int geom, int KT, int sms,
                                  int threads, size_t smem, cudaStream_t stream);
-constexpr int kStreamHeaderBytes = 256;   // barriers + bookkeeping ahead of the stages
+// Shared memory ahead of the stages: full[8] and empty[8] barriers (128 B), two
+// flags (8 B), then 8 per-stage item records (int4 at byte 144); stages start
+// 128-byte aligned after it.
+constexpr int kStreamHeaderBytes = 512;
 
 // Device error flag raised by bounded waits that gave up (0 = none); reading
 // clears it.  Synchronises with the device.

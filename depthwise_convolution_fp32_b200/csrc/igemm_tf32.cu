@@ -165,18 +165,19 @@ __device__ __forceinline__ float rcp_ftz(float x) {
     return y;
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(dev::smem_addr(bar)) : "memory");
-}
-
 // Output tile t -> (n, g, row tile, column tile); column tiles vary fastest so
-// CTAs running side by side share input rows in L2.
+// CTAs running side by side share input rows in L2.  Tiles are taken from the
+// last image backwards: the split pass that runs just before writes the images
+// forwards, so the GEMM starts on the split operands still in L2, and the
+// images it finishes last (the first ones) are where a following pass over
+// the output starts.
 struct IgTile {
     int n, g, p0, q0, sp;
 };
 
 __device__ __forceinline__ IgTile ig_tile(const IgemmParams &p, int t) {
     IgTile r;
+    t = p.n_tiles - 1 - t;
     const int nsp = p.n_qt * p.n_pt;
     r.sp = t % nsp;
     const int rest = t / nsp;
@@ -447,12 +448,15 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
             const int q = tl.q0 + m;
             const bool qvalid = q < p.Q;
             const int rows = ok ? min(p.TH, p.P - tl.p0) : 0;   // valid output rows of the tile
-            float *ybase = p.y + ((long long)tl.n * p.K + (long long)tl.g * p.kpg) * plane + q;
+            // this thread's output column of row tl.p0, channel tl.g*kpg of image tl.n
+            float *ybase = p.y + ((long long)tl.n * p.K + (long long)tl.g * p.kpg) * plane +
+                           (long long)tl.p0 * p.Q + q;
             const uint32_t tbase = tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)buf * acc_cols;
 #pragma unroll 1
             for (int c0 = cpart * PART; c0 < (cpart + 1) * PART; c0 += CW) {
-                // plain: a = acc + bias.  chain: t = -(acc*scale + bias*scale)*log2(e)
-                // (so that the logistic is 1 / (1 + 2^t)) as acc*mul + add
+                // plain: a = acc * mul + add.  chain: t = -(acc*scale + bias*scale)*log2(e)
+                // = acc * mul + add, and the logistic is 1 / (1 + 2^t): 2^t overflows
+                // to +inf for very negative arguments, and 1 / inf is exactly the limit 0
                 float mul[CW], add[CW];
 #pragma unroll
                 for (int jj = 0; jj < CW; ++jj) {
@@ -470,6 +474,8 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
                 float shift[GPC], s1[GPC], s2[GPC];
 #pragma unroll
                 for (int gg = 0; gg < GPC; ++gg) { shift[gg] = 0.f; s1[gg] = 0.f; s2[gg] = 0.f; }
+                // output pointer of channel c0 in the current row; channels are `plane` apart
+                float *yc = ybase + (long long)c0 * plane;
                 // rows are processed two at a time so one TMEM load latency covers both
 #pragma unroll 1
                 for (int i = 0; i < p.TH; i += 2) {
@@ -484,11 +490,7 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
                         const bool rvalid = i + h < rows;            // warp-uniform
                         if constexpr (CHAIN) {
 #pragma unroll
-                            for (int jj = 0; jj < CW; ++jj) {
-                                // 2^t overflows past 128: clamp keeps 1 + 2^t finite
-                                const float e = ex2_ftz(fminf(fmaf(v[jj], mul[jj], add[jj]), 126.f));
-                                v[jj] = rcp_ftz(1.f + e);
-                            }
+                            for (int jj = 0; jj < CW; ++jj) v[jj] = rcp_ftz(1.f + ex2_ftz(fmaf(v[jj], mul[jj], add[jj])));
                             if (rvalid && i + h == 0) {
 #pragma unroll
                                 for (int gg = 0; gg < GPC; ++gg) shift[gg] = __shfl_sync(0xffffffffu, v[gg * GW], 0);
@@ -502,9 +504,9 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
                             }
                         }
                         if (rvalid && qvalid) {
-                            float *yr = ybase + (long long)c0 * plane + (long long)(tl.p0 + i + h) * p.Q;
+                            float *yr = yc;
 #pragma unroll
-                            for (int jj = 0; jj < CW; ++jj) yr[(long long)jj * plane] = v[jj];
+                            for (int jj = 0; jj < CW; ++jj, yr += plane) *yr = v[jj];
                             if constexpr (CHAIN) {
 #pragma unroll
                                 for (int jj = 0; jj < CW; ++jj) {
@@ -514,17 +516,22 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
                                 }
                             }
                         }
+                        yc += p.Q;
                     }
                 }
                 if (c0 + CW >= (cpart + 1) * PART) {
                     // last TMEM read of this tile by this warp: hand the buffer back
                     dev::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&acce[buf]);
+                    if (lane == 0) dev::mbar_arrive(&acce[buf]);
                 }
                 if constexpr (CHAIN) {
                     const unsigned vmask = __ballot_sync(0xffffffffu, qvalid);
-                    const double cnt = (double)(__popc(vmask) * rows * GW);
+                    const int cnt_i = __popc(vmask) * rows * GW;
+                    // 1/count: FP32 reciprocal refined by one Newton step in FP64 (count < 2^24)
+                    const double cnt = (double)cnt_i;
+                    double inv = (double)__frcp_rn((float)cnt_i);
+                    inv = inv * (2.0 - cnt * inv);
 #pragma unroll
                     for (int gg = 0; gg < GPC; ++gg) {
                         double S1 = (double)s1[gg], S2 = (double)s2[gg];
@@ -537,10 +544,10 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
                             const int k0 = tl.g * p.kpg + c0 + gg * GW;   // first channel of the fragment
                             const int G = k0 / p.kgn;
                             const int fr = fpg > 1 ? (k0 % p.kgn) / CW : 0;
-                            const double mean = cnt > 0.0 ? (double)shift[gg] + S1 / cnt : 0.0;
-                            const double m2 = cnt > 0.0 ? fmax(S2 - S1 * S1 / cnt, 0.0) : 0.0;
+                            const double mean = cnt_i > 0 ? (double)shift[gg] + S1 * inv : 0.0;
+                            const double m2 = cnt_i > 0 ? fmax(S2 - S1 * S1 * inv, 0.0) : 0.0;
                             p.gn_part[((long long)tl.n * p.gn_groups + G) * p.slots + (tl.sp * 4 + lq) * fpg + fr] =
-                                make_float4((float)cnt, (float)mean, (float)m2, 0.f);
+                                make_float4((float)cnt_i, (float)mean, (float)m2, 0.f);
                         }
                     }
                 }

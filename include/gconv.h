@@ -203,10 +203,15 @@ GCONV_API const char *gconv2d_plan_name_ex(int N, int C, int H, int W, int K, in
                               int stride_h, int stride_w, int pad_h, int pad_w, int dil_h, int dil_w,
                               int groups);
 
-/* Force a kernel family for subsequent calls on this process, by name
- * ("auto" restores per-shape dispatch).  A forced family that cannot run a
- * shape makes that call return GCONV_ERR_UNSUPPORTED.  Returns
- * GCONV_ERR_INVALID_ARG for an unknown name.  Intended for measurement. */
+/* Force a kernel family for subsequent calls on this process, by name:
+ * "direct_stream", "direct_blocked", "direct" (streaming when possible, else
+ * blocked), "direct_cpasync" (blocked, cp.async staging), "generic",
+ * "igemm"; a ":kt1" / ":kt2" / ":kt4" / ":kt8" suffix also fixes the direct
+ * kernels' output channels per thread.  "auto" restores per-shape dispatch
+ * (the measured table compiled into the library, then the planner's rules).
+ * A forced family that cannot run a shape makes that call return
+ * GCONV_ERR_UNSUPPORTED.  Returns GCONV_ERR_INVALID_ARG for an unknown name.
+ * Intended for measurement (A/B runs, regenerating the table). */
 GCONV_API gconv_status_t gconv_force_kernel(const char *name);
 
 /* Status of the bounded waits inside the kernels since the last query:

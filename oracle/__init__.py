@@ -63,6 +63,8 @@ def _load():
                                      + [l, p, p, p, p, p, p])
         lib.oracle_num_threads.restype = i
         lib.oracle_num_threads.argtypes = []
+        lib.oracle_set_num_threads.restype = None
+        lib.oracle_set_num_threads.argtypes = [i]
         _lib = lib
         return lib
 
@@ -199,3 +201,8 @@ def conv2d_affine_clamp(x, w, scale=None, shift=None, lo=-np.inf, hi=np.inf, str
 def num_threads() -> int:
     """OpenMP threads the oracle runs with."""
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """OpenMP threads for later calls (timing only; results do not depend on it)."""
+    _load().oracle_set_num_threads(int(n))

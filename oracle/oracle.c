@@ -256,3 +256,16 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* Threads for later calls (the benchmark times the oracle on all host cores
+ * and on one); n < 1 leaves the setting unchanged.  Results do not depend on
+ * it: threads only split independent outputs. */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

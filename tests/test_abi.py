@@ -100,10 +100,29 @@ def test_chain_rejects_invalid_arguments(lib):
     assert call(gamma=FAKE + 2) == gc.ERR_INVALID_ARG
 
 
+def _table_family(shape, chain=0):
+    """The family the compiled-in measured table picks for a shape, or None."""
+    import json
+    path = os.path.join(ROOT, "depthwise_convolution_fp32_b200", "dispatch_table.json")
+    if not os.path.exists(path):
+        return None
+    for e in json.load(open(path))["entries"]:
+        if e["shape"] == list(shape) and e.get("chain", 0) == chain:
+            return e["best"].split(":")[0]
+    return None
+
+
 def test_plan_names(lib):
-    assert gc.plan_name(4, 144, 56, 56, 144, 3, 3, 1, 1, 1, 144) == "direct_stream_3x3s1p1"
+    # the headline depthwise workload: the measured table's choice, else (14 MB, latency-bound) blocked
+    fam = _table_family((4, 144, 56, 56, 144, 3, 3, 1, 1, 1, 144))
+    want = "direct_stream_3x3s1p1" if fam == "direct_stream" else "direct_tma_3x3s1p1"
+    assert gc.plan_name(4, 144, 56, 56, 144, 3, 3, 1, 1, 1, 144) == want
+    # outside the table: an 822 MB depthwise problem streams
+    assert gc.plan_name(32, 256, 112, 112, 256, 3, 3, 1, 1, 1, 256, 0) in (
+        "direct_stream_3x3s1p1" if _table_family((32, 256, 112, 112, 256, 3, 3, 1, 1, 1, 256)) in
+        (None, "direct_stream") else "direct_tma_3x3s1p1",)
     assert gc.plan_name(2, 16, 14, 14, 16, 3, 3, 1, 1, 1, 16) == "direct_3x3s1p1"   # rows not 16-byte multiples
-    assert gc.plan_name(1, 8, 29, 32, 8, 3, 3, 2, 1, 1, 8) == "direct_stream_3x3s2p1"
+    assert gc.plan_name(16, 64, 128, 128, 64, 3, 3, 2, 1, 1, 64) == "direct_stream_3x3s2p1"
     # the fused chain's conv stage never streams (its epilogue reduces statistics per CTA)
     assert not gc.plan_name(2, 16, 30, 32, 16, 3, 3, 1, 1, 1, 16, chain=True).startswith("direct_stream")
     assert gc.plan_name(1, 8, 16, 16, 8, 3, 3, 1, 1, 2, 4) == "direct_generic"
