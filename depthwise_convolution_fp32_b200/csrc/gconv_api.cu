@@ -23,7 +23,7 @@ constexpr int kBarFloats = 32;               // shared memory reserved for mbarr
 
 enum ForceMode : int {
     kForceAuto = 0, kForceDirect = 1, kForceGeneric = 2, kForceCpAsync = 3, kForceIgemm = 4,
-    kForceBlocked = 5, kForceStream = 6
+    kForceBlocked = 5, kForceStream = 6, kForceIgemmSplit = 7, kForceIgemmFused = 8
 };
 std::atomic<int> g_force{kForceAuto};
 std::atomic<int> g_force_kt{0};   // channels per thread forced for the direct kernels (0: planner's rule)
@@ -649,10 +649,38 @@ int env_int(const char *name) {
     return e ? std::atoi(e) : 0;
 }
 
+// Chain design on the implicit-GEMM path (GCONV_CHAIN_DESIGN=store|recompute
+// overrides): recompute runs the GEMM twice and never writes the logistic
+// output; store writes it and normalizes it in a streaming pass.
+bool chain_recompute(const Shape &s) {
+    static const int mode = [] {
+        const char *e = std::getenv("GCONV_CHAIN_DESIGN");
+        if (e && !std::strcmp(e, "store")) return 0;
+        if (e && !std::strcmp(e, "recompute")) return 1;
+        return -1;
+    }();
+    if (mode >= 0) return mode == 1;
+    return true;
+}
+
+// Whether the implicit GEMM stages x raw and converts it in shared memory
+// (GCONV_IGEMM_FUSED=0/1 overrides): on by default where the fused variant fits.
+bool igemm_fused_wanted() {
+    static const int v = [] {
+        const char *e = std::getenv("GCONV_IGEMM_FUSED");
+        return e ? std::atoi(e) : -1;
+    }();
+    return v != 0;
+}
+
 // Stride-1 convolutions whose groups hold a multiple of 8 input channels and
 // 32/64/128/256 output channels run as an implicit GEMM on the tensor cores.
-bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
+// Implicit-GEMM plan.  fused: x is staged raw by TMA and converted in shared
+// memory (N = 32 only, rows 16-byte multiples), so no split pass and no x
+// workspace; otherwise the split pass writes the padded operand tensors.
+bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl, bool fused = false) {
     if (s.stride != 1 || s.sw != 1 || s.cpg % 8 != 0 || !igemm_supported_nt(s.kpg)) return false;
+    if (fused && (s.kpg != 32 || s.W % 4 != 0)) return false;
     const int kgn = chain ? s.K / gn_groups : 1;
     // chain epilogue: groups nest inside a conv group, widths 1..16 or multiples of 16
     if (chain && (s.kpg > 64 || s.kpg % kgn != 0 || (kgn > 16 && kgn % 16 != 0))) return false;
@@ -671,22 +699,31 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     // output rows per tile: two accumulator buffers of TH*NT columns fit TMEM
     int TH = std::max(1, std::min(8, 256 / NT));
     if (force_th > 0) TH = force_th;
+    if (fused) TH = igemm_fused_th();   // the fused issue loop is compiled for it
+    if (TH > s.P && fused) return false;
     TH = std::min(TH, s.P);
     const size_t limit = 227 * 1024 - igemm_header_bytes(NT, chain);
     const int b_bytes = 32 * s.S * NT;              // one w operand slice: S taps x 8 channels x NT
-    int AR = 0, a_bytes = 0, sa = 0, sb = 0;
+    const int COLSR = COLS + 4;                     // fused raw box: room to round the start down to 4
+    int AR = 0, a_bytes = 0, sa = 0, sb = 0, raw_bytes = 0;
     for (; TH >= 1; --TH) {
         AR = TH + (s.R - 1) * s.dil;               // staged rows serving every tap row
         if (AR > 256) continue;
         a_bytes = 32 * COLS * AR;                   // one x operand tile: 2 quads x AR x COLS x 16 B
+        raw_bytes = fused ? 8 * AR * COLSR * 4 : 0;
+        const size_t lim = limit - (size_t)raw_bytes;
         sa = force_sa > 0 ? std::min(force_sa, 4) : 2;
         sb = force_sb > 0 ? std::min(force_sb, 4) : 4;
-        while (sb > 2 && (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes > limit) --sb;
-        while (sa > 1 && (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes > limit) --sa;
-        while (sb > 1 && (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes > limit) --sb;
-        if ((size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes <= limit) break;
+        // weights resident when every slice fits (they are then loaded once per CTA)
+        if (fused && s.cpg / 8 * s.R <= 4) sb = std::max(sb, s.cpg / 8 * s.R);
+        while (sb > 2 && (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes > lim) --sb;
+        while (sa > 1 && (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes > lim) --sa;
+        while (sb > 1 && (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes > lim) --sb;
+        if ((size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes <= lim && (!fused || sa == 2)) break;
+        if (fused) return false;
     }
     if (TH < 1) return false;
+    if (fused && (COLSR > 256 || raw_bytes <= 0)) return false;
     int tmem_cols = 32;
     while (tmem_cols < 2 * TH * NT) tmem_cols *= 2;
     if (tmem_cols > 512) return false;
@@ -716,10 +753,14 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     p.gn_groups = chain ? gn_groups : 0;
     p.kgn = kgn;
     p.slots = p.n_qt * p.n_pt * (chain ? igemm_partials_per_tile(NT, kgn) : 1);
+    p.fused = fused ? 1 : 0;
+    p.COLSR = fused ? COLSR : 0;
+    p.raw_bytes = raw_bytes;
+    p.rr = fused ? 1 : 0;
     pl.grid = dim3((unsigned)std::min<long long>(n_tiles, sm_count()));
-    pl.smem = igemm_header_bytes(NT, chain) + (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes;
+    pl.smem = igemm_header_bytes(NT, chain) + (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes + raw_bytes;
 
-    const size_t xbytes = (size_t)s.N * s.C * (size_t)Hp * (size_t)Wp * sizeof(float);
+    const size_t xbytes = fused ? 0 : (size_t)s.N * s.C * (size_t)Hp * (size_t)Wp * sizeof(float);
     const size_t wbytes = (size_t)s.K * s.cpg * s.R * s.S * sizeof(float);
     pl.off_xl = align256(xbytes);
     pl.off_wh = pl.off_xl + align256(xbytes);
@@ -731,13 +772,29 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     return true;
 }
 
+bool force_is_igemm() {
+    const int f = g_force.load(std::memory_order_relaxed);
+    return f == kForceIgemm || f == kForceIgemmSplit || f == kForceIgemmFused;
+}
+
+// A fused plan stages x by TMA, which needs x 16-byte aligned: otherwise
+// re-plan the split variant (returns false when that does not fit either).
+bool igemm_plan_for_pointer(const Shape &s, bool chain, int gn_groups, const float *x, IgemmPlan &pl) {
+    if (!pl.prm.fused || aligned16(x)) return true;
+    if (g_force.load(std::memory_order_relaxed) == kForceIgemmFused) return false;
+    return plan_igemm(s, chain, gn_groups, pl, false);
+}
+
 // Whether the dispatcher sends a shape to the implicit GEMM.
 bool use_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     const int force = g_force.load(std::memory_order_relaxed);
     if (force == kForceDirect || force == kForceGeneric || force == kForceCpAsync || force == kForceBlocked ||
         force == kForceStream)
         return false;
-    if (!plan_igemm(s, chain, gn_groups, pl)) return false;
+    if (force == kForceIgemmFused) return plan_igemm(s, chain, gn_groups, pl, true);
+    if (force == kForceIgemmSplit) return plan_igemm(s, chain, gn_groups, pl, false);
+    if (!(igemm_fused_wanted() && plan_igemm(s, chain, gn_groups, pl, true)) && !plan_igemm(s, chain, gn_groups, pl))
+        return false;
     if (force == kForceIgemm) return true;
     if (const DispatchEntry *e = table_choice(s, chain)) return e->family == kTabIgemm;
     // outside the table: enough reduction depth and output channels for the tensor cores to win
@@ -746,10 +803,16 @@ bool use_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
 
 // Launch the split passes and the GEMM; chain additionally runs the GroupNorm
 // finalize and normalize passes.
-// Tensor maps over the split x operands in the workspace (x_hi, cross terms).
-bool igemm_maps(const Shape &s, const IgemmPlan &pl, void *ws, TensorMap *tm) {
+// Tensor maps over the split x operands in the workspace (x_hi, cross terms);
+// for the fused variant a map over x itself ([N*C][H][W], box COLSR x AR x 8).
+bool igemm_maps(const Shape &s, const IgemmPlan &pl, void *ws, TensorMap *tm, const float *x = nullptr) {
     char *base = reinterpret_cast<char *>(ws);
     const IgemmParams &p = pl.prm;
+    if (p.fused) {
+        std::memset(&tm[1], 0, sizeof(tm[1]));
+        return x && aligned16(x) &&
+               cached_x_tensor_map(&tm[0], x, (long long)s.N * s.C, s.H, s.W, p.COLSR, p.AR, 8);
+    }
     const long long quads = (long long)s.N * (s.C / 4);
     return make_nc4hw4_tile_map(&tm[0], reinterpret_cast<float *>(base), quads, p.Hp, p.Wp, p.COLS, p.AR) &&
            make_nc4hw4_tile_map(&tm[1], reinterpret_cast<float *>(base + pl.off_xl), quads, p.Hp, p.Wp, p.COLS,
@@ -769,7 +832,7 @@ gconv_status_t run_igemm(const Shape &s, IgemmPlan &pl, const float *x, const fl
     TensorMap own[2];
     const TensorMap *tm = maps;
     if (!tm) {
-        if (!igemm_maps(s, pl, ws, own)) return GCONV_ERR_UNSUPPORTED;
+        if (!igemm_maps(s, pl, ws, own, x)) return GCONV_ERR_UNSUPPORTED;
         tm = own;
     }
     p.wh = reinterpret_cast<const float4 *>(wh);
@@ -779,10 +842,16 @@ gconv_status_t run_igemm(const Shape &s, IgemmPlan &pl, const float *x, const fl
     p.y = y;
     const bool chain = gn_groups > 0;
     p.gn_part = chain ? reinterpret_cast<float4 *>(base + pl.off_part) : nullptr;
-    if (launch_split_x(x, xh, xl, s.N, s.C, s.H, s.W, s.pad, s.pw, p.Hp, p.Wp, stream) != cudaSuccess)
+    if (!p.fused && launch_split_x(x, xh, xl, s.N, s.C, s.H, s.W, s.pad, s.pw, p.Hp, p.Wp, stream) != cudaSuccess)
         return GCONV_ERR_CUDA;
     if (split_w && launch_split_w(w, wh, wl, s.K, s.cpg, s.R, s.S, s.groups, stream) != cudaSuccess)
         return GCONV_ERR_CUDA;
+    // the chain either stores the logistic output and normalizes it in a
+    // streaming pass (store), or runs the GEMM twice: statistics only, then the
+    // normalized result straight from the accumulators (recompute; y is written
+    // once and the logistic output never reaches memory)
+    const bool recompute = chain && chain_recompute(s);
+    p.chain_mode = recompute ? 1 : 0;
     if (launch_igemm(p, tm, chain ? 1 : 0, pl.grid, pl.smem, stream) != cudaSuccess) return GCONV_ERR_CUDA;
     if (!chain) return GCONV_OK;
     GnParams g;
@@ -797,6 +866,13 @@ gconv_status_t run_igemm(const Shape &s, IgemmPlan &pl, const float *x, const fl
     const long long per_cta = g.vec ? 4LL * 256 * 8 : 256LL * 8;
     g.chunks = (int)std::max<long long>(1, (g.PQ + per_cta - 1) / per_cta);
     if (launch_gn_finalize(g, stream) != cudaSuccess) return GCONV_ERR_CUDA;
+    if (recompute) {
+        p.chain_mode = 2;
+        p.gn_stats = g.stats;
+        p.gamma = gamma;
+        p.beta = beta;
+        return launch_igemm(p, tm, 1, pl.grid, pl.smem, stream) == cudaSuccess ? GCONV_OK : GCONV_ERR_CUDA;
+    }
     if (launch_gn_normalize(g, stream) != cudaSuccess) return GCONV_ERR_CUDA;
     return GCONV_OK;
 }
@@ -825,27 +901,28 @@ gconv_status_t run_chain_igemm(const Shape &s, const IgemmPlan &full, const floa
     const int B = chain_chunk_images(s, full);
     Shape sc = s;
     sc.N = B;
+    const bool fused = full.prm.fused != 0;
     IgemmPlan first;
     if (B == s.N) first = full;
-    else if (!plan_igemm(sc, true, gn_groups, first)) return GCONV_ERR_UNSUPPORTED;
+    else if (!plan_igemm(sc, true, gn_groups, first, fused)) return GCONV_ERR_UNSUPPORTED;
     void *ws = nullptr;
     gconv_status_t st = ensure_workspace(first.ws_bytes, stream, &ws);
     if (st != GCONV_OK) return st;
-    TensorMap maps[2];
-    if (!igemm_maps(sc, first, ws, maps)) return GCONV_ERR_UNSUPPORTED;
+    TensorMap maps[2];   // split variant: maps over the workspace, the same for every chunk
+    if (!fused && !igemm_maps(sc, first, ws, maps)) return GCONV_ERR_UNSUPPORTED;
     const long long x_img = (long long)s.C * s.H * s.W, y_img = (long long)s.K * s.P * s.Q;
     for (int n0 = 0; n0 < s.N; n0 += B) {
         const int nb = std::min(B, s.N - n0);
         if (nb == B) {
             IgemmPlan cur = first;
             st = run_igemm(sc, cur, x + n0 * x_img, w, bias, scale, gn_groups, gamma, beta, eps, y + n0 * y_img, ws,
-                           stream, maps, n0 == 0);
+                           stream, fused ? nullptr : maps, n0 == 0);
         } else {
             // a shorter last chunk: its own plan (workspace offsets and maps follow N)
             Shape sl = s;
             sl.N = nb;
             IgemmPlan cur;
-            if (!plan_igemm(sl, true, gn_groups, cur)) return GCONV_ERR_UNSUPPORTED;
+            if (!plan_igemm(sl, true, gn_groups, cur, fused)) return GCONV_ERR_UNSUPPORTED;
             st = run_igemm(sl, cur, x + n0 * x_img, w, bias, scale, gn_groups, gamma, beta, eps, y + n0 * y_img, ws,
                            stream);
         }
@@ -869,7 +946,7 @@ gconv_status_t conv_fwd_shape(const Shape &s, const float *x, const float *w, co
     if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) return GCONV_ERR_INVALID_ARG;
     if (aff_scale && (reinterpret_cast<uintptr_t>(aff_scale) & 3u)) return GCONV_ERR_INVALID_ARG;
     IgemmPlan ig;
-    if (use_igemm(s, false, 1, ig)) {
+    if (use_igemm(s, false, 1, ig) && igemm_plan_for_pointer(s, false, 1, x, ig)) {
         void *ws = nullptr;
         if ((st = ensure_workspace(ig.ws_bytes, stream, &ws)) != GCONV_OK) return st;
         ig.prm.aff_scale = aff_scale;
@@ -878,7 +955,7 @@ gconv_status_t conv_fwd_shape(const Shape &s, const float *x, const float *w, co
         ig.prm.hi = hi;
         return run_igemm(s, ig, x, w, bias, nullptr, 0, nullptr, nullptr, 0.f, y, ws, stream);
     }
-    if (g_force.load(std::memory_order_relaxed) == kForceIgemm) return GCONV_ERR_UNSUPPORTED;
+    if (force_is_igemm()) return GCONV_ERR_UNSUPPORTED;
     DirectPlan pl;
     const bool x_vec = (s.W % 4 == 0) && aligned16(x);
     if (!cached_direct_plan(s, x_vec, pl)) return GCONV_ERR_UNSUPPORTED;
@@ -977,8 +1054,11 @@ gconv_status_t gconv_force_kernel(const char *name) {
     else if (!std::strcmp(fam, "igemm")) mode = kForceIgemm;
     else if (!std::strcmp(fam, "direct_blocked")) mode = kForceBlocked;
     else if (!std::strcmp(fam, "direct_stream")) mode = kForceStream;
+    else if (!std::strcmp(fam, "igemm_split")) mode = kForceIgemmSplit;
+    else if (!std::strcmp(fam, "igemm_fused")) mode = kForceIgemmFused;
     else return GCONV_ERR_INVALID_ARG;
-    if (kt && (mode == kForceAuto || mode == kForceIgemm)) return GCONV_ERR_INVALID_ARG;
+    if (kt && (mode == kForceAuto || mode == kForceIgemm || mode == kForceIgemmSplit || mode == kForceIgemmFused))
+        return GCONV_ERR_INVALID_ARG;
     g_force = mode;
     g_force_kt = kt;
     return GCONV_OK;
@@ -991,7 +1071,7 @@ const char *gconv2d_plan_name(int N, int C, int H, int W, int K, int R, int S, i
     if (st == GCONV_ERR_INVALID_ARG) return "invalid";
     if (st != GCONV_OK) return "unsupported";
     IgemmPlan ig;
-    if (use_igemm(s, chain != 0, chain ? s.K : 1, ig)) return "igemm_tf32_bf16x";
+    if (use_igemm(s, chain != 0, chain ? s.K : 1, ig)) return ig.prm.fused ? "igemm_tf32_bf16x_fused" : "igemm_tf32_bf16x";
     DirectPlan pl;
     int gn = 1;
     if (!choose_direct(s, chain != 0, gn, s.W % 4 == 0, pl)) return "unsupported";
@@ -1023,7 +1103,7 @@ const char *gconv2d_plan_name_ex(int N, int C, int H, int W, int K, int R, int S
     if (st == GCONV_ERR_INVALID_ARG) return "invalid";
     if (st != GCONV_OK) return "unsupported";
     IgemmPlan ig;
-    if (use_igemm(s, false, 1, ig)) return "igemm_tf32_bf16x";
+    if (use_igemm(s, false, 1, ig)) return ig.prm.fused ? "igemm_tf32_bf16x_fused" : "igemm_tf32_bf16x";
     DirectPlan pl;
     if (!choose_direct(s, false, 1, s.W % 4 == 0, pl)) return "unsupported";
     if (pl.stream) return geom_name_stream(pl.geom);
@@ -1051,7 +1131,7 @@ size_t gconv2d_chain_workspace_size(int N, int C, int H, int W, int K, int R, in
         Shape sc = s;
         sc.N = B;
         IgemmPlan first;
-        return plan_igemm(sc, true, gn_groups, first) ? first.ws_bytes : 0;
+        return plan_igemm(sc, true, gn_groups, first, ig.prm.fused != 0) ? first.ws_bytes : 0;
     }
     DirectPlan pl;
     if (!choose_direct(s, true, gn_groups, s.W % 4 == 0, pl)) return 0;
@@ -1078,9 +1158,9 @@ gconv_status_t gconv2d_bias_scale_sigmoid_groupnorm_fwd(const float *x, const fl
     for (const void *q : {(const void *)bias, (const void *)scale, (const void *)gamma, (const void *)beta})
         if (q && (reinterpret_cast<uintptr_t>(q) & 3u)) return GCONV_ERR_INVALID_ARG;
     IgemmPlan ig;
-    if (use_igemm(s, true, gn_groups, ig))
+    if (use_igemm(s, true, gn_groups, ig) && igemm_plan_for_pointer(s, true, gn_groups, x, ig))
         return run_chain_igemm(s, ig, x, w, bias, scale, gn_groups, gamma, beta, eps, y, stream);
-    if (g_force.load(std::memory_order_relaxed) == kForceIgemm) return GCONV_ERR_UNSUPPORTED;
+    if (force_is_igemm()) return GCONV_ERR_UNSUPPORTED;
     DirectPlan pl;
     const bool x_vec = (s.W % 4 == 0) && aligned16(x);
     if (!choose_direct(s, true, gn_groups, x_vec, pl)) return GCONV_ERR_UNSUPPORTED;

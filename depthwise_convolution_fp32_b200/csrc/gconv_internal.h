@@ -145,14 +145,26 @@ struct IgemmParams {
     const float *aff_scale;    // null: 1
     int clamp;
     float lo, hi;
+    // chain epilogue: 0 = store a + partial statistics; 1 = partial statistics
+    // only; 2 = y = (a - mean) * rstd * gamma + beta from gn_stats, stored
+    int chain_mode;
+    const float2 *gn_stats;    // [N*gn_groups] (mean, rstd) for mode 2
+    const float *gamma, *beta;
+    // fused variant (N = 32, TH = igemm_fused_th()): x is staged raw by TMA
+    // ([8 channels][AR rows][COLSR columns], tensor map over x itself) into a
+    // ring of rr slots of raw_bytes and converted to the operand layout in
+    // shared memory by converter warps; no split pass, no x workspace
+    int fused;
+    int COLSR, raw_bytes, rr;
 };
 
 int igemm_supported_nt(int kpg);
+int igemm_fused_th();
 size_t igemm_header_bytes(int nt, bool chain);
 // GroupNorm partials the chain epilogue writes per tile and group (one per
 // TMEM lane quarter and per channel chunk the group spans)
 int igemm_partials_per_tile(int nt, int kgn);
-int igemm_threads(int nt);
+int igemm_threads(int nt, bool fused);
 // 4-D tensor map over a padded NC4HW4 tensor [quads][Hp][Wp][4] viewed as
 // [quads][Hp][Wp/16][64 floats]; one box is a whole x tile of one channel
 // step: 2 quads x box_rows rows x box_cols (multiple of 16) pixels.

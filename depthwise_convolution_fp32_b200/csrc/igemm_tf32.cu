@@ -143,7 +143,15 @@ __global__ void __launch_bounds__(256) split_w_kernel(const float *__restrict__ 
 // output channels, 8 (2 per lane quarter, 16-column chunks) for wider tiles,
 // so the epilogue keeps enough warps in flight without spilling registers.
 __host__ __device__ constexpr int ig_epi_warps(int NT) { return NT <= 32 ? 16 : 8; }
-__host__ __device__ constexpr int ig_threads(int NT) { return 64 + 32 * ig_epi_warps(NT); }
+// Fused variant: two converter warps between the MMA warp and the epilogue.
+constexpr int kConvWarps = 2;
+__host__ __device__ constexpr int ig_conv_warps(bool fused) { return fused ? kConvWarps : 0; }
+__host__ __device__ constexpr int ig_threads(int NT, bool fused = false) {
+    return 64 + 32 * ig_conv_warps(fused) + 32 * ig_epi_warps(NT);
+}
+// Output rows per tile of the fused variant (N = 32): 6 rows keep two x
+// operand stages, a raw staging slot and the resident weights in shared memory.
+constexpr int kFusedTH = 6;
 // shared memory ahead of the stage ring: barriers, TMEM slot, abort flag
 __host__ __device__ constexpr int ig_header(int NT, bool chain) { return 1024; }
 
@@ -269,8 +277,8 @@ __device__ __forceinline__ bool ig_mma_loop(const IgemmParams &p, uint32_t tmem,
 // tile j overlaps the MMAs of tile j+1.
 // KGN: 0 = plain convolution; otherwise the GroupNorm group width of the
 // chain (1, 2, 4, 8, 16, or 32 standing for any multiple of 16).
-template <int NT, int KGN>
-__global__ void __launch_bounds__(ig_threads(NT), 1)
+template <int NT, int KGN, bool FUSED>
+__global__ void __launch_bounds__(ig_threads(NT, FUSED), 1)
     igemm_tf32x3_kernel(const __grid_constant__ TensorMap tmh, const __grid_constant__ TensorMap tmc,
                         const IgemmParams p) {
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -283,7 +291,10 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
     uint32_t *tslot = reinterpret_cast<uint32_t *>(fullA + 20);
     int *abort_flag = reinterpret_cast<int *>(fullA + 21);
     uint64_t *drain = fullA + 22;                           // every issued MMA has completed
+    uint64_t *rawFull = fullA + 24;                         // [2] fused: raw x box landed
+    uint64_t *rawEmpty = fullA + 26;                        // [2] fused: raw slot converted
     constexpr bool CHAIN = KGN > 0;
+    constexpr int CWARPS = ig_conv_warps(FUSED);
     unsigned char *stages = smem + ig_header(NT, CHAIN);
 
     const int tid = threadIdx.x;
@@ -293,14 +304,20 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
     const uint32_t b_slot = 2u * p.b_bytes;   // w_hi + w_lo slice of one (channel step, tap row)
     unsigned char *ringA = stages;
     unsigned char *ringB = stages + (size_t)p.sa * a_slot;
+    unsigned char *ringR = ringB + (size_t)p.sb * b_slot;   // fused: raw x boxes
     const uint32_t acc_cols = (uint32_t)(p.TH * NT);
 
     if (tid == 0) {
         for (int s = 0; s < 4; ++s) {
-            dev::mbar_init(&fullA[s], 1);
+            // fused: an x stage is complete when every converter warp has arrived
+            dev::mbar_init(&fullA[s], FUSED ? CWARPS : 1);
             dev::mbar_init(&emptyA[s], 1);
             dev::mbar_init(&fullB[s], 1);
             dev::mbar_init(&emptyB[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            dev::mbar_init(&rawFull[s], 1);
+            dev::mbar_init(&rawEmpty[s], CWARPS > 0 ? CWARPS : 1);
         }
         for (int b = 0; b < 2; ++b) {
             dev::mbar_init(&accf[b], 1);
@@ -337,14 +354,30 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
             for (int cc8 = 0; cc8 < p.CC8 && ok; ++cc8, ++ia) {
                 const int sa = ia % p.sa, ua = ia / p.sa;
                 if (lane == 0) {
-                    if (ua > 0 && !dev::mbar_wait_bounded(&emptyA[sa], (ua - 1) & 1)) ok = false;
-                    if (*(volatile int *)abort_flag) ok = false;
-                    if (ok) {
-                        dev::mbar_arrive_expect_tx(&fullA[sa], a_slot);
-                        unsigned char *st = ringA + (size_t)sa * a_slot;
-                        const int cz = z0 + cc8 * 2;
-                        dev::tma_load_4d(st, &tmh, &fullA[sa], 0, tl.q0 / 16, tl.p0, cz);
-                        dev::tma_load_4d(st + p.a_bytes, &tmc, &fullA[sa], 0, tl.q0 / 16, tl.p0, cz);
+                    if constexpr (FUSED) {
+                        // raw x box [8 channels][AR rows][COLSR columns] starting at the
+                        // tile's first input row and at its first input column rounded
+                        // down to 4 (16-byte TMA coordinate); zero fill = padding
+                        const int sr = ia % p.rr, ur = ia / p.rr;
+                        if (ur > 0 && !dev::mbar_wait_bounded(&rawEmpty[sr], (ur - 1) & 1)) ok = false;
+                        if (*(volatile int *)abort_flag) ok = false;
+                        if (ok) {
+                            const int x0 = tl.q0 - p.pad_w;
+                            dev::mbar_arrive_expect_tx(&rawFull[sr], (uint32_t)p.raw_bytes);
+                            dev::tma_load_3d(ringR + (size_t)sr * p.raw_bytes, &tmh, &rawFull[sr],
+                                             x0 - (((x0 % 4) + 4) % 4), tl.p0 - p.pad,
+                                             tl.n * p.C + tl.g * p.cpg + cc8 * 8);
+                        }
+                    } else {
+                        if (ua > 0 && !dev::mbar_wait_bounded(&emptyA[sa], (ua - 1) & 1)) ok = false;
+                        if (*(volatile int *)abort_flag) ok = false;
+                        if (ok) {
+                            dev::mbar_arrive_expect_tx(&fullA[sa], a_slot);
+                            unsigned char *st = ringA + (size_t)sa * a_slot;
+                            const int cz = z0 + cc8 * 2;
+                            dev::tma_load_4d(st, &tmh, &fullA[sa], 0, tl.q0 / 16, tl.p0, cz);
+                            dev::tma_load_4d(st + p.a_bytes, &tmc, &fullA[sa], 0, tl.q0 / 16, tl.p0, cz);
+                        }
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -376,8 +409,13 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
         if (lane == 0) {
             // copies still in flight (only after an abort): wait, bounded, for the
             // last phase issued on every slot before the CTA may exit
-            for (int j = ia > p.sa ? ia - p.sa : 0; j < ia; ++j)
-                dev::mbar_wait_bounded(&fullA[j % p.sa], (uint32_t)(j / p.sa) & 1u);
+            if constexpr (FUSED) {
+                for (int j = ia > p.rr ? ia - p.rr : 0; j < ia; ++j)
+                    dev::mbar_wait_bounded(&rawFull[j % p.rr], (uint32_t)(j / p.rr) & 1u);
+            } else {
+                for (int j = ia > p.sa ? ia - p.sa : 0; j < ia; ++j)
+                    dev::mbar_wait_bounded(&fullA[j % p.sa], (uint32_t)(j / p.sa) & 1u);
+            }
             if (p.b_resident) {
                 for (int j = 0; j < ib; ++j) dev::mbar_wait_bounded(&fullB[j], 0);
             } else {
@@ -392,7 +430,7 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
             // loop bounds fixed at compile time for the common geometries
             // (dilation 1, default rows per tile): the issue loop then runs
             // back to back on constant operand offsets
-            constexpr int THD = ig_default_th(NT);
+            constexpr int THD = FUSED ? kFusedTH : ig_default_th(NT);
             const bool d1 = p.dil == 1 && p.dil_w == 1 && p.TH == THD;
             bool ok;
             if (d1 && p.R == 3 && p.S == 3) ok = ig_mma_loop<NT, THD, 3, 3>(p, tmem, ringA, ringB, a_slot, b_slot, fullA, emptyA, fullB, emptyB, accf, acce);
@@ -407,6 +445,75 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
             // arrives once every MMA this thread issued has completed
             dev::mma_commit(drain);
             dev::mbar_wait_bounded(drain, 0);
+        }
+        __syncwarp();
+    } else if (FUSED && warp < 2 + CWARPS) {
+        // ---------------------------------------------------------- converter
+        // Per tile and 8-channel step: wait for the raw x box and for the x stage
+        // to be free, then write the stage as the split pass would: per staged
+        // pixel (row, column) the tf32 parts of the 8 channels as two 16-byte
+        // quads and the bf16 cross-term operand ([bf16(x_hi) x 8], [bf16(x - x_hi) x 8])
+        // as two 16-byte chunks, in the same layout the TMA boxes of the unfused
+        // variant deliver.  Identical arithmetic, so identical results.
+        constexpr int CT = 32 * CWARPS;
+        const int ctid = tid - 64;
+        const int AR = p.AR, COLS = p.COLS, COLSR = p.COLSR;
+        const int plane_r = AR * COLSR;           // floats between raw channel planes
+        const int npx = AR * COLS;
+        const int dq = CT / COLS, dr = CT % COLS;  // pixel-index step as (rows, columns)
+        int ia = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            const IgTile tl = ig_tile(p, t);
+            const int cofs = ((tl.q0 - p.pad_w) % 4 + 4) % 4;
+            for (int cc8 = 0; cc8 < p.CC8; ++cc8, ++ia) {
+                const int sa = ia % p.sa, ua = ia / p.sa, sr = ia % p.rr, ur = ia / p.rr;
+                if (*(volatile int *)abort_flag) ok = false;
+                if (ok && !dev::mbar_wait_bounded(&rawFull[sr], (uint32_t)ur & 1u)) ok = false;
+                if (ok && ua > 0 && !dev::mbar_wait_bounded(&emptyA[sa], (uint32_t)(ua - 1) & 1u)) ok = false;
+                if (!__all_sync(0xffffffffu, ok)) {
+                    ok = false;
+                    break;
+                }
+                const float *raw = reinterpret_cast<const float *>(ringR + (size_t)sr * p.raw_bytes) + cofs;
+                float4 *dh = reinterpret_cast<float4 *>(ringA + (size_t)sa * a_slot);
+                uint4 *dc = reinterpret_cast<uint4 *>(ringA + (size_t)sa * a_slot + p.a_bytes);
+                int row = ctid / COLS, col = ctid % COLS;
+                for (int px = ctid; px < npx; px += CT) {
+                    const float *src = raw + row * COLSR + col;
+                    float hi[8], lo[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float v = src[j * plane_r];
+                        hi[j] = dev::to_tf32(v);
+                        lo[j] = v - hi[j];
+                    }
+                    const int cell = row * COLS + col;   // quad / chunk 0; quad / chunk 1 is npx cells on
+                    dh[cell] = make_float4(hi[0], hi[1], hi[2], hi[3]);
+                    dh[cell + npx] = make_float4(hi[4], hi[5], hi[6], hi[7]);
+                    dc[cell] = make_uint4(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]),
+                                          pack_bf16x2(hi[4], hi[5]), pack_bf16x2(hi[6], hi[7]));
+                    dc[cell + npx] = make_uint4(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]),
+                                                pack_bf16x2(lo[4], lo[5]), pack_bf16x2(lo[6], lo[7]));
+                    col += dr;
+                    row += dq;
+                    if (col >= COLS) {
+                        col -= COLS;
+                        ++row;
+                    }
+                }
+                // generic-proxy writes visible to the tensor core (async proxy)
+                asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                __syncwarp();
+                if (lane == 0) {
+                    dev::mbar_arrive(&rawEmpty[sr]);
+                    dev::mbar_arrive(&fullA[sa]);
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            *abort_flag = 1;
+            atomicExch(&g_igemm_error, 1);
         }
         __syncwarp();
     } else {
@@ -424,7 +531,7 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
         constexpr int GPC = CHAIN ? (KGN >= CW ? 1 : CW / KGN) : 1;
         constexpr int GW = CHAIN ? (KGN >= CW ? CW : KGN) : CW;
         constexpr float kLog2e = 1.4426950408889634f;
-        const int ew = warp - 2;                 // 0..EPW-1
+        const int ew = warp - 2 - CWARPS;        // 0..EPW-1
         const int lq = warp & 3;                 // TMEM lane quarter this warp may access
         const int cpart = ew >> 2;               // column block of this warp
         const int m = lq * 32 + lane;
@@ -474,6 +581,21 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
                 float shift[GPC], s1[GPC], s2[GPC];
 #pragma unroll
                 for (int gg = 0; gg < GPC; ++gg) { shift[gg] = 0.f; s1[gg] = 0.f; s2[gg] = 0.f; }
+                // chain mode 2: y = (a - mean) * (rstd * gamma) + beta with the group's
+                // finished statistics, the same three roundings as the normalize pass
+                float nmean[CHAIN ? CW : 1], nmul[CHAIN ? CW : 1], nadd[CHAIN ? CW : 1];
+                if constexpr (CHAIN) {
+                    if (p.chain_mode == 2) {
+#pragma unroll
+                        for (int jj = 0; jj < CW; ++jj) {
+                            const int k = tl.g * p.kpg + c0 + jj;
+                            const float2 st = p.gn_stats[(long long)tl.n * p.gn_groups + k / p.kgn];
+                            nmean[jj] = st.x;
+                            nmul[jj] = (float)((double)st.y * (double)__ldg(p.gamma + k));
+                            nadd[jj] = __ldg(p.beta + k);
+                        }
+                    }
+                }
                 // output pointer of channel c0 in the current row; channels are `plane` apart
                 float *yc = ybase + (long long)c0 * plane;
                 // rows are processed two at a time so one TMEM load latency covers both
@@ -491,7 +613,7 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
                         if constexpr (CHAIN) {
 #pragma unroll
                             for (int jj = 0; jj < CW; ++jj) v[jj] = rcp_ftz(1.f + ex2_ftz(fmaf(v[jj], mul[jj], add[jj])));
-                            if (rvalid && i + h == 0) {
+                            if (p.chain_mode != 2 && rvalid && i + h == 0) {
 #pragma unroll
                                 for (int gg = 0; gg < GPC; ++gg) shift[gg] = __shfl_sync(0xffffffffu, v[gg * GW], 0);
                             }
@@ -504,16 +626,23 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
                             }
                         }
                         if (rvalid && qvalid) {
-                            float *yr = yc;
-#pragma unroll
-                            for (int jj = 0; jj < CW; ++jj, yr += plane) *yr = v[jj];
                             if constexpr (CHAIN) {
+                                if (p.chain_mode == 2) {
 #pragma unroll
-                                for (int jj = 0; jj < CW; ++jj) {
-                                    const float d = v[jj] - shift[jj / GW];
-                                    s1[jj / GW] += d;
-                                    s2[jj / GW] = fmaf(d, d, s2[jj / GW]);
+                                    for (int jj = 0; jj < CW; ++jj) v[jj] = fmaf(v[jj] - nmean[jj], nmul[jj], nadd[jj]);
+                                } else {
+#pragma unroll
+                                    for (int jj = 0; jj < CW; ++jj) {
+                                        const float d = v[jj] - shift[jj / GW];
+                                        s1[jj / GW] += d;
+                                        s2[jj / GW] = fmaf(d, d, s2[jj / GW]);
+                                    }
                                 }
+                            }
+                            if (!CHAIN || p.chain_mode != 1) {   // mode 1 keeps only the statistics
+                                float *yr = yc;
+#pragma unroll
+                                for (int jj = 0; jj < CW; ++jj, yr += plane) *yr = v[jj];
                             }
                         }
                         yc += p.Q;
@@ -525,7 +654,7 @@ __global__ void __launch_bounds__(ig_threads(NT), 1)
                     __syncwarp();
                     if (lane == 0) dev::mbar_arrive(&acce[buf]);
                 }
-                if constexpr (CHAIN) {
+                if (CHAIN && p.chain_mode != 2) {
                     const unsigned vmask = __ballot_sync(0xffffffffu, qvalid);
                     const int cnt_i = __popc(vmask) * rows * GW;
                     // 1/count: FP32 reciprocal refined by one Newton step in FP64 (count < 2^24)
@@ -575,9 +704,9 @@ cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-template <int NT, int KGN>
+template <int NT, int KGN, bool FUSED>
 cudaError_t launch_nt(const IgemmParams &p, const TensorMap *tm, dim3 grid, size_t smem, cudaStream_t st) {
-    auto kern = igemm_tf32x3_kernel<NT, KGN>;
+    auto kern = igemm_tf32x3_kernel<NT, KGN, FUSED>;
     // the shared-memory opt-in is per function and device: raise it to the
     // planner's ceiling once per device instead of on every launch
     static std::atomic<unsigned long long> opted{0};
@@ -590,20 +719,20 @@ cudaError_t launch_nt(const IgemmParams &p, const TensorMap *tm, dim3 grid, size
         if (bit) opted.fetch_or(bit, std::memory_order_acq_rel);
     }
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
-    return launch_ex(kern, grid, dim3(ig_threads(NT)), smem, st, tm[0], tm[1], p);
+    return launch_ex(kern, grid, dim3(ig_threads(NT, FUSED)), smem, st, tm[0], tm[1], p);
 }
 
-template <int NT>
+template <int NT, bool FUSED>
 cudaError_t launch_chain_nt(const IgemmParams &p, const TensorMap *tm, dim3 grid, size_t smem,
                             cudaStream_t st) {
     switch (p.kgn) {
-        case 1: return launch_nt<NT, 1>(p, tm, grid, smem, st);
-        case 2: return launch_nt<NT, 2>(p, tm, grid, smem, st);
-        case 4: return launch_nt<NT, 4>(p, tm, grid, smem, st);
-        case 8: return launch_nt<NT, 8>(p, tm, grid, smem, st);
-        case 16: return launch_nt<NT, 16>(p, tm, grid, smem, st);
+        case 1: return launch_nt<NT, 1, FUSED>(p, tm, grid, smem, st);
+        case 2: return launch_nt<NT, 2, FUSED>(p, tm, grid, smem, st);
+        case 4: return launch_nt<NT, 4, FUSED>(p, tm, grid, smem, st);
+        case 8: return launch_nt<NT, 8, FUSED>(p, tm, grid, smem, st);
+        case 16: return launch_nt<NT, 16, FUSED>(p, tm, grid, smem, st);
         default:
-            if (p.kgn % 16 == 0) return launch_nt<NT, 32>(p, tm, grid, smem, st);
+            if (p.kgn % 16 == 0) return launch_nt<NT, 32, FUSED>(p, tm, grid, smem, st);
             return cudaErrorInvalidValue;
     }
 }
@@ -633,7 +762,7 @@ int igemm_partials_per_tile(int nt, int kgn) {
     return 4 * (kgn > cw ? kgn / cw : 1);
 }
 
-int igemm_threads(int nt) { return ig_threads(nt); }
+int igemm_threads(int nt, bool fused) { return ig_threads(nt, fused); }
 
 bool make_nc4hw4_tile_map(TensorMap *tm, const float *base, long long quads, int Hp, int Wp, int box_cols,
                           int box_rows) {
@@ -670,21 +799,27 @@ cudaError_t launch_split_w(const float *w, float *wh, float *wl, int K, int cpg,
 
 cudaError_t launch_igemm(const IgemmParams &p, const TensorMap *tm, int chain, dim3 grid, size_t smem,
                          cudaStream_t st) {
+    if (p.fused) {   // N = 32 only
+        if (p.kpg != 32 || p.TH != kFusedTH) return cudaErrorInvalidValue;
+        return chain ? launch_chain_nt<32, true>(p, tm, grid, smem, st) : launch_nt<32, 0, true>(p, tm, grid, smem, st);
+    }
     if (chain) {
         switch (p.kpg) {
-            case 32: return launch_chain_nt<32>(p, tm, grid, smem, st);
-            case 64: return launch_chain_nt<64>(p, tm, grid, smem, st);
+            case 32: return launch_chain_nt<32, false>(p, tm, grid, smem, st);
+            case 64: return launch_chain_nt<64, false>(p, tm, grid, smem, st);
             default: return cudaErrorInvalidValue;
         }
     }
     switch (p.kpg) {
-        case 32: return launch_nt<32, 0>(p, tm, grid, smem, st);
-        case 64: return launch_nt<64, 0>(p, tm, grid, smem, st);
-        case 128: return launch_nt<128, 0>(p, tm, grid, smem, st);
-        case 256: return launch_nt<256, 0>(p, tm, grid, smem, st);
+        case 32: return launch_nt<32, 0, false>(p, tm, grid, smem, st);
+        case 64: return launch_nt<64, 0, false>(p, tm, grid, smem, st);
+        case 128: return launch_nt<128, 0, false>(p, tm, grid, smem, st);
+        case 256: return launch_nt<256, 0, false>(p, tm, grid, smem, st);
         default: return cudaErrorInvalidValue;
     }
 }
+
+int igemm_fused_th() { return kFusedTH; }
 
 int read_and_clear_igemm_error() {
     int v = 0, zero = 0;

@@ -488,7 +488,7 @@ def test_igemm_matches_oracle(oracle_mod, geo):
                            x_dist="normal", bias=bias)
     gc.force_kernel("igemm")
     try:
-        assert gc.plan_name(N, C, H, W, K, R, S, st, pad, dil, g) == "igemm_tf32_bf16x"
+        assert gc.plan_name(N, C, H, W, K, R, S, st, pad, dil, g).startswith("igemm_tf32_bf16x")
         full_check(oracle_mod, d, st, pad, dil, g, "igemm " + str(geo))
     finally:
         gc.force_kernel("auto")
@@ -516,6 +516,102 @@ def test_chain_paths_agree_with_oracle(oracle_mod, mode):
         gc.force_kernel("auto")
     ref = _chain_ref(oracle_mod, d, 1, 0, 1, 1, 1e-5)
     assert_chain_close(y, ref, d["scale"].numpy(), d["gamma"].numpy(), 1e-5, 4, f"{mode} chain")
+
+
+# ---------------------------------------------------- fused operand staging (igemm)
+# The fused implicit GEMM stages x raw by TMA and converts it in shared memory;
+# the conversion is the split pass's arithmetic, so both give the same bits.
+FUSED_GEOMS = [
+    # N, C, H, W, K, R, S, stride, pad, dil, groups, bias
+    (2, 8, 19, 36, 32, 3, 3, 1, 1, 1, 1, True),       # padding 1: raw box starts left of the image
+    (1, 8, 20, 152, 32, 3, 3, 1, 0, 1, 1, False),     # two column tiles, ragged
+    (2, 16, 10, 20, 64, 3, 3, 1, 1, 1, 2, True),      # two groups, two channel steps
+    (1, 24, 11, 24, 32, 3, 5, 1, 1, 1, 1, False),     # R != S, three channel steps
+    (1, 16, 17, 32, 32, 3, 3, 1, 2, 2, 1, True),      # dilation 2, pad 2 (start not a multiple of 4)
+    (2, 8, 64, 68, 32, 3, 3, 1, 3, 1, 1, True),       # pad 3
+]
+
+
+@pytest.mark.parametrize("geo", FUSED_GEOMS, ids=lambda g: "x".join(map(str, g[:11])))
+def test_fused_igemm_matches_split_bitwise_and_oracle(oracle_mod, geo):
+    N, C, H, W, K, R, S, st, pad, dil, g, bias = geo
+    d = inputs.conv_inputs(N, C, H, W, K, R, S, g, seed=23 + zlib.crc32(repr(geo).encode()) % 1000,
+                           x_dist="normal", bias=bias)
+    outs = {}
+    for mode in ("igemm_fused", "igemm_split"):
+        gc.force_kernel(mode)
+        try:
+            plan = gc.plan_name(N, C, H, W, K, R, S, st, pad, dil, g)
+            assert plan == ("igemm_tf32_bf16x_fused" if mode == "igemm_fused" else "igemm_tf32_bf16x"), plan
+            outs[mode] = run_conv(d, st, pad, dil, g).cpu()
+        finally:
+            gc.force_kernel("auto")
+    assert torch.equal(outs["igemm_fused"], outs["igemm_split"])
+    ref, acc = oracle_mod.conv2d(d["x"], d["w"], d.get("bias"), st, pad, dil, g, return_absacc=True)
+    assert_conv_close(outs["igemm_fused"].numpy(), ref, acc, "fused " + str(geo))
+    assert gc.library().gconv_device_error_status() == gc.OK
+
+
+@pytest.mark.parametrize("cfg", [(2, 8, 40, 40, 32, 8, 1.0), (3, 8, 37, 44, 32, 2, 1.0), (2, 8, 24, 24, 32, 32, 3.0)])
+def test_fused_chain_matches_split_bitwise_and_oracle(oracle_mod, cfg):
+    N, C, H, W, K, gn, std = cfg
+    d = inputs.chain_inputs(N, C, H, W, K, 3, 3, 1, gn, seed=90 + N * H, bias_scale_std=std, affine="random")
+    outs = {}
+    for mode in ("igemm_fused", "igemm_split"):
+        gc.force_kernel(mode)
+        try:
+            outs[mode] = _chain_dev(d, 1, 0, 1, 1, 1e-5).cpu()
+        finally:
+            gc.force_kernel("auto")
+    assert torch.equal(outs["igemm_fused"], outs["igemm_split"])
+    ref = _chain_ref(oracle_mod, d, 1, 0, 1, 1, 1e-5)
+    assert_chain_close(outs["igemm_fused"].numpy(), ref, d["scale"].numpy(), d["gamma"].numpy(), 1e-5, K // gn,
+                       "fused chain " + str(cfg))
+
+
+_STORE_DESIGN_SCRIPT = r"""
+import sys, json
+sys.path.insert(0, sys.argv[1]); sys.path.insert(0, sys.argv[1] + "/tests")
+import numpy as np, torch
+import depthwise_convolution_fp32_b200 as gc
+from depthwise_convolution_fp32_b200 import inputs
+import oracle
+from tolerance import assert_chain_close
+d = inputs.chain_inputs(2, 8, 40, 44, 32, 3, 3, 1, 8, seed=95, bias_scale_std=1.0, affine="random")
+outs = []
+for mode in ("igemm_fused", "igemm_split"):
+    gc.force_kernel(mode)
+    y = gc.conv2d_bias_scale_sigmoid_groupnorm(d["x"].cuda(), d["w"].cuda(), (d["b_conv"] + d["b_extra"]).cuda(),
+                                               d["scale"].cuda(), 8, d["gamma"].cuda(), d["beta"].cuda(), 1e-5,
+                                               1, 0, 1, 1)
+    torch.cuda.synchronize()
+    outs.append(y.cpu())
+gc.force_kernel("auto")
+ref = oracle.chain(d["x"], d["w"], d["b_conv"], d["b_extra"], d["scale"], 8, d["gamma"], d["beta"], 1e-5, 1, 0, 1, 1)
+assert torch.equal(outs[0], outs[1])
+assert_chain_close(outs[0].numpy(), ref, d["scale"].numpy(), d["gamma"].numpy(), 1e-5, 4, "store design")
+np.save(sys.argv[2], outs[0].numpy())
+print("ok")
+"""
+
+
+def test_chain_store_design_matches_recompute_bitwise(tmp_path):
+    """The chain's other design (GEMM stores the logistic output, a streaming
+    pass normalizes it) gives the same bits as the default (GEMM twice:
+    statistics, then the normalized output); the design is chosen once per
+    process, so the other one runs in a child process."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = tmp_path / "store.npy"
+    env = dict(os.environ, GCONV_CHAIN_DESIGN="store")
+    r = subprocess.run([sys.executable, "-c", _STORE_DESIGN_SCRIPT, root, str(out)], env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr
+    d = inputs.chain_inputs(2, 8, 40, 44, 32, 3, 3, 1, 8, seed=95, bias_scale_std=1.0, affine="random")
+    y = _chain_dev(d, 1, 0, 1, 1, 1e-5).cpu().numpy()
+    assert np.array_equal(y, np.load(out))
 
 
 # ------------------------------------------------------------ affine + clamp epilogue
