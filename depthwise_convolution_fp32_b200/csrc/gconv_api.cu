@@ -640,7 +640,27 @@ struct IgemmPlan {
     dim3 grid;
     size_t smem;
     size_t off_xl, off_wh, off_wl, off_part, off_stats, ws_bytes;
+    int pack = 1;     // original conv groups per GEMM group (block-diagonal weights when > 1)
 };
+
+// The same convolution with gp consecutive groups packed into one: groups/gp
+// groups of gp*cpg input and gp*kpg output channels (block-diagonal weights).
+Shape packed_shape(const Shape &s, int gp) {
+    Shape t = s;
+    t.groups = s.groups / gp;
+    t.cpg = s.cpg * gp;
+    t.kpg = s.kpg * gp;
+    return t;
+}
+
+// Packing factor that brings a narrow group to the tensor path's 32 output
+// channels (0 when the shape cannot be packed so).
+int igemm_pack(const Shape &s) {
+    if (s.kpg >= 32 || 32 % s.kpg != 0) return 0;
+    const int gp = 32 / s.kpg;
+    if (s.groups % gp != 0 || (s.cpg * gp) % 8 != 0) return 0;
+    return gp;
+}
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
@@ -699,8 +719,7 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl, bool f
     // output rows per tile: two accumulator buffers of TH*NT columns fit TMEM
     int TH = std::max(1, std::min(8, 256 / NT));
     if (force_th > 0) TH = force_th;
-    if (fused) TH = igemm_fused_th();   // the fused issue loop is compiled for it
-    if (TH > s.P && fused) return false;
+    if (fused) TH = igemm_fused_th();   // the fused issue loop is compiled for it (fewer rows run it unrolled less)
     TH = std::min(TH, s.P);
     const size_t limit = 227 * 1024 - igemm_header_bytes(NT, chain);
     const int b_bytes = 32 * s.S * NT;              // one w operand slice: S taps x 8 channels x NT
@@ -720,7 +739,6 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl, bool f
         while (sa > 1 && (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes > lim) --sa;
         while (sb > 1 && (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes > lim) --sb;
         if ((size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes <= lim && (!fused || sa == 2)) break;
-        if (fused) return false;
     }
     if (TH < 1) return false;
     if (fused && (COLSR > 256 || raw_bytes <= 0)) return false;
@@ -772,6 +790,11 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl, bool f
     return true;
 }
 
+const char *igemm_name(const IgemmPlan &ig) {
+    if (ig.pack > 1) return ig.prm.fused ? "igemm_tf32_bf16x_fused_packed" : "igemm_tf32_bf16x_packed";
+    return ig.prm.fused ? "igemm_tf32_bf16x_fused" : "igemm_tf32_bf16x";
+}
+
 bool force_is_igemm() {
     const int f = g_force.load(std::memory_order_relaxed);
     return f == kForceIgemm || f == kForceIgemmSplit || f == kForceIgemmFused;
@@ -782,7 +805,10 @@ bool force_is_igemm() {
 bool igemm_plan_for_pointer(const Shape &s, bool chain, int gn_groups, const float *x, IgemmPlan &pl) {
     if (!pl.prm.fused || aligned16(x)) return true;
     if (g_force.load(std::memory_order_relaxed) == kForceIgemmFused) return false;
-    return plan_igemm(s, chain, gn_groups, pl, false);
+    const int gp = pl.pack;
+    if (!plan_igemm(gp > 1 ? packed_shape(s, gp) : s, chain, gn_groups, pl, false)) return false;
+    pl.pack = gp;
+    return true;
 }
 
 // Whether the dispatcher sends a shape to the implicit GEMM.
@@ -791,14 +817,19 @@ bool use_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     if (force == kForceDirect || force == kForceGeneric || force == kForceCpAsync || force == kForceBlocked ||
         force == kForceStream)
         return false;
-    if (force == kForceIgemmFused) return plan_igemm(s, chain, gn_groups, pl, true);
-    if (force == kForceIgemmSplit) return plan_igemm(s, chain, gn_groups, pl, false);
-    if (!(igemm_fused_wanted() && plan_igemm(s, chain, gn_groups, pl, true)) && !plan_igemm(s, chain, gn_groups, pl))
+    // groups narrower than the tensor path's 32 output channels run packed
+    const int gp = igemm_pack(s);
+    const Shape sp = gp ? packed_shape(s, gp) : s;
+    pl.pack = gp ? gp : 1;
+    if (force == kForceIgemmFused) return plan_igemm(sp, chain, gn_groups, pl, true);
+    if (force == kForceIgemmSplit) return plan_igemm(sp, chain, gn_groups, pl, false);
+    if (!(igemm_fused_wanted() && plan_igemm(sp, chain, gn_groups, pl, true)) && !plan_igemm(sp, chain, gn_groups, pl))
         return false;
     if (force == kForceIgemm) return true;
     if (const DispatchEntry *e = table_choice(s, chain)) return e->family == kTabIgemm;
-    // outside the table: enough reduction depth and output channels for the tensor cores to win
-    return s.cpg * s.R * s.S >= 64;
+    // outside the table: enough reduction depth and output channels for the tensor cores to win;
+    // packed groups only where measured (the table)
+    return !gp && s.cpg * s.R * s.S >= 64;
 }
 
 // Launch the split passes and the GEMM; chain additionally runs the GroupNorm
@@ -844,7 +875,7 @@ gconv_status_t run_igemm(const Shape &s, IgemmPlan &pl, const float *x, const fl
     p.gn_part = chain ? reinterpret_cast<float4 *>(base + pl.off_part) : nullptr;
     if (!p.fused && launch_split_x(x, xh, xl, s.N, s.C, s.H, s.W, s.pad, s.pw, p.Hp, p.Wp, stream) != cudaSuccess)
         return GCONV_ERR_CUDA;
-    if (split_w && launch_split_w(w, wh, wl, s.K, s.cpg, s.R, s.S, s.groups, stream) != cudaSuccess)
+    if (split_w && launch_split_w(w, wh, wl, s.K, p.cpg, s.R, s.S, p.groups, stream, pl.pack) != cudaSuccess)
         return GCONV_ERR_CUDA;
     // the chain either stores the logistic output and normalizes it in a
     // streaming pass (store), or runs the GEMM twice: statistics only, then the
@@ -902,9 +933,11 @@ gconv_status_t run_chain_igemm(const Shape &s, const IgemmPlan &full, const floa
     Shape sc = s;
     sc.N = B;
     const bool fused = full.prm.fused != 0;
+    const int gp = full.pack;
     IgemmPlan first;
     if (B == s.N) first = full;
-    else if (!plan_igemm(sc, true, gn_groups, first, fused)) return GCONV_ERR_UNSUPPORTED;
+    else if (!plan_igemm(gp > 1 ? packed_shape(sc, gp) : sc, true, gn_groups, first, fused)) return GCONV_ERR_UNSUPPORTED;
+    first.pack = gp;
     void *ws = nullptr;
     gconv_status_t st = ensure_workspace(first.ws_bytes, stream, &ws);
     if (st != GCONV_OK) return st;
@@ -922,7 +955,9 @@ gconv_status_t run_chain_igemm(const Shape &s, const IgemmPlan &full, const floa
             Shape sl = s;
             sl.N = nb;
             IgemmPlan cur;
-            if (!plan_igemm(sl, true, gn_groups, cur, fused)) return GCONV_ERR_UNSUPPORTED;
+            if (!plan_igemm(gp > 1 ? packed_shape(sl, gp) : sl, true, gn_groups, cur, fused))
+                return GCONV_ERR_UNSUPPORTED;
+            cur.pack = gp;
             st = run_igemm(sl, cur, x + n0 * x_img, w, bias, scale, gn_groups, gamma, beta, eps, y + n0 * y_img, ws,
                            stream);
         }
@@ -1071,7 +1106,7 @@ const char *gconv2d_plan_name(int N, int C, int H, int W, int K, int R, int S, i
     if (st == GCONV_ERR_INVALID_ARG) return "invalid";
     if (st != GCONV_OK) return "unsupported";
     IgemmPlan ig;
-    if (use_igemm(s, chain != 0, chain ? s.K : 1, ig)) return ig.prm.fused ? "igemm_tf32_bf16x_fused" : "igemm_tf32_bf16x";
+    if (use_igemm(s, chain != 0, chain ? s.K : 1, ig)) return igemm_name(ig);
     DirectPlan pl;
     int gn = 1;
     if (!choose_direct(s, chain != 0, gn, s.W % 4 == 0, pl)) return "unsupported";
@@ -1103,7 +1138,7 @@ const char *gconv2d_plan_name_ex(int N, int C, int H, int W, int K, int R, int S
     if (st == GCONV_ERR_INVALID_ARG) return "invalid";
     if (st != GCONV_OK) return "unsupported";
     IgemmPlan ig;
-    if (use_igemm(s, false, 1, ig)) return ig.prm.fused ? "igemm_tf32_bf16x_fused" : "igemm_tf32_bf16x";
+    if (use_igemm(s, false, 1, ig)) return igemm_name(ig);
     DirectPlan pl;
     if (!choose_direct(s, false, 1, s.W % 4 == 0, pl)) return "unsupported";
     if (pl.stream) return geom_name_stream(pl.geom);
@@ -1131,7 +1166,8 @@ size_t gconv2d_chain_workspace_size(int N, int C, int H, int W, int K, int R, in
         Shape sc = s;
         sc.N = B;
         IgemmPlan first;
-        return plan_igemm(sc, true, gn_groups, first, ig.prm.fused != 0) ? first.ws_bytes : 0;
+        return plan_igemm(ig.pack > 1 ? packed_shape(sc, ig.pack) : sc, true, gn_groups, first, ig.prm.fused != 0)
+                   ? first.ws_bytes : 0;
     }
     DirectPlan pl;
     if (!choose_direct(s, true, gn_groups, s.W % 4 == 0, pl)) return 0;

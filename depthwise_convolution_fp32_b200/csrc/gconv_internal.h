@@ -172,8 +172,9 @@ bool make_nc4hw4_tile_map(TensorMap *tm, const float *base, long long quads, int
                           int box_rows);
 cudaError_t launch_split_x(const float *x, float *xh, float *xl, int N, int C, int H, int W, int pad_h, int pad_w,
                            int Hp, int Wp, cudaStream_t st);
+// groups, cpg: the GEMM's; gp > 1 packs gp original groups into each (block-diagonal weights)
 cudaError_t launch_split_w(const float *w, float *wh, float *wl, int K, int cpg, int R, int S, int groups,
-                           cudaStream_t st);
+                           cudaStream_t st, int gp = 1);
 // tm: x_hi tile map, cross-term tile map
 cudaError_t launch_igemm(const IgemmParams &p, const TensorMap *tm, int chain, dim3 grid, size_t smem,
                          cudaStream_t st);

@@ -107,9 +107,14 @@ __global__ void __launch_bounds__(256) split_x_kernel(const float *__restrict__ 
 //   wh: [g][c8][r][s][2][kpg][4]   tf32 parts (two channel quads)
 //   wc: [g][c8][r][s][2][kpg][8]   bf16 parts: chunk 0 = bf16(w - w_hi), chunk 1 = bf16(w_hi)
 // so that the bf16 MMA over K = 16 computes x_hi*w_lo + x_lo*w_hi.
+// Packed groups (gp > 1): the GEMM runs gp consecutive conv groups as one
+// group of gp*cpg input and gp*kpg output channels whose weights are block
+// diagonal: output kk of the packed group reads input c only when both belong
+// to the same original group (kk / kpg0 == c / cpg0), else the weight is 0.
+// kpg and cpg here are the packed sizes, kpg0 and cpg0 the original ones.
 __global__ void __launch_bounds__(256) split_w_kernel(const float *__restrict__ w, float4 *__restrict__ wh,
                                                       uint4 *__restrict__ wc, int kpg, int cpg, int R, int S,
-                                                      long long cells) {
+                                                      long long cells, int gp, int kpg0, int cpg0) {
     dev::griddep_wait();
     dev::griddep_launch_dependents();
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < cells;
@@ -120,11 +125,18 @@ __global__ void __launch_bounds__(256) split_w_kernel(const float *__restrict__ 
         const int r = (int)(t % R); t /= R;
         const int c8 = (int)(t % (cpg / 8));
         const long long g = t / (cpg / 8);
-        const long long k = g * kpg + kk;
         float hi[8], lo[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const float v = __ldg(w + ((k * cpg + c8 * 8 + j) * R + r) * S + s);
+            const int c = c8 * 8 + j;
+            float v;
+            if (gp == 1) {
+                v = __ldg(w + (((g * kpg + kk) * cpg + c) * R + r) * S + s);
+            } else {
+                const int b = kk / kpg0;   // original group of the output, within the pack
+                const long long k0 = (g * gp + b) * kpg0 + kk % kpg0;
+                v = (c / cpg0 == b) ? __ldg(w + ((k0 * cpg0 + c % cpg0) * R + r) * S + s) : 0.f;
+            }
             hi[j] = dev::to_tf32(v);
             lo[j] = v - hi[j];
         }
@@ -789,18 +801,19 @@ cudaError_t launch_split_x(const float *x, float *xh, float *xl, int N, int C, i
 }
 
 cudaError_t launch_split_w(const float *w, float *wh, float *wl, int K, int cpg, int R, int S, int groups,
-                           cudaStream_t st) {
+                           cudaStream_t st, int gp) {
+    // groups, cpg: the GEMM's (packed) ones; the original groups hold cpg/gp channels
     const int kpg = K / groups;
     const long long cells = (long long)groups * (cpg / 8) * R * S * kpg;
     const long long blocks = std::min<long long>((cells + 255) / 256, 148LL * 8);
     return launch_ex(split_w_kernel, dim3((unsigned)blocks), dim3(256), 0, st, w, reinterpret_cast<float4 *>(wh),
-                     reinterpret_cast<uint4 *>(wl), kpg, cpg, R, S, cells);
+                     reinterpret_cast<uint4 *>(wl), kpg, cpg, R, S, cells, gp, kpg / gp, cpg / gp);
 }
 
 cudaError_t launch_igemm(const IgemmParams &p, const TensorMap *tm, int chain, dim3 grid, size_t smem,
                          cudaStream_t st) {
     if (p.fused) {   // N = 32 only
-        if (p.kpg != 32 || p.TH != kFusedTH) return cudaErrorInvalidValue;
+        if (p.kpg != 32) return cudaErrorInvalidValue;
         return chain ? launch_chain_nt<32, true>(p, tm, grid, smem, st) : launch_nt<32, 0, true>(p, tm, grid, smem, st);
     }
     if (chain) {

@@ -569,6 +569,51 @@ def test_fused_chain_matches_split_bitwise_and_oracle(oracle_mod, cfg):
                        "fused chain " + str(cfg))
 
 
+# groups with fewer than 32 output channels packed 32/kpg to a tensor-core tile
+# (block-diagonal weights): grouped, depthwise and channel-multiplier shapes
+PACKED_GEOMS = [
+    # N, C, H, W, K, R, S, stride, pad, dil, groups, bias
+    (2, 32, 20, 24, 32, 3, 3, 1, 1, 1, 4, True),      # 8 channels per group: 4 groups per tile
+    (1, 64, 16, 40, 64, 3, 3, 1, 1, 1, 8, False),     # two packed groups
+    (1, 32, 14, 28, 32, 3, 3, 1, 1, 1, 8, True),      # 4 channels per group: 8 per tile
+    (1, 32, 16, 32, 32, 3, 3, 1, 1, 1, 32, True),     # depthwise: 32 groups per tile
+    (1, 16, 16, 24, 32, 3, 3, 1, 1, 1, 16, False),    # depthwise with channel multiplier 2
+    (2, 32, 9, 140, 32, 3, 3, 1, 0, 1, 4, True),      # ragged, two column tiles
+]
+
+
+@pytest.mark.parametrize("geo", PACKED_GEOMS, ids=lambda g: "x".join(map(str, g[:11])))
+def test_packed_groups_on_tensor_cores_match_oracle(oracle_mod, geo):
+    N, C, H, W, K, R, S, st, pad, dil, g, bias = geo
+    d = inputs.conv_inputs(N, C, H, W, K, R, S, g, seed=29 + zlib.crc32(repr(geo).encode()) % 1000,
+                           x_dist="normal", bias=bias)
+    ref, acc = oracle_mod.conv2d(d["x"], d["w"], d.get("bias"), st, pad, dil, g, return_absacc=True)
+    outs = {}
+    for mode in ("igemm_fused", "igemm_split"):
+        gc.force_kernel(mode)
+        try:
+            plan = gc.plan_name(N, C, H, W, K, R, S, st, pad, dil, g)
+            assert plan.startswith("igemm") and plan.endswith("packed"), plan
+            outs[mode] = run_conv(d, st, pad, dil, g).cpu()
+        finally:
+            gc.force_kernel("auto")
+        assert_conv_close(outs[mode].numpy(), ref, acc, f"{mode} packed " + str(geo))
+    assert torch.equal(outs["igemm_fused"], outs["igemm_split"])
+    assert gc.library().gconv_device_error_status() == gc.OK
+
+
+def test_packed_groups_in_the_chain(oracle_mod):
+    d = inputs.chain_inputs(2, 32, 20, 24, 32, 3, 3, 4, 8, seed=97, bias_scale_std=1.0, affine="random")
+    gc.force_kernel("igemm")
+    try:
+        assert gc.plan_name(2, 32, 20, 24, 32, 3, 3, 1, 0, 1, 4, chain=True).endswith("packed")
+        y = _chain_dev(d, 1, 0, 1, 4, 1e-5).cpu().numpy()
+    finally:
+        gc.force_kernel("auto")
+    ref = _chain_ref(oracle_mod, d, 1, 0, 1, 4, 1e-5)
+    assert_chain_close(y, ref, d["scale"].numpy(), d["gamma"].numpy(), 1e-5, 4, "packed chain")
+
+
 _STORE_DESIGN_SCRIPT = r"""
 import sys, json
 sys.path.insert(0, sys.argv[1]); sys.path.insert(0, sys.argv[1] + "/tests")
