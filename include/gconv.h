@@ -80,7 +80,16 @@ GCONV_API gconv_status_t gconv2d_output_size(int H, int W, int R, int S, int str
  * bias: [K] device pointer or NULL for none.
  * Requires N >= 1, C, K, R, S, stride, dilation >= 1, pad >= 0,
  * groups >= 1 dividing C and K, P, Q >= 1, and every tensor smaller than
- * 2^31 elements per sample plane product (N*C*H*W, N*K*P*Q < 2^62). */
+ * 2^31 elements per sample plane product (N*C*H*W, N*K*P*Q < 2^62).
+ * Workspace: shapes that run on the tensor-core implicit GEMM keep their
+ * split weights in the library-owned workspace of the current device (see
+ * gconv_reserve_workspace); when the GEMM cannot stage x itself (rows not a
+ * multiple of 16 bytes, more than 32 output channels per group, ...) the
+ * workspace also holds two padded copies of x, about 2 * N*C*(H+pad)*(W+pad)
+ * floats (about 540 MB for x[8,32,512,512]).  gconv2d_chain_workspace_size
+ * and gconv2d_plan_name report what a shape needs.  Calls on different
+ * streams that can overlap on the GPU share that workspace and must be
+ * ordered by the caller; calls on one stream are always safe. */
 GCONV_API gconv_status_t gconv2d_fwd(const float *x, const float *w, const float *bias,
                            int N, int C, int H, int W, int K, int R, int S,
                            int stride, int pad, int dilation, int groups,
@@ -180,7 +189,9 @@ GCONV_API gconv_status_t gconv2d_bias_scale_sigmoid_groupnorm_fwd_noalloc(
 /* Bytes of the fixed scratch array the allocation-free chain may use. */
 GCONV_API size_t gconv_noalloc_scratch_capacity(void);
 
-/* Bytes of workspace the fused chain needs for this shape (0 on invalid input). */
+/* Bytes of workspace the fused chain needs for this shape (0 on invalid input
+ * or when the chain's conv stage runs on the direct kernels, whose only scratch
+ * is the partial statistics: then the size of those). */
 GCONV_API size_t gconv2d_chain_workspace_size(int N, int C, int H, int W, int K, int R, int S,
                                     int stride, int pad, int dilation, int groups,
                                     int gn_groups);

@@ -495,6 +495,24 @@ def test_igemm_matches_oracle(oracle_mod, geo):
     assert gc.library().gconv_device_error_status() == gc.OK
 
 
+def test_igemm_calls_back_to_back_on_one_stream(oracle_mod):
+    """Two implicit-GEMM convolutions queued on one stream with different inputs
+    share the workspace; stream order keeps them apart (both exact to the oracle)."""
+    geo = (2, 32, 24, 36, 64, 5, 9, 1, 2, 1, 1)   # 64 output channels: the split variant (x copies in the workspace)
+    N, C, H, W, K, R, S, st, pad, dil, g = geo
+    d1 = inputs.conv_inputs(N, C, H, W, K, R, S, g, seed=4800, x_dist="normal", w_bound=0.05)
+    d2 = inputs.conv_inputs(N, C, H, W, K, R, S, g, seed=4801, x_dist="uniform01", w_bound=0.05)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        y1 = gc.conv2d(d1["x"].cuda(), d1["w"].cuda(), None, st, pad, dil, g)
+        y2 = gc.conv2d(d2["x"].cuda(), d2["w"].cuda(), None, st, pad, dil, g)
+    torch.cuda.synchronize()
+    assert gc.plan_name(N, C, H, W, K, R, S, st, pad, dil, g).startswith("igemm")
+    for d, y in ((d1, y1), (d2, y2)):
+        ref, acc = oracle_mod.conv2d(d["x"], d["w"], None, st, pad, dil, g, return_absacc=True)
+        assert_conv_close(y.cpu().numpy(), ref, acc, "back-to-back igemm")
+
+
 def test_dense_5x9_direct_path_small(oracle_mod):
     """The CUDA-core direct path on the dense asymmetric shape (the dispatcher's alternative)."""
     d = inputs.conv_inputs(1, 32, 37, 70, 64, 5, 9, 1, 78, x_dist="uniform01",
@@ -553,20 +571,23 @@ def test_fused_igemm_matches_split_bitwise_and_oracle(oracle_mod, geo):
 
 
 @pytest.mark.parametrize("cfg", [(2, 8, 40, 40, 32, 8, 1.0), (3, 8, 37, 44, 32, 2, 1.0), (2, 8, 24, 24, 32, 32, 3.0)])
-def test_fused_chain_matches_split_bitwise_and_oracle(oracle_mod, cfg):
+def test_fused_chain_matches_oracle(oracle_mod, cfg):
+    """Both operand stagings in the chain against the oracle.  (Their outputs
+    are not compared bit for bit: the fused variant tiles 6 output rows, the
+    split one 8, so the GroupNorm partial sums are rounded in other groupings.)"""
     N, C, H, W, K, gn, std = cfg
     d = inputs.chain_inputs(N, C, H, W, K, 3, 3, 1, gn, seed=90 + N * H, bias_scale_std=std, affine="random")
-    outs = {}
+    ref = _chain_ref(oracle_mod, d, 1, 0, 1, 1, 1e-5)
     for mode in ("igemm_fused", "igemm_split"):
         gc.force_kernel(mode)
         try:
-            outs[mode] = _chain_dev(d, 1, 0, 1, 1, 1e-5).cpu()
+            assert gc.plan_name(N, C, H, W, K, 3, 3, 1, 0, 1, 1, chain=True) == (
+                "igemm_tf32_bf16x_fused" if mode == "igemm_fused" else "igemm_tf32_bf16x")
+            y = _chain_dev(d, 1, 0, 1, 1, 1e-5).cpu()
         finally:
             gc.force_kernel("auto")
-    assert torch.equal(outs["igemm_fused"], outs["igemm_split"])
-    ref = _chain_ref(oracle_mod, d, 1, 0, 1, 1, 1e-5)
-    assert_chain_close(outs["igemm_fused"].numpy(), ref, d["scale"].numpy(), d["gamma"].numpy(), 1e-5, K // gn,
-                       "fused chain " + str(cfg))
+        assert_chain_close(y.numpy(), ref, d["scale"].numpy(), d["gamma"].numpy(), 1e-5, K // gn,
+                           f"{mode} chain " + str(cfg))
 
 
 # groups with fewer than 32 output channels packed 32/kpg to a tensor-core tile
