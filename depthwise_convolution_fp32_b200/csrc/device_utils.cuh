@@ -103,6 +103,13 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
 }
 
 // ---- TMA ---------------------------------------------------------------------
+// Bring a tensor map (a __grid_constant__ kernel parameter) into the
+// descriptor cache ahead of its first use; safe before griddep_wait, since
+// the map is a launch parameter, not memory another grid writes.
+__device__ __forceinline__ void prefetch_tensormap(const void *tmap) {
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
 // 3-D tiled load of one box into shared memory; completion is signalled on
 // `bar` as transaction bytes.  Out-of-bounds elements are zero-filled.  The
 // innermost coordinate times 4 bytes must be a multiple of 16.

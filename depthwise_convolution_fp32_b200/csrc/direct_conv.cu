@@ -281,6 +281,7 @@ __global__ void __launch_bounds__(256, 2)
 
     if constexpr (TMA) {
         if (tid == 0) {
+            dev::prefetch_tensormap(&tm);
             for (int b = 0; b < p.nb; ++b) dev::mbar_init(&bars[b], 1);
             dev::fence_mbar_init();
         }
@@ -557,6 +558,7 @@ __global__ void __launch_bounds__(288, KT >= 8 ? 1 : (KT >= 4 ? 2 : 3))
     const int S = p.stages;
 
     if (tid == 0) {
+        dev::prefetch_tensormap(&tm);
         for (int s = 0; s < S; ++s) {
             dev::mbar_init(&full[s], 33);       // lane 0's expect_tx + 32 cp.async arrivals
             dev::mbar_init(&empty[s], (uint32_t)n_cwarps);

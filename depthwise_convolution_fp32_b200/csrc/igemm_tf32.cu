@@ -320,6 +320,8 @@ __global__ void __launch_bounds__(ig_threads(NT, FUSED), 1)
     const uint32_t acc_cols = (uint32_t)(p.TH * NT);
 
     if (tid == 0) {
+        dev::prefetch_tensormap(&tmh);
+        if constexpr (!FUSED) dev::prefetch_tensormap(&tmc);
         for (int s = 0; s < 4; ++s) {
             // fused: an x stage is complete when every converter warp has arrived
             dev::mbar_init(&fullA[s], FUSED ? CWARPS : 1);
