@@ -679,6 +679,9 @@ def candidate_families(gc, s, chain):
     gc.force_kernel("igemm")
     if gc.plan_name(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil, s.groups, chain).startswith("igemm"):
         c.append("igemm")
+    gc.force_kernel("winograd")
+    if gc.plan_name(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil, s.groups, chain).startswith("winograd"):
+        c.append("winograd")
     gc.force_kernel("auto")
     return c
 
@@ -727,7 +730,8 @@ def write_dispatch_table(args, gc, device, l2, batches=3, per_batch=20):
                 us[name] = round(statistics.mean(t), 3)
             finally:
                 gc.force_kernel("auto")
-        best = min(us, key=us.get)
+        fastest = min(us.values())
+        best = next(n for n in cands if us[n] <= 1.01 * fastest)   # within 1%: the earlier candidate
         entries.append({"workload": wk.name, "shape": [s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil,
                                                        s.groups],
                         "chain": 1 if wk.chain else 0, "best": best, "us": us})

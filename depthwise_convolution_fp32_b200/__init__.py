@@ -146,27 +146,38 @@ def _torch():
     return _torch_mod
 
 
+_F32 = None
+
+
 def _dev(t, name, allow_none=False):
+    global _F32
     if t is None:
         if allow_none:
             return None
         raise ValueError(f"{name} is required")
-    torch = _torch()
-    if not isinstance(t, torch.Tensor):
-        raise TypeError(f"{name} must be a torch.Tensor")
-    if not (t.is_cuda and t.dtype is torch.float32 and t.is_contiguous()):
+    if _F32 is None:
+        _F32 = _torch().float32
+    try:
+        ok = t.is_cuda and t.dtype is _F32 and t.is_contiguous()
+    except AttributeError:
+        raise TypeError(f"{name} must be a torch.Tensor") from None
+    if not ok:
         raise ValueError(f"{name} must be a contiguous float32 CUDA tensor "
                          f"(got device={t.device}, dtype={t.dtype}, contiguous={t.is_contiguous()})")
     return t.data_ptr()
 
 
+_RAW_STREAM = None
+
+
 def _stream(t):
     """The raw handle of the current stream on t's device."""
-    torch = _torch()
-    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
-    if raw is not None:
-        return ctypes.c_void_p(raw(t.get_device()))
-    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+    global _RAW_STREAM
+    if _RAW_STREAM is None:
+        torch = _torch()
+        _RAW_STREAM = getattr(torch._C, "_cuda_getCurrentRawStream", None) or \
+            (lambda d: torch.cuda.current_stream(d).cuda_stream)
+    return _RAW_STREAM(t.get_device())
 
 
 def _pair(v, name):
@@ -207,19 +218,30 @@ def _output(x, out, shape):
     return out
 
 
+_FWD = None
+
+
 def conv2d(x, w, bias=None, stride=1, padding=0, dilation=1, groups=1, out=None):
     """y = conv2d(x, w) (+ bias) on the GPU; x[N,C,H,W], w[K,C/groups,R,S].
     stride, padding and dilation are ints or (h, w) pairs."""
+    global _FWD
     N, C, H, W = x.shape
     K, cpg, R, S = w.shape
-    (sh, sw), (ph, pw), (dh, dw) = _pair(stride, "stride"), _pair(padding, "padding"), _pair(dilation, "dilation")
+    if type(stride) is int and type(padding) is int and type(dilation) is int:
+        sh = sw = stride
+        ph = pw = padding
+        dh = dw = dilation
+    else:
+        (sh, sw), (ph, pw), (dh, dw) = _pair(stride, "stride"), _pair(padding, "padding"), _pair(dilation, "dilation")
     if cpg * groups != C:
         raise ValueError("w.shape[1] * groups must equal C")
     if sh == sw and ph == pw and dh == dw:
         P, Q = _out_size(H, W, R, S, sh, ph, dh)
         out = _output(x, out, (N, K, P, Q))
-        st = library().gconv2d_fwd(_dev(x, "x"), _dev(w, "w"), _dev(bias, "bias", True),
-                                   N, C, H, W, K, R, S, sh, ph, dh, groups, _dev(out, "out"), _stream(x))
+        if _FWD is None:
+            _FWD = library().gconv2d_fwd
+        st = _FWD(_dev(x, "x"), _dev(w, "w"), _dev(bias, "bias", True),
+                  N, C, H, W, K, R, S, sh, ph, dh, groups, _dev(out, "out"), _stream(x))
         if st:
             _check(st, "gconv2d_fwd")
         return out

@@ -23,7 +23,7 @@ constexpr int kBarFloats = 32;               // shared memory reserved for mbarr
 
 enum ForceMode : int {
     kForceAuto = 0, kForceDirect = 1, kForceGeneric = 2, kForceCpAsync = 3, kForceIgemm = 4,
-    kForceBlocked = 5, kForceStream = 6, kForceIgemmSplit = 7, kForceIgemmFused = 8
+    kForceBlocked = 5, kForceStream = 6, kForceIgemmSplit = 7, kForceIgemmFused = 8, kForceWinograd = 9
 };
 std::atomic<int> g_force{kForceAuto};
 std::atomic<int> g_force_kt{0};   // channels per thread forced for the direct kernels (0: planner's rule)
@@ -70,7 +70,7 @@ gconv_status_t make_shape(Shape &s, int N, int C, int H, int W, int K, int R, in
 // at build time): the fastest of the streaming direct kernel, the blocked
 // direct kernel and the implicit GEMM, with the direct kernels' channels per
 // thread, timed per shape; shapes not in the table follow the planner's rules.
-enum TableFamily : int { kTabStream = 1, kTabBlocked = 2, kTabIgemm = 3 };
+enum TableFamily : int { kTabStream = 1, kTabBlocked = 2, kTabIgemm = 3, kTabWinograd = 4 };
 struct DispatchEntry {
     int key[12];   // N, C, H, W, K, R, S, stride, pad, dilation, groups, chain
     int family;
@@ -439,6 +439,66 @@ bool plan_stream(const Shape &s, int geom, bool x_vec, DirectPlan &pl, int kt_re
     pl.grid = dim3(0);
     pl.stream = 1;
     return true;
+}
+
+// Winograd F(2x2, 3x3) plan: 3x3, stride 1, dilation 1, equal padding on both
+// axes, at least 2 channels per group and per thread (KT = 4, else 2).
+struct WinoPlan {
+    WinoParams prm;
+    int KT;
+    dim3 grid;
+    int threads;
+    size_t smem;
+};
+
+bool plan_winograd(const Shape &s, WinoPlan &pl) {
+    if (s.R != 3 || s.S != 3 || s.stride != 1 || s.dil != 1 || !s.square() || s.cpg < 2) return false;
+    const int KT = s.kpg % 4 == 0 ? 4 : (s.kpg % 2 == 0 ? 2 : 0);
+    if (!KT) return false;
+    WinoParams &p = pl.prm;
+    std::memset(&p, 0, sizeof(p));
+    int TX = std::min(16, (s.Q + 1) / 2), TY = std::min(8, (s.P + 1) / 2);
+    const int m = s.kpg / KT;
+    int KZ = 1;
+    auto smem_of = [&](int tx, int ty, int kz) {
+        const size_t u = (size_t)s.cpg * 16 * kz * KT;
+        return (u + (size_t)s.cpg * (2 * ty + 2) * (2 * tx + 2)) * sizeof(float);
+    };
+    for (;;) {
+        KZ = 1;
+        for (int z = 1; z <= m; ++z)
+            if (m % z == 0 && TX * TY * z <= 256 && smem_of(TX, TY, z) <= 100 * 1024) KZ = z;
+        if (smem_of(TX, TY, KZ) <= 227 * 1024) break;
+        if (TY > 1) TY = (TY + 1) / 2;
+        else if (TX > 1) TX = (TX + 1) / 2;
+        else return false;
+    }
+    p.N = s.N; p.C = s.C; p.H = s.H; p.W = s.W; p.K = s.K; p.P = s.P; p.Q = s.Q; p.pad = s.pad;
+    p.cpg = s.cpg; p.kpg = s.kpg; p.groups = s.groups;
+    p.TX = TX; p.TY = TY; p.KZ = KZ; p.KB = KZ * KT;
+    p.n_qt = ceil_div(s.Q, 2 * TX);
+    p.n_pt = ceil_div(s.P, 2 * TY);
+    p.n_kb = s.kpg / p.KB;
+    p.pitch = 2 * TX + 2;
+    p.u_floats = s.cpg * 16 * p.KB;
+    const long long gx = (long long)p.n_qt * p.n_pt, gy = (long long)s.groups * p.n_kb;
+    if (gx > 0x7fffffffLL || gy > 65535 || s.N > 65535) return false;
+    pl.KT = KT;
+    pl.grid = dim3((unsigned)gx, (unsigned)gy, (unsigned)s.N);
+    pl.threads = (TX * TY * KZ + 31) / 32 * 32;
+    pl.smem = smem_of(TX, TY, KZ);
+    return true;
+}
+
+// Whether the dispatcher runs a shape on the Winograd kernel: forced, or
+// measured fastest (the table); never by rule.
+bool use_winograd(const Shape &s, bool chain) {
+    const int force = g_force.load(std::memory_order_relaxed);
+    if (chain) return false;
+    if (force == kForceWinograd) return true;
+    if (force != kForceAuto) return false;
+    const DispatchEntry *e = table_choice(s, false);
+    return e && e->family == kTabWinograd;
 }
 
 // Direct-kernel plan for the current forcing mode: in automatic mode the
@@ -815,7 +875,7 @@ bool igemm_plan_for_pointer(const Shape &s, bool chain, int gn_groups, const flo
 bool use_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     const int force = g_force.load(std::memory_order_relaxed);
     if (force == kForceDirect || force == kForceGeneric || force == kForceCpAsync || force == kForceBlocked ||
-        force == kForceStream)
+        force == kForceStream || force == kForceWinograd)
         return false;
     // groups narrower than the tensor path's 32 output channels run packed
     const int gp = igemm_pack(s);
@@ -991,6 +1051,19 @@ gconv_status_t conv_fwd_shape(const Shape &s, const float *x, const float *w, co
         return run_igemm(s, ig, x, w, bias, nullptr, 0, nullptr, nullptr, 0.f, y, ws, stream);
     }
     if (force_is_igemm()) return GCONV_ERR_UNSUPPORTED;
+    if (use_winograd(s, false)) {
+        WinoPlan wp;
+        if (!plan_winograd(s, wp)) {
+            if (g_force.load(std::memory_order_relaxed) == kForceWinograd) return GCONV_ERR_UNSUPPORTED;
+        } else {
+            WinoParams &q = wp.prm;
+            q.x = x; q.w = w; q.bias = bias; q.y = y;
+            q.aff_scale = aff_scale; q.clamp = clamp; q.lo = lo; q.hi = hi;
+            q.vec_out = (s.Q % 2 == 0) && (reinterpret_cast<uintptr_t>(y) & 7u) == 0;
+            return launch_winograd(q, wp.KT, wp.grid, wp.threads, wp.smem, stream) == cudaSuccess ? GCONV_OK
+                                                                                               : GCONV_ERR_CUDA;
+        }
+    }
     DirectPlan pl;
     const bool x_vec = (s.W % 4 == 0) && aligned16(x);
     if (!cached_direct_plan(s, x_vec, pl)) return GCONV_ERR_UNSUPPORTED;
@@ -1091,8 +1164,10 @@ gconv_status_t gconv_force_kernel(const char *name) {
     else if (!std::strcmp(fam, "direct_stream")) mode = kForceStream;
     else if (!std::strcmp(fam, "igemm_split")) mode = kForceIgemmSplit;
     else if (!std::strcmp(fam, "igemm_fused")) mode = kForceIgemmFused;
+    else if (!std::strcmp(fam, "winograd")) mode = kForceWinograd;
     else return GCONV_ERR_INVALID_ARG;
-    if (kt && (mode == kForceAuto || mode == kForceIgemm || mode == kForceIgemmSplit || mode == kForceIgemmFused))
+    if (kt && (mode == kForceAuto || mode == kForceIgemm || mode == kForceIgemmSplit || mode == kForceIgemmFused ||
+               mode == kForceWinograd))
         return GCONV_ERR_INVALID_ARG;
     g_force = mode;
     g_force_kt = kt;
@@ -1107,6 +1182,9 @@ const char *gconv2d_plan_name(int N, int C, int H, int W, int K, int R, int S, i
     if (st != GCONV_OK) return "unsupported";
     IgemmPlan ig;
     if (use_igemm(s, chain != 0, chain ? s.K : 1, ig)) return igemm_name(ig);
+    WinoPlan wp;
+    if (use_winograd(s, chain != 0) && plan_winograd(s, wp)) return "winograd_f2x2_3x3";
+    if (g_force.load(std::memory_order_relaxed) == kForceWinograd) return "unsupported";
     DirectPlan pl;
     int gn = 1;
     if (!choose_direct(s, chain != 0, gn, s.W % 4 == 0, pl)) return "unsupported";
@@ -1139,6 +1217,9 @@ const char *gconv2d_plan_name_ex(int N, int C, int H, int W, int K, int R, int S
     if (st != GCONV_OK) return "unsupported";
     IgemmPlan ig;
     if (use_igemm(s, false, 1, ig)) return igemm_name(ig);
+    WinoPlan wp;
+    if (use_winograd(s, false) && plan_winograd(s, wp)) return "winograd_f2x2_3x3";
+    if (g_force.load(std::memory_order_relaxed) == kForceWinograd) return "unsupported";
     DirectPlan pl;
     if (!choose_direct(s, false, 1, s.W % 4 == 0, pl)) return "unsupported";
     if (pl.stream) return geom_name_stream(pl.geom);
@@ -1196,7 +1277,7 @@ gconv_status_t gconv2d_bias_scale_sigmoid_groupnorm_fwd(const float *x, const fl
     IgemmPlan ig;
     if (use_igemm(s, true, gn_groups, ig) && igemm_plan_for_pointer(s, true, gn_groups, x, ig))
         return run_chain_igemm(s, ig, x, w, bias, scale, gn_groups, gamma, beta, eps, y, stream);
-    if (force_is_igemm()) return GCONV_ERR_UNSUPPORTED;
+    if (force_is_igemm() || g_force.load(std::memory_order_relaxed) == kForceWinograd) return GCONV_ERR_UNSUPPORTED;
     DirectPlan pl;
     const bool x_vec = (s.W % 4 == 0) && aligned16(x);
     if (!choose_direct(s, true, gn_groups, x_vec, pl)) return GCONV_ERR_UNSUPPORTED;

@@ -120,6 +120,23 @@ cudaError_t launch_wait_timeout_probe(unsigned spins, cudaStream_t stream);
 int direct_rpt(int KT);   // rows per thread the variant with KT uses
 int direct_fast_window_chunks(int geom);   // 16-byte chunks one thread reads per row
 
+// ---- Winograd F(2x2, 3x3) on the CUDA cores ---------------------------------
+struct WinoParams {
+    const float *x, *w, *bias;
+    float *y;
+    const float *aff_scale;   // affine + clamp epilogue: null = 1
+    int clamp;
+    float lo, hi;
+    int N, C, H, W, K, P, Q, pad, cpg, kpg, groups;
+    int TX, TY;               // Winograd tiles (2x2 outputs) per CTA along q and p
+    int KZ, KB;               // channel slices of KT per CTA, KB = KZ*KT output channels
+    int n_qt, n_pt, n_kb;
+    int pitch;                // floats per staged row (2*TX + 2)
+    int u_floats;             // floats of the transformed filters [cpg][16][KB]
+    int vec_out;              // y rows 8-byte aligned and Q even: float2 stores
+};
+cudaError_t launch_winograd(const WinoParams &p, int KT, dim3 grid, int threads, size_t smem, cudaStream_t st);
+
 // ---- implicit GEMM on tcgen05 (tf32 main term + bf16 cross terms) ----------
 struct IgemmParams {
     const float4 *wh, *wl;     // split weights [g][cpg/8][r][s][2][kpg][4]

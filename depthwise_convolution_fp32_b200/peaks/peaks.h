@@ -12,12 +12,17 @@
  * 3 timing failed, 4 a bounded wait in the MMA kernel gave up. */
 #ifndef GCONV_PEAKS_H_
 #define GCONV_PEAKS_H_
+#if defined(__GNUC__)
+#define GPEAKS_API __attribute__((visibility("default")))
+#else
+#define GPEAKS_API
+#endif
 #ifdef __cplusplus
 extern "C" {
 #endif
-int gpeaks_ffma(int iters, double *ms, double *flops);
-int gpeaks_mma_tf32(int iters, double *ms, double *flops);
-int gpeaks_mma_bf16(int iters, double *ms, double *flops);
+GPEAKS_API int gpeaks_ffma(int iters, double *ms, double *flops);
+GPEAKS_API int gpeaks_mma_tf32(int iters, double *ms, double *flops);
+GPEAKS_API int gpeaks_mma_bf16(int iters, double *ms, double *flops);
 #ifdef __cplusplus
 }
 #endif

@@ -133,14 +133,14 @@ def test_plan_names(lib):
 
 def test_force_kernel_names(lib):
     for n in ("generic", "direct", "direct_cpasync", "direct_blocked", "direct_stream", "igemm", "igemm_split",
-              "igemm_fused", "direct_stream:kt2", "direct_blocked:kt8", "auto"):
+              "igemm_fused", "winograd", "direct_stream:kt2", "direct_blocked:kt8", "auto"):
         gc.force_kernel(n)
     gc.force_kernel("direct_blocked")
     try:
         assert gc.plan_name(4, 144, 56, 56, 144, 3, 3, 1, 1, 1, 144) == "direct_tma_3x3s1p1"
     finally:
         gc.force_kernel("auto")
-    for bad in ("cudnn", "igemm:kt4", "auto:kt2", "direct:kt3", "direct_stream:"):
+    for bad in ("cudnn", "igemm:kt4", "auto:kt2", "direct:kt3", "direct_stream:", "winograd:kt4"):
         with pytest.raises(gc.GconvError):
             gc.force_kernel(bad)
     gc.force_kernel("auto")
@@ -179,3 +179,11 @@ def test_per_axis_entry_point_validates_and_plans(lib):
     assert gc.plan_name(2, 32, 24, 36, 64, 5, 9, 1, (2, 4), 1, 1).startswith("igemm_tf32_bf16x")
     assert gc.plan_name(4, 144, 56, 56, 144, 3, 3, (1, 1), (1, 1), (1, 1), 144) == \
         gc.plan_name(4, 144, 56, 56, 144, 3, 3, 1, 1, 1, 144)
+
+
+def test_peaks_library_exports_its_microbenchmarks():
+    """The benchmark's roofline microbenchmarks build as their own library
+    (not part of the C ABI) and export their three entry points."""
+    lib = ctypes.CDLL(build.build_peaks())
+    for name in ("gpeaks_ffma", "gpeaks_mma_tf32", "gpeaks_mma_bf16"):
+        assert hasattr(lib, name), name

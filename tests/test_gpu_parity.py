@@ -635,6 +635,53 @@ def test_packed_groups_in_the_chain(oracle_mod):
     assert_chain_close(y, ref, d["scale"].numpy(), d["gamma"].numpy(), 1e-5, 4, "packed chain")
 
 
+# Winograd F(2x2, 3x3) on the CUDA cores: same convolution, 16 multiplies per
+# 2x2 tile and input channel; its FP32 error stays inside the conv bound
+WINO_GEOMS = [
+    # N, C, H, W, K, R, S, stride, pad, dil, groups, bias
+    (2, 32, 20, 24, 32, 3, 3, 1, 1, 1, 4, True),      # 8 channels per group (the FP32-bound sweep case)
+    (1, 64, 17, 23, 64, 3, 3, 1, 1, 1, 8, False),     # odd sizes: ragged 2x2 tiles
+    (1, 16, 9, 13, 32, 3, 3, 1, 0, 1, 2, True),       # pad 0, channel multiplier 2
+    (2, 8, 33, 40, 8, 3, 3, 1, 1, 1, 1, False),       # dense
+    (1, 24, 15, 14, 48, 3, 3, 1, 2, 1, 3, True),      # pad 2
+    (1, 8, 1, 9, 4, 3, 3, 1, 1, 1, 2, False),         # one output row, 2 channels per thread
+    (4, 512, 28, 28, 512, 3, 3, 1, 1, 1, 64, False),  # a sweep shape (cpg 8)
+]
+
+
+@pytest.mark.parametrize("geo", WINO_GEOMS, ids=lambda g: "x".join(map(str, g[:11])))
+def test_winograd_matches_oracle(oracle_mod, geo):
+    N, C, H, W, K, R, S, st, pad, dil, g, bias = geo
+    d = inputs.conv_inputs(N, C, H, W, K, R, S, g, seed=31 + zlib.crc32(repr(geo).encode()) % 1000,
+                           x_dist="normal", bias=bias)
+    gc.force_kernel("winograd")
+    try:
+        assert gc.plan_name(N, C, H, W, K, R, S, st, pad, dil, g) == "winograd_f2x2_3x3"
+        full_check(oracle_mod, d, st, pad, dil, g, "winograd " + str(geo))
+    finally:
+        gc.force_kernel("auto")
+
+
+def test_winograd_affine_clamp_and_unsupported():
+    d = inputs.conv_inputs(2, 32, 16, 20, 32, 3, 3, 4, seed=4900, x_dist="normal")
+    x, w = d["x"].cuda(), d["w"].cuda()
+    sc = torch.rand(32, device="cuda") + 0.5
+    sh = torch.randn(32, device="cuda")
+    ref = gc.conv2d_affine_clamp(x, w, sc, sh, 0.0, 6.0, 1, 1, 1, 4)
+    gc.force_kernel("winograd")
+    try:
+        y = gc.conv2d_affine_clamp(x, w, sc, sh, 0.0, 6.0, 1, 1, 1, 4)
+        torch.cuda.synchronize()
+        # depthwise (one channel per group) and stride 2 are not Winograd shapes: refused, not rerouted
+        assert gc.plan_name(1, 8, 16, 16, 8, 3, 3, 1, 1, 1, 8) == "unsupported"
+        with pytest.raises(gc.GconvError) as e:
+            gc.conv2d(x, w, None, 2, 1, 1, 4)
+        assert e.value.status == gc.ERR_UNSUPPORTED
+    finally:
+        gc.force_kernel("auto")
+    assert float((y - ref).abs().max()) < 1e-3 and float(y.min()) >= 0 and float(y.max()) <= 6
+
+
 _STORE_DESIGN_SCRIPT = r"""
 import sys, json
 sys.path.insert(0, sys.argv[1]); sys.path.insert(0, sys.argv[1] + "/tests")
