@@ -665,8 +665,9 @@ def candidate_families(gc, s, chain):
     for fam in ("direct_stream", "direct_blocked"):
         if chain and fam == "direct_stream":
             continue
+        kpg = s.K // s.groups
         for kt in (1, 2, 4, 8):
-            if s.kpg % kt:
+            if kpg % kt:
                 continue
             if chain and (wl.FUSED_CHAIN.conv.K // wl.FUSED_CHAIN.gn_groups) % kt and \
                     kt % (wl.FUSED_CHAIN.conv.K // wl.FUSED_CHAIN.gn_groups):
@@ -676,9 +677,10 @@ def candidate_families(gc, s, chain):
             plan = gc.plan_name(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil, s.groups, chain)
             if plan not in ("unsupported", "invalid") and (fam != "direct_stream" or "stream" in plan):
                 c.append(name)
-    gc.force_kernel("igemm")
-    if gc.plan_name(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil, s.groups, chain).startswith("igemm"):
-        c.append("igemm")
+    for fam in ("igemm_split", "igemm_fused"):
+        gc.force_kernel(fam)
+        if gc.plan_name(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil, s.groups, chain).startswith("igemm"):
+            c.append(fam)
     gc.force_kernel("winograd")
     if gc.plan_name(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.stride, s.pad, s.dil, s.groups, chain).startswith("winograd"):
         c.append("winograd")

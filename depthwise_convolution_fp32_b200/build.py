@@ -53,7 +53,7 @@ def _stale(target: str, deps: list[str]) -> bool:
 
 TABLE_JSON = os.path.join(PKG, "dispatch_table.json")
 TABLE_INC = os.path.join(BUILD_DIR, "gconv_dispatch_table.inc")
-TABLE_FAMILIES = {"direct_stream": 1, "direct_blocked": 2, "igemm": 3, "winograd": 4}
+TABLE_FAMILIES = {"direct_stream": 1, "direct_blocked": 2, "igemm_split": 3, "winograd": 4, "igemm_fused": 5}
 
 
 def write_dispatch_table() -> str:

@@ -70,7 +70,7 @@ gconv_status_t make_shape(Shape &s, int N, int C, int H, int W, int K, int R, in
 // at build time): the fastest of the streaming direct kernel, the blocked
 // direct kernel and the implicit GEMM, with the direct kernels' channels per
 // thread, timed per shape; shapes not in the table follow the planner's rules.
-enum TableFamily : int { kTabStream = 1, kTabBlocked = 2, kTabIgemm = 3, kTabWinograd = 4 };
+enum TableFamily : int { kTabStream = 1, kTabBlocked = 2, kTabIgemm = 3, kTabWinograd = 4, kTabIgemmFused = 5 };
 struct DispatchEntry {
     int key[12];   // N, C, H, W, K, R, S, stride, pad, dilation, groups, chain
     int family;
@@ -744,11 +744,13 @@ bool chain_recompute(const Shape &s) {
 }
 
 // Whether the implicit GEMM stages x raw and converts it in shared memory
-// (GCONV_IGEMM_FUSED=0/1 overrides): on by default where the fused variant fits.
+// outside the measured table (GCONV_IGEMM_FUSED=1 turns it on): off, since on
+// the chain workload the split pass plus 8-row tiles measured faster than the
+// fused variant's 6-row tiles (0.88 against 1.04 ms).
 bool igemm_fused_wanted() {
     static const int v = [] {
         const char *e = std::getenv("GCONV_IGEMM_FUSED");
-        return e ? std::atoi(e) : -1;
+        return e ? std::atoi(e) : 0;
     }();
     return v != 0;
 }
@@ -883,10 +885,12 @@ bool use_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl) {
     pl.pack = gp ? gp : 1;
     if (force == kForceIgemmFused) return plan_igemm(sp, chain, gn_groups, pl, true);
     if (force == kForceIgemmSplit) return plan_igemm(sp, chain, gn_groups, pl, false);
-    if (!(igemm_fused_wanted() && plan_igemm(sp, chain, gn_groups, pl, true)) && !plan_igemm(sp, chain, gn_groups, pl))
+    const DispatchEntry *e = force == kForceAuto ? table_choice(s, chain) : nullptr;
+    const bool fused = e ? e->family == kTabIgemmFused : igemm_fused_wanted();
+    if (!(fused && plan_igemm(sp, chain, gn_groups, pl, true)) && !plan_igemm(sp, chain, gn_groups, pl))
         return false;
     if (force == kForceIgemm) return true;
-    if (const DispatchEntry *e = table_choice(s, chain)) return e->family == kTabIgemm;
+    if (e) return e->family == kTabIgemm || e->family == kTabIgemmFused;
     // outside the table: enough reduction depth and output channels for the tensor cores to win;
     // packed groups only where measured (the table)
     return !gp && s.cpg * s.R * s.S >= 64;
