@@ -48,6 +48,10 @@
 #include "device_utils.cuh"
 #include "gconv_internal.h"
 
+#ifndef GCONV_FFMA2
+#define GCONV_FFMA2 0
+#endif
+
 namespace gconv {
 
 namespace {
@@ -144,13 +148,45 @@ __device__ __forceinline__ void fma_window(float (&acc)[RPT][kV][KT], const floa
                 if (rem < 0 || rem % g::ST != 0 || rem / g::ST >= RPT) continue;
                 const int rp = rem / g::ST;
 #pragma unroll
-                for (int s = 0; s < g::S; ++s)
+                for (int s = 0; s < g::S; ++s) {
+#if GCONV_FFMA2
+                    // paired FP32 FMAs (two per lane and instruction, each rounded
+                    // as fmaf): channel pairs when KT >= 2, else column pairs
+                    if constexpr (KT % 2 == 0) {
+#pragma unroll
+                        for (int v = 0; v < kV; ++v) {
+                            const float xv = xr[win::OFF + v * g::ST + s * g::D];
+                            const float2 xx = make_float2(xv, xv);
+#pragma unroll
+                            for (int k = 0; k < KT; k += 2) {
+                                float2 a = make_float2(acc[rp][v][k], acc[rp][v][k + 1]);
+                                a = __ffma2_rn(make_float2(wr[r * g::S + s][k], wr[r * g::S + s][k + 1]), xx, a);
+                                acc[rp][v][k] = a.x;
+                                acc[rp][v][k + 1] = a.y;
+                            }
+                        }
+                        continue;
+                    } else {
+                        const float w0 = wr[r * g::S + s][0];
+                        const float2 ww = make_float2(w0, w0);
+#pragma unroll
+                        for (int v = 0; v < kV; v += 2) {
+                            float2 a = make_float2(acc[rp][v][0], acc[rp][v + 1][0]);
+                            a = __ffma2_rn(ww, make_float2(xr[win::OFF + v * g::ST + s * g::D],
+                                                           xr[win::OFF + (v + 1) * g::ST + s * g::D]), a);
+                            acc[rp][v][0] = a.x;
+                            acc[rp][v + 1][0] = a.y;
+                        }
+                        continue;
+                    }
+#endif
 #pragma unroll
                     for (int v = 0; v < kV; ++v) {
                         const float xv = xr[win::OFF + v * g::ST + s * g::D];
 #pragma unroll
                         for (int k = 0; k < KT; ++k) acc[rp][v][k] = fmaf(wr[r * g::S + s][k], xv, acc[rp][v][k]);
                     }
+                }
             }
         }
     } else {
