@@ -239,6 +239,25 @@ __device__ __forceinline__ void tmem_ld8_pair(uint32_t ta, uint32_t tb, float (&
     }
 }
 
+// Zero 32 lanes x CW columns of TMEM starting at taddr (lane field = this
+// warp's lane quarter); completion is awaited by tmem_wait_st.
+template <int CW>
+__device__ __forceinline__ void tmem_st_zero(uint32_t taddr) {
+    static_assert(CW == 8 || CW == 16, "chunk width");
+    const uint32_t z = 0u;
+    if constexpr (CW == 16) {
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};\n" ::"r"(
+                taddr),
+            "r"(z)
+            : "memory");
+    } else {
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1};\n" ::"r"(taddr), "r"(z)
+                     : "memory");
+    }
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
 template <int CW>
 __device__ __forceinline__ void tmem_ld_pair(uint32_t ta, uint32_t tb, float (&va)[CW], float (&vb)[CW]) {
     static_assert(CW == 8 || CW == 16, "chunk width");

@@ -48,10 +48,6 @@
 #include "device_utils.cuh"
 #include "gconv_internal.h"
 
-#ifndef GCONV_FFMA2
-#define GCONV_FFMA2 0
-#endif
-
 namespace gconv {
 
 namespace {
@@ -149,9 +145,10 @@ __device__ __forceinline__ void fma_window(float (&acc)[RPT][kV][KT], const floa
                 const int rp = rem / g::ST;
 #pragma unroll
                 for (int s = 0; s < g::S; ++s) {
-#if GCONV_FFMA2
-                    // paired FP32 FMAs (two per lane and instruction, each rounded
-                    // as fmaf): channel pairs when KT >= 2, else column pairs
+                    // channel pairs: paired FP32 FMAs (two per lane and instruction,
+                    // each rounded as fmaf, so the same bits) halve the FMA issue
+                    // slots; one channel keeps scalar FMAs (its column pairs would
+                    // need register moves: measured slower)
                     if constexpr (KT % 2 == 0) {
 #pragma unroll
                         for (int v = 0; v < kV; ++v) {
@@ -166,20 +163,7 @@ __device__ __forceinline__ void fma_window(float (&acc)[RPT][kV][KT], const floa
                             }
                         }
                         continue;
-                    } else {
-                        const float w0 = wr[r * g::S + s][0];
-                        const float2 ww = make_float2(w0, w0);
-#pragma unroll
-                        for (int v = 0; v < kV; v += 2) {
-                            float2 a = make_float2(acc[rp][v][0], acc[rp][v + 1][0]);
-                            a = __ffma2_rn(ww, make_float2(xr[win::OFF + v * g::ST + s * g::D],
-                                                           xr[win::OFF + (v + 1) * g::ST + s * g::D]), a);
-                            acc[rp][v][0] = a.x;
-                            acc[rp][v + 1][0] = a.y;
-                        }
-                        continue;
                     }
-#endif
 #pragma unroll
                     for (int v = 0; v < kV; ++v) {
                         const float xv = xr[win::OFF + v * g::ST + s * g::D];

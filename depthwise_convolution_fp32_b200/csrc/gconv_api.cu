@@ -388,8 +388,14 @@ bool plan_stream(const Shape &s, int geom, bool x_vec, DirectPlan &pl, int kt_re
         return gb;
     };
     int GB = pick_gb(s.groups);
-    // enough items for about two CTAs per SM: fewer groups, rows, then slices per item
-    const long long target = 2LL * sm_count();
+    // enough items per SM (GCONV_STREAM_ITEMS_PER_SM, default 2) that the
+    // last round of items is a small part of the work: fewer groups, rows,
+    // then slices per item
+    static const int per_sm = [] {
+        const char *e = std::getenv("GCONV_STREAM_ITEMS_PER_SM");
+        return e ? std::max(1, std::atoi(e)) : 2;
+    }();
+    const long long target = (long long)per_sm * sm_count();
     auto items = [&]() { return (long long)s.N * (m / KZ) * (s.groups / GB) * n_qt * n_pt; };
     for (int guard = 0; guard < 64 && items() < target; ++guard) {
         if (GB > 1) {
@@ -784,25 +790,48 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl, bool f
     if (fused) TH = igemm_fused_th();   // the fused issue loop is compiled for it (fewer rows run it unrolled less)
     TH = std::min(TH, s.P);
     const size_t limit = 227 * 1024 - igemm_header_bytes(NT, chain);
-    const int b_bytes = 32 * s.S * NT;              // one w operand slice: S taps x 8 channels x NT
     const int COLSR = COLS + 4;                     // fused raw box: room to round the start down to 4
-    int AR = 0, a_bytes = 0, sa = 0, sb = 0, raw_bytes = 0;
-    for (; TH >= 1; --TH) {
-        AR = TH + (s.R - 1) * s.dil;               // staged rows serving every tap row
-        if (AR > 256) continue;
+    // tap rows folded into one MMA (dilation 1 along H).  GCONV_IGEMM_FOLD: 0 off,
+    // 1 (default) plain convolutions only, 2 the chain too.  The chain's GEMM is
+    // bound by its epilogue (logistic, statistics, normalisation), where the
+    // folded issue measured 2-3% slower; without that epilogue it runs 1.4x faster.
+    static const int fold_env = [] {
+        const char *e = std::getenv("GCONV_IGEMM_FOLD");
+        return e ? std::atoi(e) : 1;
+    }();
+    const bool fold = fold_env == 2 || (fold_env == 1 && !chain);
+    const int rf_pref = (fold && s.dil == 1) ? igemm_fold_rf(NT, s.R) : 1;
+    int AR = 0, a_bytes = 0, b_bytes = 0, sa = 0, sb = 0, raw_bytes = 0, RF = 1, RC = s.R;
+    // stage ring for RF folded rows and TH output rows; a folded plan keeps two
+    // x stages and double-buffered (or resident) weights, else it is not taken
+    auto fit = [&](int rf, int th) {
+        RF = rf;
+        RC = (s.R + rf - 1) / rf;
+        b_bytes = 32 * s.S * rf * NT;               // one w operand slice: S taps x RF rows x 8 channels x NT
+        AR = th + (s.R - 1) * s.dil;                // staged rows serving every tap row
+        if (AR > 256) return false;
         a_bytes = 32 * COLS * AR;                   // one x operand tile: 2 quads x AR x COLS x 16 B
         raw_bytes = fused ? 8 * AR * COLSR * 4 : 0;
         const size_t lim = limit - (size_t)raw_bytes;
+        const int slices = s.cpg / 8 * RC;
         sa = force_sa > 0 ? std::min(force_sa, 4) : 2;
         sb = force_sb > 0 ? std::min(force_sb, 4) : 4;
         // weights resident when every slice fits (they are then loaded once per CTA)
-        if (fused && s.cpg / 8 * s.R <= 4) sb = std::max(sb, s.cpg / 8 * s.R);
-        while (sb > 2 && (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes > lim) --sb;
-        while (sa > 1 && (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes > lim) --sa;
-        while (sb > 1 && (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes > lim) --sb;
-        if ((size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes <= lim && (!fused || sa == 2)) break;
+        if (fused && slices <= 4) sb = std::max(sb, slices);
+        auto bytes = [&] { return (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes; };
+        if (rf > 1) sb = std::min(sb, slices);      // no more slots than slices
+        while (sb > 2 && bytes() > lim) --sb;
+        while (sa > 1 && bytes() > lim) --sa;
+        while (sb > 1 && bytes() > lim) --sb;
+        if (bytes() > lim || (fused && sa != 2)) return false;
+        return rf == 1 || (sa >= 2 && (sb >= 2 || slices <= sb));
+    };
+    bool planned = rf_pref > 1 && fit(rf_pref, TH);
+    while (!planned && TH >= 1) {
+        planned = fit(1, TH);
+        if (!planned) --TH;
     }
-    if (TH < 1) return false;
+    if (!planned) return false;
     if (fused && (COLSR > 256 || raw_bytes <= 0)) return false;
     int tmem_cols = 32;
     while (tmem_cols < 2 * TH * NT) tmem_cols *= 2;
@@ -814,6 +843,8 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl, bool f
     p.pad = s.pad; p.dil = s.dil; p.groups = s.groups; p.cpg = s.cpg; p.kpg = s.kpg; p.P = s.P; p.Q = s.Q;
     p.pad_w = s.pw; p.dil_w = s.dw;
     p.CC8 = s.cpg / 8;
+    p.RF = RF;
+    p.RC = RC;
     p.TH = TH;
     p.COLS = COLS;
     p.Hp = (int)Hp;
@@ -826,7 +857,7 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl, bool f
     p.AR = AR;
     p.sa = sa;
     p.sb = sb;
-    p.b_resident = p.CC8 * s.R <= sb ? 1 : 0;
+    p.b_resident = p.CC8 * RC <= sb ? 1 : 0;
     p.a_bytes = a_bytes;
     p.b_bytes = b_bytes;
     p.tmem_cols = tmem_cols;
@@ -841,7 +872,7 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl, bool f
     pl.smem = igemm_header_bytes(NT, chain) + (size_t)sa * 2 * a_bytes + (size_t)sb * 2 * b_bytes + raw_bytes;
 
     const size_t xbytes = fused ? 0 : (size_t)s.N * s.C * (size_t)Hp * (size_t)Wp * sizeof(float);
-    const size_t wbytes = (size_t)s.K * s.cpg * s.R * s.S * sizeof(float);
+    const size_t wbytes = (size_t)s.K * s.cpg * RC * RF * s.S * sizeof(float);
     pl.off_xl = align256(xbytes);
     pl.off_wh = pl.off_xl + align256(xbytes);
     pl.off_wl = pl.off_wh + align256(wbytes);
@@ -939,7 +970,7 @@ gconv_status_t run_igemm(const Shape &s, IgemmPlan &pl, const float *x, const fl
     p.gn_part = chain ? reinterpret_cast<float4 *>(base + pl.off_part) : nullptr;
     if (!p.fused && launch_split_x(x, xh, xl, s.N, s.C, s.H, s.W, s.pad, s.pw, p.Hp, p.Wp, stream) != cudaSuccess)
         return GCONV_ERR_CUDA;
-    if (split_w && launch_split_w(w, wh, wl, s.K, p.cpg, s.R, s.S, p.groups, stream, pl.pack) != cudaSuccess)
+    if (split_w && launch_split_w(w, wh, wl, s.K, p.cpg, s.R, s.S, p.RF, p.groups, stream, pl.pack) != cudaSuccess)
         return GCONV_ERR_CUDA;
     // the chain either stores the logistic output and normalizes it in a
     // streaming pass (store), or runs the GEMM twice: statistics only, then the

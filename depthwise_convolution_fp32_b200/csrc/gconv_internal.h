@@ -139,13 +139,15 @@ cudaError_t launch_winograd(const WinoParams &p, int KT, dim3 grid, int threads,
 
 // ---- implicit GEMM on tcgen05 (tf32 main term + bf16 cross terms) ----------
 struct IgemmParams {
-    const float4 *wh, *wl;     // split weights [g][cpg/8][r][s][2][kpg][4]
+    const float4 *wh, *wl;     // split weights [g][cpg/8][RC][s][2][RF][kpg][4], tap rows of a chunk descending
     const float *bias, *scale; // bias may be null; scale only for the chain
     float *y;
     float4 *gn_part;           // chain only
     int N, C, H, W, K, R, S, pad, dil, groups, cpg, kpg, P, Q;   // pad, dil: H axis
     int pad_w, dil_w;          // W axis
     int CC8;                   // cpg / 8 (K-steps of 8 channels)
+    int RF;                    // filter tap rows folded into the N extent of one MMA (dilation 1)
+    int RC;                    // chunks of RF tap rows: ceil(R / RF); one weight slice each
     int TH;                    // output rows per tile (one 128-pixel M tile each)
     int AR;                    // staged x rows per channel step: TH + (R-1)*dil
     int COLS;                  // staged columns per row (>= 128 + (S-1)*dil, multiple of 16)
@@ -154,7 +156,7 @@ struct IgemmParams {
     int n_qt, n_pt;
     int n_tiles;               // N * groups * n_pt * n_qt
     int sa, sb;                // slots of the x-tile ring and of the weight-slice ring
-    int b_resident;            // 1: all CC8*R weight slices fit the ring and are loaded once per CTA
+    int b_resident;            // 1: all CC8*RC weight slices fit the ring and are loaded once per CTA
     int a_bytes, b_bytes;      // one x operand (hi or lo) tile / one w operand slice
     int tmem_cols;
     int gn_groups, kgn, slots;  // chain: partials per (image, group) = tiles per image x per-tile partials
@@ -177,6 +179,7 @@ struct IgemmParams {
 
 int igemm_supported_nt(int kpg);
 int igemm_fused_th();
+int igemm_fold_rf(int nt, int R);   // tap rows one MMA covers when the plan folds them
 size_t igemm_header_bytes(int nt, bool chain);
 // GroupNorm partials the chain epilogue writes per tile and group (one per
 // TMEM lane quarter and per channel chunk the group spans)
@@ -190,7 +193,7 @@ bool make_nc4hw4_tile_map(TensorMap *tm, const float *base, long long quads, int
 cudaError_t launch_split_x(const float *x, float *xh, float *xl, int N, int C, int H, int W, int pad_h, int pad_w,
                            int Hp, int Wp, cudaStream_t st);
 // groups, cpg: the GEMM's; gp > 1 packs gp original groups into each (block-diagonal weights)
-cudaError_t launch_split_w(const float *w, float *wh, float *wl, int K, int cpg, int R, int S, int groups,
+cudaError_t launch_split_w(const float *w, float *wh, float *wl, int K, int cpg, int R, int S, int RF, int groups,
                            cudaStream_t st, int gp = 1);
 // tm: x_hi tile map, cross-term tile map
 cudaError_t launch_igemm(const IgemmParams &p, const TensorMap *tm, int chain, dim3 grid, size_t smem,

@@ -103,9 +103,12 @@ __global__ void __launch_bounds__(256) split_x_kernel(const float *__restrict__ 
     }
 }
 
-// w[K][cpg][R][S] -> per (g, c8, r, s, output channel kk), 8 input channels:
-//   wh: [g][c8][r][s][2][kpg][4]   tf32 parts (two channel quads)
-//   wc: [g][c8][r][s][2][kpg][8]   bf16 parts: chunk 0 = bf16(w - w_hi), chunk 1 = bf16(w_hi)
+// w[K][cpg][R][S] -> per (g, c8, r, s, output channel kk), 8 input channels,
+// the tap rows taken in chunks of RF (rc = r / RF, row j = RF-1 - r % RF
+// within the chunk: descending, so that one MMA over a chunk's rows writes
+// consecutive output rows; rows past R in the last chunk are zero):
+//   wh: [g][c8][rc][s][2][RF][kpg][4]   tf32 parts (two channel quads)
+//   wc: [g][c8][rc][s][2][RF][kpg][8]   bf16 parts: chunk 0 = bf16(w - w_hi), chunk 1 = bf16(w_hi)
 // so that the bf16 MMA over K = 16 computes x_hi*w_lo + x_lo*w_hi.
 // Packed groups (gp > 1): the GEMM runs gp consecutive conv groups as one
 // group of gp*cpg input and gp*kpg output channels whose weights are block
@@ -114,7 +117,8 @@ __global__ void __launch_bounds__(256) split_x_kernel(const float *__restrict__ 
 // kpg and cpg here are the packed sizes, kpg0 and cpg0 the original ones.
 __global__ void __launch_bounds__(256) split_w_kernel(const float *__restrict__ w, float4 *__restrict__ wh,
                                                       uint4 *__restrict__ wc, int kpg, int cpg, int R, int S,
-                                                      long long cells, int gp, int kpg0, int cpg0) {
+                                                      int RF, long long cells, int gp, int kpg0, int cpg0) {
+    const int RP = (R + RF - 1) / RF * RF;   // tap rows including the zero ones
     dev::griddep_wait();
     dev::griddep_launch_dependents();
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < cells;
@@ -122,7 +126,7 @@ __global__ void __launch_bounds__(256) split_w_kernel(const float *__restrict__ 
         long long t = i;
         const int kk = (int)(t % kpg); t /= kpg;
         const int s = (int)(t % S); t /= S;
-        const int r = (int)(t % R); t /= R;
+        const int r = (int)(t % RP); t /= RP;
         const int c8 = (int)(t % (cpg / 8));
         const long long g = t / (cpg / 8);
         float hi[8], lo[8];
@@ -130,7 +134,9 @@ __global__ void __launch_bounds__(256) split_w_kernel(const float *__restrict__ 
         for (int j = 0; j < 8; ++j) {
             const int c = c8 * 8 + j;
             float v;
-            if (gp == 1) {
+            if (r >= R) {
+                v = 0.f;
+            } else if (gp == 1) {
                 v = __ldg(w + (((g * kpg + kk) * cpg + c) * R + r) * S + s);
             } else {
                 const int b = kk / kpg0;   // original group of the output, within the pack
@@ -140,14 +146,16 @@ __global__ void __launch_bounds__(256) split_w_kernel(const float *__restrict__ 
             hi[j] = dev::to_tf32(v);
             lo[j] = v - hi[j];
         }
-        // slot of (g, c8, r, s): [2][kpg] cells
-        const long long base = ((((g * (cpg / 8) + c8) * R + r) * S + s) * 2) * kpg + kk;
+        // cell of (g, c8, rc, s, quad 0, row j, kk); quad 1 is RF*kpg cells on
+        const int rc = r / RF, j = RF - 1 - r % RF;
+        const long long base = (((((g * (cpg / 8) + c8) * (RP / RF) + rc) * S + s) * 2) * RF + j) * kpg + kk;
+        const long long q1 = (long long)RF * kpg;
         wh[base] = make_float4(hi[0], hi[1], hi[2], hi[3]);
-        wh[base + kpg] = make_float4(hi[4], hi[5], hi[6], hi[7]);
+        wh[base + q1] = make_float4(hi[4], hi[5], hi[6], hi[7]);
         wc[base] = make_uint4(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]), pack_bf16x2(lo[4], lo[5]),
                               pack_bf16x2(lo[6], lo[7]));
-        wc[base + kpg] = make_uint4(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]), pack_bf16x2(hi[4], hi[5]),
-                                    pack_bf16x2(hi[6], hi[7]));
+        wc[base + q1] = make_uint4(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]), pack_bf16x2(hi[4], hi[5]),
+                                   pack_bf16x2(hi[6], hi[7]));
     }
 }
 
@@ -173,15 +181,21 @@ __host__ __device__ constexpr int ig_chunk_width(int NT) {
     return NT / (ig_epi_warps(NT) / 4) < 16 ? NT / (ig_epi_warps(NT) / 4) : 16;
 }
 
-// logistic helpers: 2^x and 1/x on the special-function unit (flush to zero)
+// 2^x on the special-function unit (flush to zero)
 __device__ __forceinline__ float ex2_ftz(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
     return y;
 }
-__device__ __forceinline__ float rcp_ftz(float x) {
+
+// Logistic 1 / (1 + 2^t): 2^t and the reciprocal on the special-function
+// unit (flush to zero).  2^t overflows to +inf for large t and 1 / inf is
+// exactly the limit 0.  (A variant with Newton-Raphson division on the FMA
+// pipe in place of the reciprocal measured slower: the epilogue is bound by
+// issue, not by the special-function unit.)
+__device__ __forceinline__ float logistic_exp2(float t) {
     float y;
-    asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(1.f + ex2_ftz(t)));
     return y;
 }
 
@@ -212,26 +226,88 @@ __device__ __forceinline__ IgTile ig_tile(const IgemmParams &p, int t) {
 // accumulator buffers of TH x NT columns.
 __host__ __device__ constexpr int ig_default_th(int NT) { return NT >= 256 ? 1 : (256 / NT < 8 ? 256 / NT : 8); }
 
+// Tap rows folded into one MMA's N extent when the planner can: as many as
+// 256 columns hold (N <= 256 for M = 128), else 1.
+__host__ __device__ constexpr int ig_fold_rf(int NT, int R) { return R < 256 / NT ? R : 256 / NT; }
+
+// MMAs of one chunk of RF filter tap rows (r0 = rc*RF ...) over one staged
+// x tile, all accumulating (the accumulators start at zero: the epilogue
+// clears what it has read).  RF = 1: for every output row i and tap column s
+// one bf16 cross-term MMA and one tf32 main-term MMA of N = NT on staged row
+// i + r0*dil.  RF > 1 (dilation 1 along H): for every staged row ir and tap
+// column s one pair whose N extent covers the chunk's tap rows r that take
+// staged row ir to an output row o = ir - r of the tile.  A chunk's weight
+// rows are stored in descending r, so those output rows are consecutive
+// accumulators in TMEM (columns o*NT ...), and the staged operand is read
+// once per (ir, s) for up to RF*NT output columns instead of once per tap
+// row.  Either way every output row receives its products in the order
+// (channel step, r, s), so the result does not depend on RF.  With TH_ > 0
+// every bound and offset is a compile-time constant once the loops unroll.
+template <int NT, int TH_, int R_, int S_, int RF_>
+__device__ __forceinline__ void ig_issue_chunk(const IgemmParams &p, int rc, uint32_t dbase, uint64_t dah,
+                                               uint64_t dal, uint64_t dbh, uint64_t dbl, int COLS) {
+    constexpr bool FIX = TH_ > 0;
+    const int TH = FIX ? TH_ : p.TH, R = FIX ? R_ : p.R, S = FIX ? S_ : p.S, RF = FIX ? RF_ : p.RF;
+    const int dil = FIX ? 1 : p.dil, dil_w = FIX ? 1 : p.dil_w;
+    constexpr uint32_t idesc = dev::idesc_tf32(128, NT);
+    constexpr uint32_t idesc_c = dev::idesc_bf16(128, NT);
+    if (RF == 1) {
+        const int arow = rc * dil;   // staged row of output row 0 for tap row rc
+#pragma unroll
+        for (int i = 0; i < TH; ++i) {
+            const uint32_t d = dbase + (uint32_t)(i * NT);
+#pragma unroll
+            for (int s = 0; s < S; ++s) {
+                // 16-byte units: staged row i + r*dil, column s*dil_w; weight tap column s
+                const uint64_t ao = (uint64_t)((i + arow) * COLS + s * dil_w);
+                const uint64_t bo = (uint64_t)(s * 2 * NT);
+                // cross terms x_hi*w_lo + x_lo*w_hi: one bf16 MMA over K = 16
+                dev::mma_bf16(d, dal + ao, dbl + bo, idesc_c, 1u);
+                // main term x_hi*w_hi: tf32 MMA over K = 8
+                dev::mma_tf32(d, dah + ao, dbh + bo, idesc, 1u);
+            }
+        }
+        return;
+    }
+    const int AR = TH + R - 1;
+    const int r0 = rc * RF, r1 = (r0 + RF < R ? r0 + RF : R) - 1;
+#pragma unroll
+    for (int ir = 0; ir < AR; ++ir) {
+        // tap rows of the chunk with 0 <= ir - r < TH, weight rows from tap hi down
+        const int hi = ir < r1 ? ir : r1;
+        const int lo = ir - TH + 1 > r0 ? ir - TH + 1 : r0;
+        if (hi < lo) continue;
+        const int n = (hi - lo + 1) * NT;
+        const uint32_t d = dbase + (uint32_t)((ir - hi) * NT);
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            const uint64_t ao = (uint64_t)(ir * COLS + s * dil_w);
+            const uint64_t bo = (uint64_t)(s * 2 * RF * NT + (r0 + RF - 1 - hi) * NT);
+            dev::mma_bf16(d, dal + ao, dbl + bo, dev::idesc_bf16(128, n), 1u);
+            dev::mma_tf32(d, dah + ao, dbh + bo, dev::idesc_tf32(128, n), 1u);
+        }
+    }
+}
+
 // MMA issuer (one thread).  For every tile and 8-channel step: wait for the
-// x tile, then per tap row r wait for its weight slice and issue, for every
-// output row i and tap s, the bf16 cross-term MMA and the tf32 main-term MMA
-// into row i's accumulator.  TH_, R_, S_ > 0 fix the loop bounds (dilation 1,
-// COLS = 128 + S_ - 1 rounded up to 16); 0 reads them from p.  Returns false
-// when a bounded wait gave up.
-template <int NT, int TH_, int R_, int S_>
+// x tile, then per chunk of RF tap rows wait for its weight slice and issue
+// its MMAs (ig_issue_chunk).  TH_, R_, S_, RF_ > 0 fix the loop bounds
+// (dilation 1, COLS = 128 + S_ - 1 rounded up to 16); 0 reads them from p.
+// Returns false when a bounded wait gave up.
+template <int NT, int TH_, int R_, int S_, int RF_>
 __device__ __forceinline__ bool ig_mma_loop(const IgemmParams &p, uint32_t tmem, const unsigned char *ringA,
                                             const unsigned char *ringB, uint32_t a_slot, uint32_t b_slot,
                                             uint64_t *fullA, uint64_t *emptyA, uint64_t *fullB, uint64_t *emptyB,
                                             uint64_t *accf, uint64_t *acce) {
-    constexpr uint32_t idesc = dev::idesc_tf32(128, NT);
-    constexpr uint32_t idesc_c = dev::idesc_bf16(128, NT);
     constexpr bool FIX = TH_ > 0;
-    const int TH = FIX ? TH_ : p.TH, R = FIX ? R_ : p.R, S = FIX ? S_ : p.S;
-    const int dil = FIX ? 1 : p.dil, dil_w = FIX ? 1 : p.dil_w;
+    const int TH = FIX ? TH_ : p.TH, R = FIX ? R_ : p.R, RF = FIX ? RF_ : p.RF;
+    const int dil = FIX ? 1 : p.dil;
     const int COLS = FIX ? (128 + S_ - 1 + 15) / 16 * 16 : p.COLS;
-    const uint32_t a_bytes = 32u * (uint32_t)COLS * (uint32_t)(TH + (R - 1) * dil);
-    const uint32_t a_lbo = a_bytes / 2;          // one channel quad / bf16 chunk apart
-    constexpr uint32_t b_lbo = NT * 16;
+    const int AR = TH + (R - 1) * dil;
+    const int RC = (R + RF - 1) / RF;
+    const uint32_t a_bytes = 32u * (uint32_t)COLS * (uint32_t)AR;
+    const uint32_t a_lbo = a_bytes / 2;                  // one channel quad / bf16 chunk apart
+    const uint32_t b_lbo = (uint32_t)(RF * NT * 16);     // the same for the weights
     const uint32_t acc_cols = (uint32_t)(TH * NT);
     int ia = 0, ib = 0, j = 0;
     for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++j) {
@@ -247,8 +323,8 @@ __device__ __forceinline__ bool ig_mma_loop(const IgemmParams &p, uint32_t tmem,
             const uint64_t dah = dev::smem_desc(xa, a_lbo, 128);
             const uint64_t dal = dev::smem_desc(xa + a_bytes, a_lbo, 128);
 #pragma unroll 1
-            for (int r = 0; r < R; ++r, ++ib) {
-                const int sb = p.b_resident ? cc8 * R + r : ib % p.sb;
+            for (int rc = 0; rc < RC; ++rc, ++ib) {
+                const int sb = p.b_resident ? cc8 * RC + rc : ib % p.sb;
                 // resident slices: loaded once, waited for on the first tile only
                 if (!p.b_resident || j == 0) {
                     if (!dev::mbar_wait_bounded(&fullB[sb], p.b_resident ? 0u : (uint32_t)((ib / p.sb) & 1)))
@@ -258,21 +334,7 @@ __device__ __forceinline__ bool ig_mma_loop(const IgemmParams &p, uint32_t tmem,
                 const unsigned char *wb = ringB + (size_t)sb * b_slot;
                 const uint64_t dbh = dev::smem_desc(wb, b_lbo, 128);
                 const uint64_t dbl = dev::smem_desc(wb + b_slot / 2, b_lbo, 128);
-#pragma unroll
-                for (int i = 0; i < TH; ++i) {
-                    const uint32_t d = dbase + (uint32_t)(i * NT);
-#pragma unroll
-                    for (int s = 0; s < S; ++s) {
-                        // 16-byte units: staged row i + r*dil, column s*dil_w
-                        const uint64_t ao = (uint64_t)((i + r * dil) * COLS + s * dil_w);
-                        const uint64_t bo = (uint64_t)(s * 2 * NT);
-                        const uint32_t acc = (cc8 > 0 || r > 0 || s > 0) ? 1u : 0u;
-                        // cross terms x_hi*w_lo + x_lo*w_hi: one bf16 MMA over K = 16
-                        dev::mma_bf16(d, dal + ao, dbl + bo, idesc_c, acc);
-                        // main term x_hi*w_hi: tf32 MMA over K = 8
-                        dev::mma_tf32(d, dah + ao, dbh + bo, idesc, 1u);
-                    }
-                }
+                ig_issue_chunk<NT, TH_, R_, S_, RF_>(p, rc, dbase, dah, dal, dbh, dbl, COLS);
                 if (!p.b_resident) dev::mma_commit(&emptyB[sb]);
             }
             dev::mma_commit(&emptyA[sa]);
@@ -349,6 +411,22 @@ __global__ void __launch_bounds__(ig_threads(NT, FUSED), 1)
     __syncthreads();
     dev::tc_fence_after();
     const uint32_t tmem = *tslot;
+    {
+        // every MMA accumulates: the epilogue warps clear both accumulator
+        // buffers once here, and afterwards each part of a buffer they have read
+        constexpr int EPW = ig_epi_warps(NT), PART = NT / (EPW / 4), CW = ig_chunk_width(NT);
+        if (warp >= 2 + CWARPS) {
+            const int ew = warp - 2 - CWARPS;
+            const uint32_t tl0 = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+            for (int c = 0; c < 2 * p.TH; ++c)
+                for (int c0 = (ew >> 2) * PART; c0 < ((ew >> 2) + 1) * PART; c0 += CW)
+                    dev::tmem_st_zero<CW>(tl0 + (uint32_t)(c * NT + c0));
+            dev::tmem_wait_st();
+        }
+        dev::tc_fence_before();
+        __syncthreads();
+        dev::tc_fence_after();
+    }
 
     dev::griddep_wait();
     dev::griddep_launch_dependents();
@@ -397,8 +475,8 @@ __global__ void __launch_bounds__(ig_threads(NT, FUSED), 1)
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 if (!ok) break;
                 if (p.b_resident && t != (int)blockIdx.x) continue;   // slices already resident
-                for (int r = 0; r < p.R; ++r, ++ib) {
-                    const int sb = p.b_resident ? cc8 * p.R + r : ib % p.sb;
+                for (int rc = 0; rc < p.RC; ++rc, ++ib) {
+                    const int sb = p.b_resident ? cc8 * p.RC + rc : ib % p.sb;
                     const int ub = p.b_resident ? 0 : ib / p.sb;
                     if (lane == 0) {
                         if (ub > 0 && !dev::mbar_wait_bounded(&emptyB[sb], (ub - 1) & 1)) ok = false;
@@ -406,7 +484,7 @@ __global__ void __launch_bounds__(ig_threads(NT, FUSED), 1)
                         if (ok) {
                             dev::mbar_arrive_expect_tx(&fullB[sb], b_slot);
                             unsigned char *wb = ringB + (size_t)sb * b_slot;
-                            const long long woff = (((long long)tl.g * p.CC8 + cc8) * p.R + r) * (p.b_bytes / 16);
+                            const long long woff = (((long long)tl.g * p.CC8 + cc8) * p.RC + rc) * (p.b_bytes / 16);
                             dev::bulk_load(wb, p.wh + woff, p.b_bytes, &fullB[sb]);
                             dev::bulk_load(wb + p.b_bytes, p.wl + woff, p.b_bytes, &fullB[sb]);
                         }
@@ -445,12 +523,17 @@ __global__ void __launch_bounds__(ig_threads(NT, FUSED), 1)
             // (dilation 1, default rows per tile): the issue loop then runs
             // back to back on constant operand offsets
             constexpr int THD = FUSED ? kFusedTH : ig_default_th(NT);
+            constexpr int F3 = ig_fold_rf(NT, 3);   // the planner's fold for 3 tap rows
             const bool d1 = p.dil == 1 && p.dil_w == 1 && p.TH == THD;
             bool ok;
-            if (d1 && p.R == 3 && p.S == 3) ok = ig_mma_loop<NT, THD, 3, 3>(p, tmem, ringA, ringB, a_slot, b_slot, fullA, emptyA, fullB, emptyB, accf, acce);
-            else if (d1 && p.R == 5 && p.S == 9) ok = ig_mma_loop<NT, THD, 5, 9>(p, tmem, ringA, ringB, a_slot, b_slot, fullA, emptyA, fullB, emptyB, accf, acce);
-            else if (d1 && p.R == 1 && p.S == 1) ok = ig_mma_loop<NT, THD, 1, 1>(p, tmem, ringA, ringB, a_slot, b_slot, fullA, emptyA, fullB, emptyB, accf, acce);
-            else ok = ig_mma_loop<NT, 0, 0, 0>(p, tmem, ringA, ringB, a_slot, b_slot, fullA, emptyA, fullB, emptyB, accf, acce);
+#define IG_LOOP(TH_, R_, S_, RF_) \
+    ig_mma_loop<NT, TH_, R_, S_, RF_>(p, tmem, ringA, ringB, a_slot, b_slot, fullA, emptyA, fullB, emptyB, accf, acce)
+            if (d1 && p.R == 3 && p.S == 3 && p.RF == F3) ok = IG_LOOP(THD, 3, 3, F3);
+            else if (d1 && p.R == 3 && p.S == 3 && p.RF == 1) ok = IG_LOOP(THD, 3, 3, 1);
+            else if (d1 && p.R == 5 && p.S == 9 && p.RF == 1) ok = IG_LOOP(THD, 5, 9, 1);
+            else if (d1 && p.R == 1 && p.S == 1) ok = IG_LOOP(THD, 1, 1, 1);
+            else ok = IG_LOOP(0, 0, 0, 0);
+#undef IG_LOOP
             if (!ok) {
                 *abort_flag = 1;
                 atomicExch(&g_igemm_error, 1);
@@ -552,6 +635,17 @@ __global__ void __launch_bounds__(ig_threads(NT, FUSED), 1)
         const long long plane = (long long)p.P * p.Q;
         // GroupNorm fragments per group (chunks of CW channels it spans)
         const int fpg = CHAIN ? (p.kgn > CW ? p.kgn / CW : 1) : 1;
+        // per-channel epilogue constants.  When a warp covers a single chunk of
+        // columns (ONE) they depend only on the conv group (and, for the chain's
+        // normalisation, the image), so they are reloaded only when those change.
+        constexpr bool ONE = PART == CW;
+        // plain: a = acc * mul + add.  chain: t = -(acc*scale + bias*scale)*log2(e)
+        // = acc * mul + add, and the logistic is 1 / (1 + 2^t) (logistic_exp2)
+        float mul[CW], add[CW];
+        // chain mode 2: y = (a - mean) * (rstd * gamma) + beta with the group's
+        // finished statistics, the same three roundings as the normalize pass
+        float nmean[CHAIN ? CW : 1], nmul[CHAIN ? CW : 1], nadd[CHAIN ? CW : 1];
+        int cur_g = -1, cur_n = -1;
         int j = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++j) {
             const IgTile tl = ig_tile(p, t);
@@ -575,31 +669,28 @@ __global__ void __launch_bounds__(ig_threads(NT, FUSED), 1)
             const uint32_t tbase = tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)buf * acc_cols;
 #pragma unroll 1
             for (int c0 = cpart * PART; c0 < (cpart + 1) * PART; c0 += CW) {
-                // plain: a = acc * mul + add.  chain: t = -(acc*scale + bias*scale)*log2(e)
-                // = acc * mul + add, and the logistic is 1 / (1 + 2^t): 2^t overflows
-                // to +inf for very negative arguments, and 1 / inf is exactly the limit 0
-                float mul[CW], add[CW];
+                const bool new_g = !ONE || tl.g != cur_g;
+                const bool new_n = new_g || tl.n != cur_n;
+                if (new_g) {
 #pragma unroll
-                for (int jj = 0; jj < CW; ++jj) {
-                    const int k = tl.g * p.kpg + c0 + jj;
-                    const float b = p.bias ? __ldg(p.bias + k) : 0.f;
-                    if constexpr (CHAIN) {
-                        const float sc = __ldg(p.scale + k);
-                        mul[jj] = -sc * kLog2e;
-                        add[jj] = -(b * sc) * kLog2e;
-                    } else {
-                        mul[jj] = p.aff_scale ? __ldg(p.aff_scale + k) : 1.f;
-                        add[jj] = b;
+                    for (int jj = 0; jj < CW; ++jj) {
+                        const int k = tl.g * p.kpg + c0 + jj;
+                        const float b = p.bias ? __ldg(p.bias + k) : 0.f;
+                        if constexpr (CHAIN) {
+                            const float sc = __ldg(p.scale + k);
+                            mul[jj] = -sc * kLog2e;
+                            add[jj] = -(b * sc) * kLog2e;
+                        } else {
+                            mul[jj] = p.aff_scale ? __ldg(p.aff_scale + k) : 1.f;
+                            add[jj] = b;
+                        }
                     }
                 }
                 float shift[GPC], s1[GPC], s2[GPC];
 #pragma unroll
                 for (int gg = 0; gg < GPC; ++gg) { shift[gg] = 0.f; s1[gg] = 0.f; s2[gg] = 0.f; }
-                // chain mode 2: y = (a - mean) * (rstd * gamma) + beta with the group's
-                // finished statistics, the same three roundings as the normalize pass
-                float nmean[CHAIN ? CW : 1], nmul[CHAIN ? CW : 1], nadd[CHAIN ? CW : 1];
                 if constexpr (CHAIN) {
-                    if (p.chain_mode == 2) {
+                    if (p.chain_mode == 2 && new_n) {
 #pragma unroll
                         for (int jj = 0; jj < CW; ++jj) {
                             const int k = tl.g * p.kpg + c0 + jj;
@@ -610,6 +701,8 @@ __global__ void __launch_bounds__(ig_threads(NT, FUSED), 1)
                         }
                     }
                 }
+                cur_g = tl.g;
+                cur_n = tl.n;
                 // output pointer of channel c0 in the current row; channels are `plane` apart
                 float *yc = ybase + (long long)c0 * plane;
                 // rows are processed two at a time so one TMEM load latency covers both
@@ -619,6 +712,9 @@ __global__ void __launch_bounds__(ig_threads(NT, FUSED), 1)
                     const bool two = i + 1 < p.TH;
                     dev::tmem_ld_pair<CW>(tbase + (uint32_t)(i * NT + c0),
                                           tbase + (uint32_t)((i + (two ? 1 : 0)) * NT + c0), vv[0], vv[1]);
+                    // read (the load has completed): clear for the tile after next
+                    dev::tmem_st_zero<CW>(tbase + (uint32_t)(i * NT + c0));
+                    if (two) dev::tmem_st_zero<CW>(tbase + (uint32_t)((i + 1) * NT + c0));
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         if (h == 1 && !two) break;
@@ -626,7 +722,7 @@ __global__ void __launch_bounds__(ig_threads(NT, FUSED), 1)
                         const bool rvalid = i + h < rows;            // warp-uniform
                         if constexpr (CHAIN) {
 #pragma unroll
-                            for (int jj = 0; jj < CW; ++jj) v[jj] = rcp_ftz(1.f + ex2_ftz(fmaf(v[jj], mul[jj], add[jj])));
+                            for (int jj = 0; jj < CW; ++jj) v[jj] = logistic_exp2(fmaf(v[jj], mul[jj], add[jj]));
                             if (p.chain_mode != 2 && rvalid && i + h == 0) {
 #pragma unroll
                                 for (int gg = 0; gg < GPC; ++gg) shift[gg] = __shfl_sync(0xffffffffu, v[gg * GW], 0);
@@ -664,6 +760,8 @@ __global__ void __launch_bounds__(ig_threads(NT, FUSED), 1)
                 }
                 if (c0 + CW >= (cpart + 1) * PART) {
                     // last TMEM read of this tile by this warp: hand the buffer back
+                    // once the clearing stores have completed
+                    dev::tmem_wait_st();
                     dev::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) dev::mbar_arrive(&acce[buf]);
@@ -802,14 +900,15 @@ cudaError_t launch_split_x(const float *x, float *xh, float *xl, int N, int C, i
                      reinterpret_cast<uint4 *>(xl), C / 8, H, W, pad_h, pad_w, Hp, Wp, cells);
 }
 
-cudaError_t launch_split_w(const float *w, float *wh, float *wl, int K, int cpg, int R, int S, int groups,
+cudaError_t launch_split_w(const float *w, float *wh, float *wl, int K, int cpg, int R, int S, int RF, int groups,
                            cudaStream_t st, int gp) {
     // groups, cpg: the GEMM's (packed) ones; the original groups hold cpg/gp channels
     const int kpg = K / groups;
-    const long long cells = (long long)groups * (cpg / 8) * R * S * kpg;
+    const int RP = (R + RF - 1) / RF * RF;
+    const long long cells = (long long)groups * (cpg / 8) * RP * S * kpg;
     const long long blocks = std::min<long long>((cells + 255) / 256, 148LL * 8);
     return launch_ex(split_w_kernel, dim3((unsigned)blocks), dim3(256), 0, st, w, reinterpret_cast<float4 *>(wh),
-                     reinterpret_cast<uint4 *>(wl), kpg, cpg, R, S, cells, gp, kpg / gp, cpg / gp);
+                     reinterpret_cast<uint4 *>(wl), kpg, cpg, R, S, RF, cells, gp, kpg / gp, cpg / gp);
 }
 
 cudaError_t launch_igemm(const IgemmParams &p, const TensorMap *tm, int chain, dim3 grid, size_t smem,
@@ -835,6 +934,7 @@ cudaError_t launch_igemm(const IgemmParams &p, const TensorMap *tm, int chain, d
 }
 
 int igemm_fused_th() { return kFusedTH; }
+int igemm_fold_rf(int nt, int R) { return ig_fold_rf(nt, R); }
 
 int read_and_clear_igemm_error() {
     int v = 0, zero = 0;

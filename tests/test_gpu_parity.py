@@ -478,6 +478,9 @@ IGEMM_GEOMS = [
     (1, 8, 6, 10, 256, 3, 3, 1, 1, 1, 1, True),       # N = 256
     (1, 24, 11, 21, 32, 3, 5, 1, 1, 1, 1, False),     # R != S, three channel steps
     (1, 8, 1, 140, 32, 1, 3, 1, 0, 1, 1, True),       # single output row
+    (1, 8, 13, 40, 32, 2, 3, 1, 0, 1, 1, True),       # two tap rows folded into one MMA
+    (1, 16, 15, 50, 32, 5, 3, 1, 2, 1, 1, False),     # 5 tap rows: too large to fold, one per MMA
+    (1, 16, 12, 30, 64, 4, 1, 1, 0, 1, 1, True),      # 4 tap rows x 64 channels: N = 256 MMAs
 ]
 
 
@@ -534,6 +537,71 @@ def test_chain_paths_agree_with_oracle(oracle_mod, mode):
         gc.force_kernel("auto")
     ref = _chain_ref(oracle_mod, d, 1, 0, 1, 1, 1e-5)
     assert_chain_close(y, ref, d["scale"].numpy(), d["gamma"].numpy(), 1e-5, 4, f"{mode} chain")
+
+
+_FOLD_SCRIPT = r"""
+import sys, json
+sys.path.insert(0, sys.argv[1])
+import numpy as np, torch
+import depthwise_convolution_fp32_b200 as gc
+from depthwise_convolution_fp32_b200 import inputs
+outs = {}
+gc.force_kernel("igemm")
+for i, geo in enumerate(json.loads(sys.argv[3])):
+    N, C, H, W, K, R, S, st, pad, dil, g, seed = geo
+    d = inputs.conv_inputs(N, C, H, W, K, R, S, g, seed=seed, x_dist="normal", bias=True)
+    y = gc.conv2d(d["x"].cuda(), d["w"].cuda(), d["bias"].cuda(), st, pad, dil, g)
+    outs[str(i)] = y.cpu().numpy()
+d = inputs.chain_inputs(2, 8, 40, 44, 32, 3, 3, 1, 8, seed=96, bias_scale_std=1.0, affine="random")
+y = gc.conv2d_bias_scale_sigmoid_groupnorm(d["x"].cuda(), d["w"].cuda(), (d["b_conv"] + d["b_extra"]).cuda(),
+                                           d["scale"].cuda(), 8, d["gamma"].cuda(), d["beta"].cuda(), 1e-5,
+                                           1, 0, 1, 1)
+outs["chain"] = y.cpu().numpy()
+np.savez(sys.argv[2], **outs)
+print("ok")
+"""
+
+FOLD_GEOMS = [
+    # N, C, H, W, K, R, S, stride, pad, dil, groups, seed
+    (2, 8, 21, 140, 32, 3, 3, 1, 1, 1, 1, 1),     # 3 tap rows x 32 channels per MMA, two column tiles
+    (1, 16, 14, 40, 64, 3, 3, 1, 0, 1, 1, 2),     # 3 x 64
+    (1, 8, 9, 18, 128, 3, 3, 1, 1, 1, 1, 3),      # 2 x 128 plus a one-row chunk
+    (1, 32, 20, 24, 32, 3, 3, 1, 1, 1, 4, 4),     # packed groups
+    (1, 8, 13, 40, 32, 2, 3, 1, 0, 1, 1, 5),      # 2 x 32
+]
+
+
+def test_igemm_folded_tap_rows_match_unfolded_bitwise(tmp_path):
+    """One MMA per (staged row, tap column) over several tap rows' weights
+    (GCONV_IGEMM_FOLD=2: plain convolutions and the chain) against one MMA per
+    tap (GCONV_IGEMM_FOLD=0).  The setting is read once per process, so each
+    runs in a child process.  Every output row receives the same products in
+    the same order, so the bits agree."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    outs = {}
+    for fold in ("0", "2"):
+        out = tmp_path / f"fold{fold}.npz"
+        env = dict(os.environ, GCONV_IGEMM_FOLD=fold)
+        r = subprocess.run([sys.executable, "-c", _FOLD_SCRIPT, root, str(out), json.dumps(FOLD_GEOMS)], env=env,
+                           capture_output=True, text=True, timeout=600)
+        assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr
+        outs[fold] = np.load(out)
+    for key in outs["0"].files:
+        assert np.array_equal(outs["0"][key], outs["2"][key]), key
+    # the default (folded plain convolutions) in this process gives the same bits too
+    gc.force_kernel("igemm")
+    try:
+        for i, geo in enumerate(FOLD_GEOMS):
+            N, C, H, W, K, R, S, st, pad, dil, g, seed = geo
+            d = inputs.conv_inputs(N, C, H, W, K, R, S, g, seed=seed, x_dist="normal", bias=True)
+            y = gc.conv2d(d["x"].cuda(), d["w"].cuda(), d["bias"].cuda(), st, pad, dil, g).cpu().numpy()
+            assert np.array_equal(y, outs["0"][str(i)]), geo
+    finally:
+        gc.force_kernel("auto")
 
 
 # ---------------------------------------------------- fused operand staging (igemm)
