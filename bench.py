@@ -952,6 +952,7 @@ def measure_sweep(gc, device, l2, hbm_peak, meas, barrier, k=20):
         torch.cuda.empty_cache()
 
     def gmean(v):
+        v = [x for x in v if x > 0]   # a shape timed at zero (e.g. under a profiler) carries no ratio
         return round(math.exp(sum(math.log(x) for x in v) / len(v)), 4) if v else None
     big = [p["frac"] for p in per if p["MB"] >= 50]
     big_hbm = [p["frac"] for p in per if p["MB"] >= 50 and p["bound"] == "hbm"]

@@ -422,7 +422,12 @@ bool plan_stream(const Shape &s, int geom, bool x_vec, DirectPlan &pl, int kt_re
     const size_t stage_bytes = (x_floats + w_floats) * sizeof(float);
     if (stage_bytes > 96 * 1024) return false;
     // about 64 KB of stages per CTA, 2 to 4 deep, so that 3 CTAs fit an SM
-    const int S = (int)std::max<size_t>(2, std::min<size_t>(4, (64 * 1024) / stage_bytes));
+    // (GCONV_STREAM_STAGES overrides).  Deeper rings for large stages (one CTA
+    // per SM, 3 stages) measured 5-18% slower on the shapes they change.
+    static const int force_stages = env_int("GCONV_STREAM_STAGES");
+    int S = (int)std::max<size_t>(2, std::min<size_t>(4, (64 * 1024) / stage_bytes));
+    if (force_stages >= 2 && force_stages <= 4 && kStreamHeaderBytes + (size_t)force_stages * stage_bytes <= 227 * 1024)
+        S = force_stages;
 
     p.N = s.N; p.C = s.C; p.H = s.H; p.W = s.W; p.K = s.K; p.R = s.R; p.S = s.S;
     p.stride = s.stride; p.pad = s.pad; p.dil = s.dil; p.groups = s.groups;
