@@ -413,8 +413,19 @@ bool plan_stream(const Shape &s, int geom, bool x_vec, DirectPlan &pl, int kt_re
     }
     const int TP = RY * RPT;
     const int KB = KT * KZ;
-    const int KBtot = GB * KB;
     const int IHt = (TP - 1) * s.stride + (s.R - 1) * s.dil + 1;
+    auto stage_of = [&](int gb) {
+        return ((size_t)gb * s.cpg * IHt * 4 * tpc + ((size_t)s.cpg * s.R * s.S * gb * KB + 31) / 32 * 32) *
+               sizeof(float);
+    };
+    // stages up to GCONV_STREAM_STAGE_KB (default 96): fewer packed groups per
+    // item beyond it
+    static const int stage_kb = [] {
+        const int v = env_int("GCONV_STREAM_STAGE_KB");
+        return v > 0 ? v : 96;
+    }();
+    while (GB > 1 && stage_of(GB) > (size_t)stage_kb * 1024) GB = pick_gb(GB - 1);
+    const int KBtot = GB * KB;
     const int planes = GB * s.cpg;
     if (IHt > 256 || planes > 256 || items() > 0x7fffffffLL) return false;
     const size_t x_floats = (size_t)planes * IHt * 4 * tpc;
