@@ -817,19 +817,22 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl, bool f
     }();
     const bool fold = fold_env == 2 || (fold_env == 1 && !chain);
     const int rf_pref = (fold && s.dil == 1) ? igemm_fold_rf(NT, s.R) : 1;
-    int AR = 0, a_bytes = 0, b_bytes = 0, sa = 0, sb = 0, raw_bytes = 0, RF = 1, RC = s.R;
+    int AR = 0, a_bytes = 0, b_bytes = 0, sa = 0, sb = 0, raw_bytes = 0, RF = 1, RC = s.R, BS = 0;
     // stage ring for RF folded rows and TH output rows; a folded plan keeps two
-    // x stages and double-buffered (or resident) weights, else it is not taken
-    auto fit = [&](int rf, int th) {
+    // x stages and double-buffered (or resident) weights, else it is not taken.
+    // bsl: one weight slice per tap column (when a whole chunk's does not fit)
+    auto fit = [&](int rf, int th, bool bsl) {
         RF = rf;
         RC = (s.R + rf - 1) / rf;
-        b_bytes = 32 * s.S * rf * NT;               // one w operand slice: S taps x RF rows x 8 channels x NT
+        BS = bsl ? 1 : 0;
+        // one w operand slice: (S or 1) tap columns x RF rows x 8 channels x NT
+        b_bytes = 32 * (bsl ? 1 : s.S) * rf * NT;
         AR = th + (s.R - 1) * s.dil;                // staged rows serving every tap row
         if (AR > 256) return false;
         a_bytes = 32 * COLS * AR;                   // one x operand tile: 2 quads x AR x COLS x 16 B
         raw_bytes = fused ? 8 * AR * COLSR * 4 : 0;
         const size_t lim = limit - (size_t)raw_bytes;
-        const int slices = s.cpg / 8 * RC;
+        const int slices = s.cpg / 8 * RC * (bsl ? s.S : 1);
         sa = force_sa > 0 ? std::min(force_sa, 4) : 2;
         sb = force_sb > 0 ? std::min(force_sb, 4) : 4;
         // weights resident when every slice fits (they are then loaded once per CTA)
@@ -842,9 +845,13 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl, bool f
         if (bytes() > lim || (fused && sa != 2)) return false;
         return rf == 1 || (sa >= 2 && (sb >= 2 || slices <= sb));
     };
-    bool planned = rf_pref > 1 && fit(rf_pref, TH);
+    // one slice per tap column (GCONV_IGEMM_FOLD_SLICES=1) measured 26% slower on
+    // the dense 5x9 workload than one MMA per tap row: the 4-slot weight ring
+    // and its per-tile reloads stall the issue; off by default
+    static const bool fold_slices = env_int("GCONV_IGEMM_FOLD_SLICES") == 1;
+    bool planned = rf_pref > 1 && (fit(rf_pref, TH, false) || (fold_slices && fit(rf_pref, TH, true)));
     while (!planned && TH >= 1) {
-        planned = fit(1, TH);
+        planned = fit(1, TH, false);
         if (!planned) --TH;
     }
     if (!planned) return false;
@@ -861,6 +868,7 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl, bool f
     p.CC8 = s.cpg / 8;
     p.RF = RF;
     p.RC = RC;
+    p.bs = BS;
     p.TH = TH;
     p.COLS = COLS;
     p.Hp = (int)Hp;
@@ -873,7 +881,7 @@ bool plan_igemm(const Shape &s, bool chain, int gn_groups, IgemmPlan &pl, bool f
     p.AR = AR;
     p.sa = sa;
     p.sb = sb;
-    p.b_resident = p.CC8 * RC <= sb ? 1 : 0;
+    p.b_resident = p.CC8 * RC * (BS ? s.S : 1) <= sb ? 1 : 0;
     p.a_bytes = a_bytes;
     p.b_bytes = b_bytes;
     p.tmem_cols = tmem_cols;

@@ -148,6 +148,7 @@ struct IgemmParams {
     int CC8;                   // cpg / 8 (K-steps of 8 channels)
     int RF;                    // filter tap rows folded into the N extent of one MMA (dilation 1)
     int RC;                    // chunks of RF tap rows: ceil(R / RF); one weight slice each
+    int bs;                    // 1: one weight slice per (chunk, tap column) instead (RF > 1 only)
     int TH;                    // output rows per tile (one 128-pixel M tile each)
     int AR;                    // staged x rows per channel step: TH + (R-1)*dil
     int COLS;                  // staged columns per row (>= 128 + (S-1)*dil, multiple of 16)

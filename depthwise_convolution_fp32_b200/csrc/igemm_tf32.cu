@@ -226,9 +226,13 @@ __device__ __forceinline__ IgTile ig_tile(const IgemmParams &p, int t) {
 // accumulator buffers of TH x NT columns.
 __host__ __device__ constexpr int ig_default_th(int NT) { return NT >= 256 ? 1 : (256 / NT < 8 ? 256 / NT : 8); }
 
-// Tap rows folded into one MMA's N extent when the planner can: as many as
-// 256 columns hold (N <= 256 for M = 128), else 1.
-__host__ __device__ constexpr int ig_fold_rf(int NT, int R) { return R < 256 / NT ? R : 256 / NT; }
+// Tap rows folded into one MMA's N extent when the planner can: the fewest
+// chunks of at most 256/NT rows (N <= 256 for M = 128), spread evenly so the
+// last chunk carries few zero rows (5 rows at NT = 64: two chunks of 3).
+__host__ __device__ constexpr int ig_fold_rf(int NT, int R) {
+    return (R + ((R + (R < 256 / NT ? R : 256 / NT) - 1) / (R < 256 / NT ? R : 256 / NT)) - 1) /
+           ((R + (R < 256 / NT ? R : 256 / NT) - 1) / (R < 256 / NT ? R : 256 / NT));
+}
 
 // MMAs of one chunk of RF filter tap rows (r0 = rc*RF ...) over one staged
 // x tile, all accumulating (the accumulators start at zero: the epilogue
@@ -289,22 +293,52 @@ __device__ __forceinline__ void ig_issue_chunk(const IgemmParams &p, int rc, uin
     }
 }
 
-// MMA issuer (one thread).  For every tile and 8-channel step: wait for the
-// x tile, then per chunk of RF tap rows wait for its weight slice and issue
-// its MMAs (ig_issue_chunk).  TH_, R_, S_, RF_ > 0 fix the loop bounds
-// (dilation 1, COLS = 128 + S_ - 1 rounded up to 16); 0 reads them from p.
-// Returns false when a bounded wait gave up.
+// The folded MMAs of one chunk (r0 = rc*RF ...) for ONE tap column s, when
+// the weights arrive as one slice per (channel step, chunk, tap column)
+// because a whole chunk's slice does not fit shared memory (p.bs).  Output row
+// o then receives its products in the order (channel step, chunk, s, r): the
+// rounding differs from one MMA per tap, within the same bound.
 template <int NT, int TH_, int R_, int S_, int RF_>
+__device__ __forceinline__ void ig_issue_tap(const IgemmParams &p, int rc, int s, uint32_t dbase, uint64_t dah,
+                                             uint64_t dal, uint64_t dbh, uint64_t dbl, int COLS) {
+    constexpr bool FIX = TH_ > 0;
+    const int TH = FIX ? TH_ : p.TH, R = FIX ? R_ : p.R, RF = FIX ? RF_ : p.RF;
+    const int dil_w = FIX ? 1 : p.dil_w;
+    const int AR = TH + R - 1;
+    const int r0 = rc * RF, r1 = (r0 + RF < R ? r0 + RF : R) - 1;
+#pragma unroll
+    for (int ir = 0; ir < AR; ++ir) {
+        const int hi = ir < r1 ? ir : r1;
+        const int lo = ir - TH + 1 > r0 ? ir - TH + 1 : r0;
+        if (hi < lo) continue;
+        const int n = (hi - lo + 1) * NT;
+        const uint32_t d = dbase + (uint32_t)((ir - hi) * NT);
+        const uint64_t ao = (uint64_t)(ir * COLS + s * dil_w);
+        const uint64_t bo = (uint64_t)((r0 + RF - 1 - hi) * NT);
+        dev::mma_bf16(d, dal + ao, dbl + bo, dev::idesc_bf16(128, n), 1u);
+        dev::mma_tf32(d, dah + ao, dbh + bo, dev::idesc_tf32(128, n), 1u);
+    }
+}
+
+// MMA issuer (one thread).  For every tile and 8-channel step: wait for the
+// x tile, then per weight slice (one per chunk of RF tap rows, or per chunk
+// and tap column when BS) wait for it and issue its MMAs (ig_issue_chunk /
+// ig_issue_tap).  TH_, R_, S_, RF_ > 0 fix the loop bounds (dilation 1,
+// COLS = 128 + S_ - 1 rounded up to 16); 0 reads them and BS from p.
+// Returns false when a bounded wait gave up.
+template <int NT, int TH_, int R_, int S_, int RF_, int BS_ = 0>
 __device__ __forceinline__ bool ig_mma_loop(const IgemmParams &p, uint32_t tmem, const unsigned char *ringA,
                                             const unsigned char *ringB, uint32_t a_slot, uint32_t b_slot,
                                             uint64_t *fullA, uint64_t *emptyA, uint64_t *fullB, uint64_t *emptyB,
                                             uint64_t *accf, uint64_t *acce) {
     constexpr bool FIX = TH_ > 0;
-    const int TH = FIX ? TH_ : p.TH, R = FIX ? R_ : p.R, RF = FIX ? RF_ : p.RF;
+    const int TH = FIX ? TH_ : p.TH, R = FIX ? R_ : p.R, RF = FIX ? RF_ : p.RF, S = FIX ? S_ : p.S;
+    const bool bs = FIX ? BS_ != 0 : p.bs != 0;
     const int dil = FIX ? 1 : p.dil;
     const int COLS = FIX ? (128 + S_ - 1 + 15) / 16 * 16 : p.COLS;
     const int AR = TH + (R - 1) * dil;
     const int RC = (R + RF - 1) / RF;
+    const int nsl = bs ? RC * S : RC;                    // weight slices per channel step
     const uint32_t a_bytes = 32u * (uint32_t)COLS * (uint32_t)AR;
     const uint32_t a_lbo = a_bytes / 2;                  // one channel quad / bf16 chunk apart
     const uint32_t b_lbo = (uint32_t)(RF * NT * 16);     // the same for the weights
@@ -322,20 +356,39 @@ __device__ __forceinline__ bool ig_mma_loop(const IgemmParams &p, uint32_t tmem,
             const unsigned char *xa = ringA + (size_t)sa * a_slot;
             const uint64_t dah = dev::smem_desc(xa, a_lbo, 128);
             const uint64_t dal = dev::smem_desc(xa + a_bytes, a_lbo, 128);
-#pragma unroll 1
-            for (int rc = 0; rc < RC; ++rc, ++ib) {
-                const int sb = p.b_resident ? cc8 * RC + rc : ib % p.sb;
-                // resident slices: loaded once, waited for on the first tile only
+            // weight slice sl of this channel step: wait for it (resident slices are
+            // loaded once and waited for on the first tile only), return its slot
+            auto take = [&](int sl, int &sb) {
+                sb = p.b_resident ? cc8 * nsl + sl : ib % p.sb;
                 if (!p.b_resident || j == 0) {
                     if (!dev::mbar_wait_bounded(&fullB[sb], p.b_resident ? 0u : (uint32_t)((ib / p.sb) & 1)))
                         return false;
                     dev::tc_fence_after();
                 }
-                const unsigned char *wb = ringB + (size_t)sb * b_slot;
-                const uint64_t dbh = dev::smem_desc(wb, b_lbo, 128);
-                const uint64_t dbl = dev::smem_desc(wb + b_slot / 2, b_lbo, 128);
-                ig_issue_chunk<NT, TH_, R_, S_, RF_>(p, rc, dbase, dah, dal, dbh, dbl, COLS);
-                if (!p.b_resident) dev::mma_commit(&emptyB[sb]);
+                return true;
+            };
+#pragma unroll 1
+            for (int rc = 0; rc < RC; ++rc) {
+                if (!bs) {
+                    int sb;
+                    if (!take(rc, sb)) return false;
+                    const unsigned char *wb = ringB + (size_t)sb * b_slot;
+                    ig_issue_chunk<NT, TH_, R_, S_, RF_>(p, rc, dbase, dah, dal, dev::smem_desc(wb, b_lbo, 128),
+                                                        dev::smem_desc(wb + b_slot / 2, b_lbo, 128), COLS);
+                    if (!p.b_resident) dev::mma_commit(&emptyB[sb]);
+                    ++ib;
+                } else {
+#pragma unroll
+                    for (int s = 0; s < S; ++s) {
+                        int sb;
+                        if (!take(rc * S + s, sb)) return false;
+                        const unsigned char *wb = ringB + (size_t)sb * b_slot;
+                        ig_issue_tap<NT, TH_, R_, S_, RF_>(p, rc, s, dbase, dah, dal, dev::smem_desc(wb, b_lbo, 128),
+                                                          dev::smem_desc(wb + b_slot / 2, b_lbo, 128), COLS);
+                        if (!p.b_resident) dev::mma_commit(&emptyB[sb]);
+                        ++ib;
+                    }
+                }
             }
             dev::mma_commit(&emptyA[sa]);
         }
@@ -475,8 +528,9 @@ __global__ void __launch_bounds__(ig_threads(NT, FUSED), 1)
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 if (!ok) break;
                 if (p.b_resident && t != (int)blockIdx.x) continue;   // slices already resident
-                for (int rc = 0; rc < p.RC; ++rc, ++ib) {
-                    const int sb = p.b_resident ? cc8 * p.RC + rc : ib % p.sb;
+                const int nsl = p.bs ? p.RC * p.S : p.RC;   // weight slices per channel step
+                for (int sl = 0; sl < nsl; ++sl, ++ib) {
+                    const int sb = p.b_resident ? cc8 * nsl + sl : ib % p.sb;
                     const int ub = p.b_resident ? 0 : ib / p.sb;
                     if (lane == 0) {
                         if (ub > 0 && !dev::mbar_wait_bounded(&emptyB[sb], (ub - 1) & 1)) ok = false;
@@ -484,7 +538,7 @@ __global__ void __launch_bounds__(ig_threads(NT, FUSED), 1)
                         if (ok) {
                             dev::mbar_arrive_expect_tx(&fullB[sb], b_slot);
                             unsigned char *wb = ringB + (size_t)sb * b_slot;
-                            const long long woff = (((long long)tl.g * p.CC8 + cc8) * p.RC + rc) * (p.b_bytes / 16);
+                            const long long woff = (((long long)tl.g * p.CC8 + cc8) * nsl + sl) * (p.b_bytes / 16);
                             dev::bulk_load(wb, p.wh + woff, p.b_bytes, &fullB[sb]);
                             dev::bulk_load(wb + p.b_bytes, p.wl + woff, p.b_bytes, &fullB[sb]);
                         }
@@ -524,13 +578,17 @@ __global__ void __launch_bounds__(ig_threads(NT, FUSED), 1)
             // back to back on constant operand offsets
             constexpr int THD = FUSED ? kFusedTH : ig_default_th(NT);
             constexpr int F3 = ig_fold_rf(NT, 3);   // the planner's fold for 3 tap rows
+            constexpr int F5 = ig_fold_rf(NT, 5);   // and for 5 (per-tap-column slices)
             const bool d1 = p.dil == 1 && p.dil_w == 1 && p.TH == THD;
             bool ok;
 #define IG_LOOP(TH_, R_, S_, RF_) \
     ig_mma_loop<NT, TH_, R_, S_, RF_>(p, tmem, ringA, ringB, a_slot, b_slot, fullA, emptyA, fullB, emptyB, accf, acce)
-            if (d1 && p.R == 3 && p.S == 3 && p.RF == F3) ok = IG_LOOP(THD, 3, 3, F3);
+            if (d1 && p.R == 3 && p.S == 3 && p.RF == F3 && !p.bs) ok = IG_LOOP(THD, 3, 3, F3);
             else if (d1 && p.R == 3 && p.S == 3 && p.RF == 1) ok = IG_LOOP(THD, 3, 3, 1);
             else if (d1 && p.R == 5 && p.S == 9 && p.RF == 1) ok = IG_LOOP(THD, 5, 9, 1);
+            else if (d1 && p.R == 5 && p.S == 9 && p.RF == F5 && p.bs)
+                ok = ig_mma_loop<NT, THD, 5, 9, F5, 1>(p, tmem, ringA, ringB, a_slot, b_slot, fullA, emptyA, fullB,
+                                                        emptyB, accf, acce);
             else if (d1 && p.R == 1 && p.S == 1) ok = IG_LOOP(THD, 1, 1, 1);
             else ok = IG_LOOP(0, 0, 0, 0);
 #undef IG_LOOP

@@ -604,6 +604,43 @@ def test_igemm_folded_tap_rows_match_unfolded_bitwise(tmp_path):
         gc.force_kernel("auto")
 
 
+_SLICES_SCRIPT = r"""
+import sys, json
+sys.path.insert(0, sys.argv[1]); sys.path.insert(0, sys.argv[1] + "/tests")
+import numpy as np, torch
+import depthwise_convolution_fp32_b200 as gc
+from depthwise_convolution_fp32_b200 import inputs
+import oracle
+from tolerance import assert_conv_close
+gc.force_kernel("igemm")
+for geo in json.loads(sys.argv[2]):
+    N, C, H, W, K, R, S, st, pad, dil, g, seed = geo
+    d = inputs.conv_inputs(N, C, H, W, K, R, S, g, seed=seed, x_dist="normal", bias=True)
+    y = gc.conv2d(d["x"].cuda(), d["w"].cuda(), d["bias"].cuda(), st, pad, dil, g).cpu().numpy()
+    ref, acc = oracle.conv2d(d["x"], d["w"], d["bias"], st, pad, dil, g, return_absacc=True)
+    assert_conv_close(y, ref, acc, "slices " + str(geo))
+print("ok")
+"""
+
+
+def test_igemm_folded_per_tap_column_slices_match_oracle():
+    """The folded GEMM with one weight slice per tap column (off by default,
+    GCONV_IGEMM_FOLD_SLICES=1, read once per process: a child process) on
+    shapes whose whole-chunk slices do not fit shared memory: 5x9 at 64
+    output channels (two chunks of 3 tap rows, one zero row) and 3x5 at 32."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    geos = [(1, 16, 12, 40, 64, 5, 9, 1, 0, 1, 1, 11), (1, 32, 9, 137, 64, 5, 9, 1, 2, 1, 1, 12),
+            (1, 24, 11, 21, 32, 3, 5, 1, 1, 1, 1, 13), (2, 32, 20, 24, 64, 7, 7, 1, 3, 1, 1, 14)]
+    env = dict(os.environ, GCONV_IGEMM_FOLD_SLICES="1")
+    r = subprocess.run([sys.executable, "-c", _SLICES_SCRIPT, root, json.dumps(geos)], env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr
+
+
 # ---------------------------------------------------- fused operand staging (igemm)
 # The fused implicit GEMM stages x raw by TMA and converts it in shared memory;
 # the conversion is the split pass's arithmetic, so both give the same bits.
