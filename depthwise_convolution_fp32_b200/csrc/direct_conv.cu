@@ -559,8 +559,11 @@ __global__ void __launch_bounds__(256, 2)
 // full load latency per tile).  Every wait is bounded; a wait that gives up
 // raises the device error flag, stops the CTA's pipeline and, before the CTA
 // exits, waits (bounded again) for the copies it has in flight.
+// Register budget: 3 CTAs per SM (72 registers) for one channel per thread;
+// 2 or more channels get 2 CTAs (96 registers), since the paired FMAs of two
+// channels spilled at 72 and measured 3-7% slower on two-channel groups.
 template <int G, int KT, int RPT, int EPI>
-__global__ void __launch_bounds__(288, KT >= 8 ? 1 : (KT >= 4 ? 2 : 3))
+__global__ void __launch_bounds__(288, KT >= 8 ? 1 : (KT >= 2 ? 2 : 3))
     direct_stream_kernel(const __grid_constant__ TensorMap tm, const DirectParams p) {
     extern __shared__ __align__(128) float smem[];
     using g = Geom<G>;
