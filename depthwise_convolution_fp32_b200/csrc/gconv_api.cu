@@ -229,8 +229,13 @@ bool plan_direct(const Shape &s, bool chain, int gn_groups, int geom, bool x_vec
     int GB = pick_gb(s.groups);
 
     // Small problems: split the work until the grid covers about two CTAs per
-    // SM (fewer groups per CTA, then fewer rows, then fewer channel slices).
-    const long long target = 2LL * sm_count();
+    // SM (GCONV_DIRECT_CTAS_PER_SM overrides): fewer groups per CTA, then fewer
+    // rows, then fewer channel slices.
+    static const int ctas_per_sm = [] {
+        const int v = env_int("GCONV_DIRECT_CTAS_PER_SM");
+        return v > 0 ? v : 2;
+    }();
+    const long long target = (long long)ctas_per_sm * sm_count();
     auto ctas = [&]() {
         return (long long)s.N * (s.kpg / (KT * KZ)) * (s.groups / GB) * n_qt * n_pt;
     };
