@@ -21,7 +21,7 @@
 // four consecutive channels in one 16-byte cell; pad zero rows on top, pad
 // zero columns on the left, zero columns up to a multiple of 16 pixels) and
 // the bf16 cross-term operand as [n][c/8][2][hp][wp][8] (same cell geometry),
-// and the weights split the same way as [g][c/8][r][s][2][kpg][4 tf32 | 8 bf16].
+// and the weights split the same way as [g][c/8][r chunk][s][2][rows][kpg][4 tf32 | 8 bf16].
 // In the tile a CTA stages ([2 channel quads][rows][cols][4], one TMA box),
 // consecutive output pixels of one row are 16 bytes apart, which is exactly
 // a K-major, no-swizzle UMMA operand with 8-row core matrices (SBO = 128 B)
@@ -34,15 +34,19 @@
 // columns, all kpg output channels of group g):
 //   warp 0 lane 0 : producer - per 8-channel step one TMA box of x_hi and one
 //                   of the cross-term operand (all staged rows and columns),
-//                   then the weight slices of the R tap rows (bulk copies;
+//                   then the weight slices of the tap-row chunks (bulk copies;
 //                   loaded once per CTA when they all fit the ring);
-//   warp 1 lane 0 : MMA issuer - for every output row i and tap (r, s) one
-//                   bf16 and one tf32 tcgen05.mma (M=128, N=kpg) into the
-//                   row's TMEM accumulator; tcgen05.commit frees the stages;
-//   other warps   : epilogue - tcgen05.ld of the accumulators, +bias, or the
-//                   chain's +bias, *scale, logistic and GroupNorm partial
-//                   statistics, coalesced stores along q; two TMEM
-//                   accumulator buffers let it overlap the next tile's MMAs.
+//   warp 1 lane 0 : MMA issuer - for every output row and tap (r, s) one bf16
+//                   and one tf32 tcgen05.mma (M=128) into the row's TMEM
+//                   accumulator; with tap rows folded (ig_issue_chunk) one
+//                   pair per staged row and tap column covers up to 256/kpg
+//                   tap rows at once (N up to 256); tcgen05.commit frees the
+//                   stages;
+//   other warps   : epilogue - tcgen05.ld of the accumulators (then cleared:
+//                   every MMA accumulates), +bias, or the chain's +bias,
+//                   *scale, logistic and GroupNorm partial statistics,
+//                   coalesced stores along q; two TMEM accumulator buffers
+//                   let it overlap the next tile's MMAs.
 #include <atomic>
 
 #include <cuda.h>
