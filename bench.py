@@ -276,7 +276,7 @@ class Workload:
                                     seed=wl.SEEDS["fused_chain"])
             self.host = d
         elif name.startswith("ring"):
-            N, C, H, W, K, R, pad, g = THRESHOLD_RING[int(name[4:])]
+            N, C, H, W, K, R, pad, g = wl.THRESHOLD_RING[int(name[4:])]
             s = wl.ConvShape(N=N, C=C, H=H, W=W, K=K, R=R, S=R, stride=1, pad=pad, groups=g)
             self.shape = s
             self.host = inputs.conv_inputs(s.N, s.C, s.H, s.W, s.K, R, R, g, 5000 + int(name[4:]),
@@ -640,20 +640,12 @@ def write_records(args, gc, device, l2, hbm_peak, meas, batches=10, per_batch=30
     print(json.dumps({"records": len(out), "file": args.records}))
 
 
-# shapes around the implicit-GEMM threshold (channels per group x taps near 64,
-# output channels per group at the tensor path's minimum of 32): x[N,C,H,W], K,
-# R=S, pad, groups
-THRESHOLD_RING = [
-    (8, 32, 56, 56, 32, 3, 1, 1), (8, 64, 56, 56, 64, 3, 1, 1), (8, 128, 28, 28, 128, 3, 1, 4),
-    (8, 16, 56, 56, 32, 3, 1, 1), (8, 8, 128, 128, 32, 3, 1, 1), (8, 64, 56, 56, 64, 1, 0, 1),
-    (8, 128, 28, 28, 128, 1, 0, 1), (8, 256, 28, 28, 256, 3, 1, 8),
-]
 
 
 def tuning_workloads():
     out = [Workload(n) for n in ("tiny_grouped", "depthwise", "fused_chain", "dense_5x9")]
     out += [Workload(f"sweep{i}") for i in range(80)]
-    for j, (N, C, H, W, K, R, pad, g) in enumerate(THRESHOLD_RING):
+    for j, (N, C, H, W, K, R, pad, g) in enumerate(wl.THRESHOLD_RING):
         out.append(Workload(f"ring{j}"))
     return out
 

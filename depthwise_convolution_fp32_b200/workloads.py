@@ -124,6 +124,15 @@ def sweep_seed(i: int) -> int:
 
 SEEDS = {"tiny_grouped": 1001, "depthwise": 1002, "fused_chain": 1004, "dense_5x9": 1005}
 
+# Shapes around the implicit-GEMM threshold (channels per group x taps near
+# 64, output channels per group at the tensor path's minimum of 32), timed for
+# the dispatch table: (N, C, H, W, K, R = S, pad, groups); seeds 5000 + index.
+THRESHOLD_RING = [
+    (8, 32, 56, 56, 32, 3, 1, 1), (8, 64, 56, 56, 64, 3, 1, 1), (8, 128, 28, 28, 128, 3, 1, 4),
+    (8, 16, 56, 56, 32, 3, 1, 1), (8, 8, 128, 128, 32, 3, 1, 1), (8, 64, 56, 56, 64, 1, 0, 1),
+    (8, 128, 28, 28, 128, 1, 0, 1), (8, 256, 28, 28, 256, 3, 1, 8),
+]
+
 
 def roofline_time_s(shape: ConvShape, hbm_gbs: float, fp32_tflops: float) -> tuple[float, str]:
     """max(bytes / HBM bandwidth, FLOPs / FP32 peak) and the binding term."""

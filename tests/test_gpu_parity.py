@@ -108,6 +108,19 @@ def sampled_check(oracle_mod, d, y_dev, stride, pad, dil, groups, what, n_random
 
 # ------------------------------------------------------------------ workloads
 
+@pytest.mark.parametrize("j", range(len(wl.THRESHOLD_RING)))
+def test_threshold_ring_default_dispatch(oracle_mod, j):
+    """The dispatch-table shapes around the implicit-GEMM threshold (several run
+    on the tensor cores with folded tap rows) through the default dispatch."""
+    N, C, H, W, K, R, pad, g = wl.THRESHOLD_RING[j]
+    d = inputs.conv_inputs(N, C, H, W, K, R, R, g, 5000 + j, x_dist="normal",
+                           w_bound=1 / math.sqrt(R * R * (C // g)))
+    y = run_conv(d, 1, pad, 1, g)
+    sampled_check(oracle_mod, d, y, 1, pad, 1, g, f"ring {j} {gc.plan_name(N, C, H, W, K, R, R, 1, pad, 1, g)}",
+                  n_random=6000, seed=j)
+    assert gc.library().gconv_device_error_status() == gc.OK
+
+
 def test_tiny_grouped_full(oracle_mod):
     s = wl.TINY_GROUPED
     d = inputs.conv_inputs(s.N, s.C, s.H, s.W, s.K, s.R, s.S, s.groups, wl.SEEDS["tiny_grouped"],
