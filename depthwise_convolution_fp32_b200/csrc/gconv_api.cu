@@ -363,9 +363,15 @@ bool plan_stream(const Shape &s, int geom, bool x_vec, DirectPlan &pl, int kt_re
     const int nch = direct_fast_window_chunks(geom);
     const int qchunks = ceil_div(s.Q, 4);
     int n_qt = ceil_div(qchunks, 32), CX = 0, tpc = 0;
+    // staged row: exactly the 16-byte chunks the item's threads read.  One TMA
+    // box per item lands at the stage base, so the row pitch needs only the
+    // box's 16-byte granularity; padding rows to 128 bytes doubled the stage of
+    // 28-column planes (36 -> 64 floats) and left one CTA per SM
+    static const int pad8 = env_int("GCONV_STREAM_PAD_ROWS");
     for (;; ++n_qt) {   // column tiles until the staged row fits one 256-element box row
         CX = ceil_div(qchunks, n_qt);
-        tpc = ((CX - 1) * s.stride + nch + 7) / 8 * 8;
+        tpc = (CX - 1) * s.stride + nch;
+        if (pad8 == 1) tpc = (tpc + 7) / 8 * 8;
         if (4 * tpc <= 256) break;
     }
     n_qt = ceil_div(qchunks, CX);
@@ -433,9 +439,10 @@ bool plan_stream(const Shape &s, int geom, bool x_vec, DirectPlan &pl, int kt_re
     const int KBtot = GB * KB;
     const int planes = GB * s.cpg;
     if (IHt > 256 || planes > 256 || items() > 0x7fffffffLL) return false;
-    const size_t x_floats = (size_t)planes * IHt * 4 * tpc;
-    const size_t w_floats = ((size_t)s.cpg * s.R * s.S * KBtot + 31) / 32 * 32;
-    const size_t stage_bytes = (x_floats + w_floats) * sizeof(float);
+    const size_t x_floats = (size_t)planes * IHt * 4 * tpc;   // 16-byte multiple: weights follow
+    // stages 128-byte aligned (the TMA destination of each item)
+    const size_t stage_floats = (x_floats + (size_t)s.cpg * s.R * s.S * KBtot + 31) / 32 * 32;
+    const size_t stage_bytes = stage_floats * sizeof(float);
     if (stage_bytes > 96 * 1024) return false;
     // about 64 KB of stages per CTA, 2 to 4 deep, so that 3 CTAs fit an SM
     // (GCONV_STREAM_STAGES overrides).  Deeper rings for large stages (one CTA
@@ -457,7 +464,7 @@ bool plan_stream(const Shape &s, int geom, bool x_vec, DirectPlan &pl, int kt_re
     p.tma = 1;
     p.n_items = (int)items();
     p.stages = S;
-    p.stage_floats = (int)(x_floats + w_floats);
+    p.stage_floats = (int)stage_floats;
     p.sw_off = (int)x_floats;
     pl.geom = geom;
     pl.KT = KT;
