@@ -444,11 +444,15 @@ bool plan_stream(const Shape &s, int geom, bool x_vec, DirectPlan &pl, int kt_re
     const size_t stage_floats = (x_floats + (size_t)s.cpg * s.R * s.S * KBtot + 31) / 32 * 32;
     const size_t stage_bytes = stage_floats * sizeof(float);
     if (stage_bytes > 96 * 1024) return false;
-    // about 64 KB of stages per CTA, 2 to 4 deep, so that 3 CTAs fit an SM
-    // (GCONV_STREAM_STAGES overrides).  Deeper rings for large stages (one CTA
-    // per SM, 3 stages) measured 5-18% slower on the shapes they change.
+    // ring of 2 to 4 stages in about 64 KB per CTA (GCONV_STREAM_RING_KB
+    // overrides, GCONV_STREAM_STAGES fixes the depth).  Larger budgets measured
+    // no better: 108 KB for the 2 CTAs per SM that two or more channels per
+    // thread allow (+0.4% on the large shapes, 6% slower on small ones), and 3
+    // stages of a large item at one CTA per SM (5-18% slower).
     static const int force_stages = env_int("GCONV_STREAM_STAGES");
-    int S = (int)std::max<size_t>(2, std::min<size_t>(4, (64 * 1024) / stage_bytes));
+    static const int ring_kb = env_int("GCONV_STREAM_RING_KB");
+    const size_t ring = (size_t)(ring_kb > 0 ? ring_kb : 64) * 1024;
+    int S = (int)std::max<size_t>(2, std::min<size_t>(4, ring / stage_bytes));
     if (force_stages >= 2 && force_stages <= 4 && kStreamHeaderBytes + (size_t)force_stages * stage_bytes <= 227 * 1024)
         S = force_stages;
 
