@@ -365,13 +365,17 @@ bool plan_stream(const Shape &s, int geom, bool x_vec, DirectPlan &pl, int kt_re
     int n_qt = ceil_div(qchunks, 32), CX = 0, tpc = 0;
     // staged row: exactly the 16-byte chunks the item's threads read.  One TMA
     // box per item lands at the stage base, so the row pitch needs only the
-    // box's 16-byte granularity; padding rows to 128 bytes doubled the stage of
-    // 28-column planes (36 -> 64 floats) and left one CTA per SM
-    static const int pad8 = env_int("GCONV_STREAM_PAD_ROWS");
+    // box's 16-byte granularity.  Padding rows to 128 bytes doubled the stage
+    // of 28-column planes (36 -> 64 floats) and left one CTA per SM; padding
+    // only where it costs at most an eighth (aligned shared loads on 112-column
+    // planes) measured no faster.  GCONV_STREAM_PAD_ROWS: 0 (default) never
+    // pad, 1 always, 2 when cheap.
+    static const int pad_rows = env_int("GCONV_STREAM_PAD_ROWS");
     for (;; ++n_qt) {   // column tiles until the staged row fits one 256-element box row
         CX = ceil_div(qchunks, n_qt);
         tpc = (CX - 1) * s.stride + nch;
-        if (pad8 == 1) tpc = (tpc + 7) / 8 * 8;
+        const int padded = (tpc + 7) / 8 * 8;
+        if (pad_rows == 1 || (pad_rows == 2 && 8 * padded <= 9 * tpc)) tpc = padded;
         if (4 * tpc <= 256) break;
     }
     n_qt = ceil_div(qchunks, CX);
