@@ -828,6 +828,13 @@ def main():
         e2e_ms, h2d, d2h = time_e2e(runner, args.steps, args.warmup, barrier)
         sync_us = time_sync_api(runner, min(args.steps, 200))
     clocks = sampler.summary(t0, t1)
+    # the same calls on one buffer set that stays in L2 (labelled L2-warm,
+    # reported beside the L2-cold headline; only when one set fits in L2)
+    warm_ms = None
+    if (wk.host["x"].numel() + wk.shape.n_out) * 4 * 2 <= l2:
+        warm = DeviceRunner(wk, device, 0)
+        warm_ms, _, _ = time_graph(warm, args.steps, args.warmup, barrier)
+        del warm
 
     ms, e2e_ms = max_over_ranks([ms, e2e_ms], device, world)
     per_step_s = ms / 1e3 / args.steps
@@ -859,6 +866,11 @@ def main():
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "roofline": roof,
+        "l2_warm": None if warm_ms is None else {
+            "us_per_step": round(warm_ms * 1e3 / args.steps, 3),
+            "GB/s": round(wk.bytes * args.steps / (warm_ms / 1e3) / 1e9, 1),
+            "note": "one buffer set reused every call (inputs and outputs resident in L2); the headline "
+                    "value is L2-cold"},
         "gpu_launches": launches * args.steps,
         "compute_peaks": dict(MEASURED_COMPUTE, note="microbenchmarks on this GPU, reported beside the "
                               "roofline denominators (alu: unit counts x clock; tensor: bf16 GEMM peak x "
