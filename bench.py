@@ -397,13 +397,13 @@ def time_graph(runner: DeviceRunner, steps: int, warmup: int, dist_barrier):
 def time_e2e(runner: DeviceRunner, steps: int, warmup: int, dist_barrier):
     """Per step: pinned host-to-device copy of the step's inputs (x and w), the
     call through the public API, and the device-to-host copy of its output.
-    Steps are pipelined over three streams with double-buffered device and
-    pinned host buffers, so step i+1's upload, step i's call and step i-1's
-    download overlap (the two copy directions have their own copy engines);
+    Steps are pipelined over three streams with a ring of device and pinned
+    host buffers (4 deep), so uploads, calls and downloads of neighbouring
+    steps overlap (the two copy directions have their own copy engines);
     every step still moves all of its bytes inside the timed region."""
     torch = runner.torch
     h = runner.wk.host
-    nb = 2
+    nb = int(os.environ.get("GCONV_E2E_BUFFERS", "4"))   # pipeline depth (2: 71, 4: 82 GB/s on the headline)
     x_host = [h["x"].pin_memory() for _ in range(nb)]
     w_host = [h["w"].pin_memory() for _ in range(nb)]
     y_host = [torch.empty(runner.ys[0].shape, dtype=torch.float32).pin_memory() for _ in range(nb)]
