@@ -398,12 +398,15 @@ def time_e2e(runner: DeviceRunner, steps: int, warmup: int, dist_barrier):
     """Per step: pinned host-to-device copy of the step's inputs (x and w), the
     call through the public API, and the device-to-host copy of its output.
     Steps are pipelined over three streams with a ring of device and pinned
-    host buffers (4 deep), so uploads, calls and downloads of neighbouring
-    steps overlap (the two copy directions have their own copy engines);
+    host buffers (4 deep, 2 for steps over 64 MB), so uploads, calls and
+    downloads of neighbouring steps overlap (the two copy directions have their own copy engines);
     every step still moves all of its bytes inside the timed region."""
     torch = runner.torch
     h = runner.wk.host
-    nb = int(os.environ.get("GCONV_E2E_BUFFERS", "4"))   # pipeline depth (2: 71, 4: 82 GB/s on the headline)
+    # pipeline depth: 4 for small steps (71 -> 82 GB/s on the headline), 2 when a
+    # step moves more than 64 MB (the pinned host buffers would reach gigabytes)
+    step_bytes = (h["x"].numel() + runner.ys[0].numel()) * 4
+    nb = int(os.environ.get("GCONV_E2E_BUFFERS", "4" if step_bytes <= 64 * 2**20 else "2"))
     x_host = [h["x"].pin_memory() for _ in range(nb)]
     w_host = [h["w"].pin_memory() for _ in range(nb)]
     y_host = [torch.empty(runner.ys[0].shape, dtype=torch.float32).pin_memory() for _ in range(nb)]
