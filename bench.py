@@ -410,8 +410,9 @@ def time_e2e(runner: DeviceRunner, steps: int, warmup: int, dist_barrier):
     x_host = [h["x"].pin_memory() for _ in range(nb)]
     w_host = [h["w"].pin_memory() for _ in range(nb)]
     y_host = [torch.empty(runner.ys[0].shape, dtype=torch.float32).pin_memory() for _ in range(nb)]
-    x_dev = [runner.xs[b % runner.n_sets] for b in range(nb)]
-    y_dev = [runner.ys[b % runner.n_sets] for b in range(nb)]
+    # one device buffer per ring slot (the rotating pool may hold a single set)
+    x_dev = [torch.empty_like(runner.xs[0]) for _ in range(nb)]
+    y_dev = [torch.empty_like(runner.ys[0]) for _ in range(nb)]
     w_dev = [torch.empty_like(runner.w) for _ in range(nb)]
     s_in, s_cp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     ev_in = [torch.cuda.Event() for _ in range(nb)]
