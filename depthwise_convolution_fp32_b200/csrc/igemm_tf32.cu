@@ -234,8 +234,9 @@ __host__ __device__ constexpr int ig_default_th(int NT) { return NT >= 256 ? 1 :
 // chunks of at most 256/NT rows (N <= 256 for M = 128), spread evenly so the
 // last chunk carries few zero rows (5 rows at NT = 64: two chunks of 3).
 __host__ __device__ constexpr int ig_fold_rf(int NT, int R) {
-    return (R + ((R + (R < 256 / NT ? R : 256 / NT) - 1) / (R < 256 / NT ? R : 256 / NT)) - 1) /
-           ((R + (R < 256 / NT ? R : 256 / NT) - 1) / (R < 256 / NT ? R : 256 / NT));
+    const int most = R < 256 / NT ? R : 256 / NT;   // tap rows one MMA can cover
+    const int chunks = (R + most - 1) / most;
+    return (R + chunks - 1) / chunks;
 }
 
 // MMAs of one chunk of RF filter tap rows (r0 = rc*RF ...) over one staged
