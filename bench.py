@@ -16,7 +16,9 @@ Timing boundaries (the "GroupConv Atlas" distinguishes both):
   value      device events around a CUDA graph holding exactly K captured
              calls; inputs stay resident in HBM; consecutive calls rotate
              through a pool of input/output buffers larger than 4 x L2, so no
-             call finds its data in L2.
+             call finds its data in L2.  The two events are record nodes
+             inside the graph, around the K calls, so the graph's own launch
+             and completion (a fixed 7-9 us per replay) stay outside.
   e2e        per step: pinned-host -> device copy of the inputs, the call,
              device -> pinned-host copy of the output, timed with events on
              the same stream.
@@ -361,36 +363,52 @@ class DeviceRunner:
         return y
 
 
+class TimedGraph:
+    """`n` calls of `body(i)` captured in one CUDA graph between two event
+    record nodes, so the events bracket the calls' device time and not the
+    graph's own launch and completion (about 7-9 us per replay, which would
+    otherwise add that much divided by n to every call).  The first replay
+    (graph upload) is untimed."""
+
+    def __init__(self, body, n, stream):
+        import torch
+        self.torch = torch
+        self.stream = stream
+        self.e0 = torch.cuda.Event(enable_timing=True, external=True)
+        self.e1 = torch.cuda.Event(enable_timing=True, external=True)
+        self.g = torch.cuda.CUDAGraph()
+        stream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(self.g, stream=stream):
+                self.e0.record(stream)
+                for i in range(n):
+                    body(i)
+                self.e1.record(stream)
+        torch.cuda.synchronize()
+        self.replay_ms()
+
+    def replay_ms(self) -> float:
+        torch = self.torch
+        with torch.cuda.stream(self.stream):
+            self.g.replay()
+        torch.cuda.synchronize()
+        return self.e0.elapsed_time(self.e1)
+
+
 def time_graph(runner: DeviceRunner, steps: int, warmup: int, dist_barrier):
     """Capture exactly `steps` calls in one CUDA graph; time one replay."""
     torch = runner.torch
     for i in range(warmup):
         runner.step(i)
     torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    stream = torch.cuda.Stream()
-    stream.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(stream):
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(steps):
-                runner.step(i)
-    torch.cuda.synchronize()
-    g.replay()                      # untimed replay: graph upload
-    torch.cuda.synchronize()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
+    tg = TimedGraph(runner.step, steps, torch.cuda.Stream())
     dist_barrier()
     torch.cuda.synchronize()
     t0 = time.perf_counter()
-    with torch.cuda.stream(stream):
-        ev0.record(stream)
-        g.replay()
-        ev1.record(stream)
-    torch.cuda.synchronize()
+    ms = tg.replay_ms()
     t1 = time.perf_counter()
     dist_barrier()
-    ms = ev0.elapsed_time(ev1)
-    del g
+    del tg
     return ms, t0, t1
 
 
@@ -545,27 +563,9 @@ def torch_conv_graph_us(r, per_batch, batches):
         for i in range(3):
             call(i)
         torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        st = torch.cuda.Stream()
-        st.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(st):
-            with torch.cuda.graph(g, stream=st):
-                for i in range(per_batch):
-                    call(i)
-        torch.cuda.synchronize()
-        g.replay()
-        torch.cuda.synchronize()
-        us = []
-        for b in range(batches):
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            with torch.cuda.stream(st):
-                e0.record(st)
-                g.replay()
-                e1.record(st)
-            torch.cuda.synchronize()
-            us.append(e0.elapsed_time(e1) * 1e3 / per_batch)
-        del g
+        tg = TimedGraph(call, per_batch, torch.cuda.Stream())
+        us = [tg.replay_ms() * 1e3 / per_batch for b in range(batches)]
+        del tg
         return statistics.mean(us)
     finally:
         torch.backends.cudnn.benchmark, torch.backends.cudnn.allow_tf32 = prev
@@ -591,27 +591,9 @@ def write_records(args, gc, device, l2, hbm_peak, meas, batches=10, per_batch=30
         for i in range(3):
             r.step(i)
         torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        st = torch.cuda.Stream()
-        st.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(st):
-            with torch.cuda.graph(g, stream=st):
-                for i in range(per_batch):
-                    r.step(i)
-        torch.cuda.synchronize()
-        g.replay()
-        torch.cuda.synchronize()
-        graph_us = []
-        for b in range(batches):
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            with torch.cuda.stream(st):
-                e0.record(st)
-                g.replay()
-                e1.record(st)
-            torch.cuda.synchronize()
-            graph_us.append(e0.elapsed_time(e1) * 1e3 / per_batch)
-        del g
+        tg = TimedGraph(r.step, per_batch, torch.cuda.Stream())
+        graph_us = [tg.replay_ms() * 1e3 / per_batch for b in range(batches)]
+        del tg
         sync_us = []
         for b in range(batches):
             lat = []
@@ -705,26 +687,9 @@ def write_dispatch_table(args, gc, device, l2, batches=3, per_batch=20):
                 for i in range(3):
                     r.step(i)
                 torch.cuda.synchronize()
-                g = torch.cuda.CUDAGraph()
-                st = torch.cuda.Stream()
-                st.wait_stream(torch.cuda.current_stream())
-                with torch.cuda.stream(st):
-                    with torch.cuda.graph(g, stream=st):
-                        for i in range(per_batch):
-                            r.step(i)
-                torch.cuda.synchronize()
-                g.replay()
-                torch.cuda.synchronize()
-                t = []
-                for b in range(batches):
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    with torch.cuda.stream(st):
-                        e0.record(st)
-                        g.replay()
-                        e1.record(st)
-                    torch.cuda.synchronize()
-                    t.append(e0.elapsed_time(e1) * 1e3 / per_batch)
-                del g
+                tg = TimedGraph(r.step, per_batch, torch.cuda.Stream())
+                t = [tg.replay_ms() * 1e3 / per_batch for b in range(batches)]
+                del tg
                 us[name] = round(statistics.mean(t), 3)
             finally:
                 gc.force_kernel("auto")
@@ -862,7 +827,7 @@ def main():
         "config": dict(wk.config(), **{
             "l2": f"rotating pool of {runner.n_sets} buffer sets, {runner.pool_bytes / 2**20:.0f} MiB "
                   f"(L2 {l2 / 2**20:.0f} MiB)",
-            "timing": "CUDA graph of exactly K calls, device events",
+            "timing": "CUDA graph of exactly K calls between two event record nodes captured in the graph",
             "parallelism": f"replicas x{world} (batch shards, no collective)",
             "kernel_family": args.force_kernel}),
         "gflops": round(gflops, 2),
@@ -1051,21 +1016,10 @@ def measure_block(device, steps, warmup):
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
             fwd()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=s):
-                for _ in range(steps):
-                    fwd()
-        torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
-        g.replay()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        g.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        graph_us = e0.elapsed_time(e1) * 1e3 / steps
-        del g
+        tg = TimedGraph(lambda i: fwd(), steps, s)
+        graph_us = tg.replay_ms() * 1e3 / steps
+        del tg
         n_sync = max(20, steps // 2)
         t0 = time.perf_counter()
         for _ in range(n_sync):
