@@ -227,8 +227,11 @@ GCONV_API gconv_status_t gconv_force_kernel(const char *name);
 
 /* Status of the bounded waits inside the kernels since the last query:
  * GCONV_ERR_TIMEOUT when a kernel gave up waiting for its own asynchronous
- * copies (its outputs for that tile were not written), GCONV_OK otherwise.
- * Reading clears the flag.  Synchronises with the current device. */
+ * copies, GCONV_OK otherwise.  After a timeout every output of the calls
+ * made since the last query is invalid, not only the tile that gave up: an
+ * aborted CTA skips its remaining tiles, and in the fused chain a missing or
+ * partial GroupNorm partial spoils the statistics of its whole (image,
+ * group).  Reading clears the flag.  Synchronises with the current device. */
 GCONV_API gconv_status_t gconv_device_error_status(void);
 
 /* The same status after the work queued on `stream` so far has finished:
