@@ -648,7 +648,7 @@ bool finish_plan(const Shape &s, bool chain, int gn_groups, const float *x, floa
     if (pl.stream) {
         // one box per work item: 4*tpc columns x IHt rows x GB*cpg planes
         if (cached_x_tensor_map(&tm, x, (long long)s.N * s.C, s.H, s.W, p.pitch, p.IHt, p.GB * s.cpg)) return true;
-        // a map the driver rejects: the blocked kernel with cp.async staging
+        // a map the CUDA driver rejects: the blocked kernel with cp.async staging
         DirectPlan again;
         if (!plan_direct(s, chain, gn_groups, pl.geom, false, again)) return false;
         again.stream = 0;
