@@ -93,7 +93,7 @@ struct alignas(64) TensorMap {
 
 // Encode a 3-D tensor map over x viewed as [N*C][H][W] with a box of
 // box_w x box_h x 1 elements (zero fill out of bounds).  Returns false when
-// the CUDA driver entry point is unavailable or rejects the map.
+// the driver entry point is unavailable or rejects the map.
 bool make_x_tensor_map(TensorMap *tm, const float *x, long long planes, int H, int W, int box_w, int box_h,
                        int box_planes = 1);
 
