@@ -39,3 +39,18 @@ def test_sweep80_shapes():
     assert len({s.cpg for s in shapes}) == 4
     saved = json.load(open(os.path.join(os.path.dirname(wl.__file__), "sweep80.json")))
     assert [list(x) for x in saved["shapes"]] == [[s.N, s.C, s.cpg, s.H] for s in shapes]
+
+
+def test_stored_traffic_matches_kernel_sources():
+    """The DRAM traffic the benchmark reports (`roofline.traffic`) comes from
+    committed ncu captures keyed to a hash of the kernel sources; after a
+    kernel change the figure is withheld until it is captured again.  Fails
+    when a page workload's stored figure no longer matches the sources."""
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    if root not in sys.path:
+        sys.path.insert(0, root)
+    import bench
+    for name in ("depthwise", "dense_5x9", "fused_chain"):
+        t = bench.stored_traffic(name)
+        assert t is not None and t > 0, f"{name}: stored traffic missing or captured from other sources"
