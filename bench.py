@@ -911,6 +911,9 @@ def measure_config(name, gc, device, l2, hbm_peak, meas, barrier, args, rank, wo
                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
            "sync_api_us": round(time_sync_api(r, k), 2)}
     del r
+    # DRAM bytes per call from the committed ncu capture of this workload (all
+    # of the call's launches), when it matches the current kernel sources
+    out["roofline"]["traffic"] = stored_traffic(name)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gbs, desc, thr = cpu_oracle_rate(wk, max(1.0, args.cpu_budget / 4))
         gbs1, _, _ = cpu_oracle_rate(wk, max(0.5, args.cpu_budget / 8), threads=1)
