@@ -194,6 +194,8 @@ int main() {
         CHECK(p.b_resident == (slices <= p.sb ? 1 : 0), "weight residency");
         CHECK(p.AR == p.TH + (p.R - 1) * p.dil, "staged rows");
         CHECK(2 * p.TH * p.kpg <= p.tmem_cols && p.tmem_cols <= 512, "tmem columns");
+        if (c.chain && c.N == 128)   // the chain workload's measured plan: 3 tap rows folded, 7-row tiles
+            CHECK(p.RF == 3 && p.TH == 7 && p.sa == 2, "chain plan RF %d TH %d sa %d", p.RF, p.TH, p.sa);
         printf("  igemm %3d %3d %4d %4d %3d %dx%d g%-3d chain%d: NT=%d TH=%d RF=%d RC=%d bs=%d sa=%d sb=%d smem=%zu\n",
                c.N, c.C, c.H, c.W, c.K, c.R, c.S, c.g, c.chain ? 1 : 0, p.kpg, p.TH, p.RF, p.RC, p.bs, p.sa, p.sb,
                pl.smem);
